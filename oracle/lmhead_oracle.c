@@ -1,0 +1,203 @@
+/*
+ * CPU oracle for the LM-head logits projection -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the tests, the smoke check and the benchmark's CPU-baseline leg may load or call
+ * this file. The product path (the CUDA library) never does, and the two share no code.
+ *
+ * What is computed, written out as the plain definition, in double precision:
+ *
+ *   S[r, v]  = sum over k = 0 .. H-1, ascending, of dec(hidden[r, k]) * dec(W[v, k])
+ *   fp32 head:   logits[r, v] = RN_fp32( alpha * S[r, v] )
+ *   NVFP4 head:  W[v, k] = e2m1(code[v, k]) * e4m3(scale[v, k / 16]) * g
+ *                logits[r, v] = RN_bf16( alpha * S[r, v] )          (one rounding, from double)
+ *
+ * Sources (the pages this library follows):
+ *  - "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)", sections
+ *    "Purpose" and "muP is folded into the fp32 GEMM (not a bypass)": out = alpha * (hidden @ w.t())
+ *    with alpha = 1/mup, bf16 inputs accumulated into fp32 without an fp32 weight copy, fp32 output.
+ *  - "FP32 LM head skip FP32 cast" (SGLang PR #32370 summary), sections on function/motivation and
+ *    the implementation breakdown: torch.mm(hidden, W.T, out_dtype=float32), a bf16 x bf16 -> fp32
+ *    product with an fp32 accumulator.
+ *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head at its declared
+ *    W4A16 precision (16-bit activations, never cast to E4M3), bf16 logits[rows, vocab], row-major
+ *    layouts (row offsets done*h*2 and done*v*2 bytes), values independent of the row count.
+ *
+ * Readings where the pages are silent (the NVFP4 layout is not printed anywhere):
+ *  - bf16 decode: the 16 bits are the top half of an IEEE binary32.
+ *  - E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa; exponent 0 is subnormal
+ *    (value 0.5 * m). Element 2j of a row is the LOW nibble of byte j, element 2j+1 the high one.
+ *  - E4M3 (the "fn" variant): bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa, no
+ *    infinities, 0x7F / 0xFF are NaN, exponent 0 is subnormal (m * 2^-9).
+ *  - Block scales are a plain row-major [V, H/16] byte array; scale j of row v covers k in
+ *    [16j, 16j+16). g is the per-tensor decode multiplier (w = q * s * g).
+ *  - Rounding is IEEE round-to-nearest-even, done once from double.
+ *
+ * Why double is exact enough: a bf16 x bf16 product has at most 16 significant bits and an
+ * e2m1 * e4m3 * g * bf16 product at most 2+4+24+8 = 38, so every product is exact in double;
+ * the double sum's error is below H * 2^-53 * sum|p|, far inside any fp32 tolerance.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "lmhead_oracle.h"
+
+/* ---------------------------------------------------------------- element decoders */
+
+double oracle_bf16_value(uint16_t bits) {
+  /* bf16 is the upper half of a binary32: widen, reinterpret, convert (all exact). */
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+double oracle_e2m1_value(uint8_t code) {
+  int sign = (code >> 3) & 1;
+  int expo = (code >> 1) & 3;
+  int mant = code & 1;
+  double mag;
+  if (expo == 0) {
+    mag = 0.5 * (double)mant; /* subnormal: 0 or 0.5 */
+  } else {
+    mag = ldexp(1.0 + 0.5 * (double)mant, expo - 1);
+  }
+  return sign ? -mag : mag;
+}
+
+double oracle_e4m3_value(uint8_t code) {
+  int sign = (code >> 7) & 1;
+  int expo = (code >> 3) & 15;
+  int mant = code & 7;
+  double mag;
+  if (expo == 15 && mant == 7) return NAN; /* the only NaN encodings: 0x7F, 0xFF */
+  if (expo == 0) {
+    mag = ldexp((double)mant, -9); /* subnormal: (m/8) * 2^-6 */
+  } else {
+    mag = ldexp(1.0 + (double)mant / 8.0, expo - 7);
+  }
+  return sign ? -mag : mag;
+}
+
+/* ---------------------------------------------------------------- one rounding from double */
+
+float oracle_round_f32(double x) {
+  /* C's double -> float conversion is IEEE round-to-nearest-even in the default mode. */
+  return (float)x;
+}
+
+uint16_t oracle_round_bf16(double x) {
+  /* Direct double -> bf16 round-to-nearest-even (never via float, which would round twice). */
+  uint16_t sign = signbit(x) ? 0x8000u : 0u;
+  double a = fabs(x);
+  if (isnan(x)) return (uint16_t)(sign | 0x7FC0u);
+  /* Largest finite bf16 is (2 - 2^-7) * 2^127; the halfway point to 2^128 and beyond rounds
+   * to infinity (the tie goes to the even neighbour, which is 2^128). */
+  if (a >= ldexp(2.0 - ldexp(1.0, -8), 127)) return (uint16_t)(sign | 0x7F80u);
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2); /* a in [2^(e2-1), 2^e2) */
+  int e = e2 - 1;          /* a in [2^e, 2^(e+1)) */
+  if (e < -126) e = -126;  /* below the normal range the spacing stays 2^-133 */
+  double ulp = ldexp(1.0, e - 7);
+  double q = a / ulp;      /* exact: division by a power of two */
+  double n = nearbyint(q); /* ties to even in the default rounding mode */
+  double r = n * ulp;      /* a bf16 value, exactly representable as float */
+  float rf = (float)r;
+  uint32_t u;
+  memcpy(&u, &rf, sizeof u);
+  return (uint16_t)(sign | (uint16_t)(u >> 16));
+}
+
+/* ---------------------------------------------------------------- the head, fp32 output */
+
+int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
+                           int64_t V, float alpha, float* logits, double* abs_sum, int threads) {
+  if (rows < 0 || H <= 0 || V <= 0) return 1;
+  if (rows == 0) return 0;
+  if (!hidden || !W || !logits) return 1;
+  const double a = (double)alpha;
+  /* hidden decoded once: hd[r * H + k] = dec(hidden[r, k]) */
+  double* hd = (double*)malloc((size_t)rows * (size_t)H * sizeof(double));
+  if (!hd) return 2;
+  for (int64_t i = 0; i < rows * H; ++i) hd[i] = oracle_bf16_value(hidden[i]);
+  int failed = 0;
+#pragma omp parallel num_threads(threads > 0 ? threads : 1)
+  {
+    double* wv = (double*)malloc((size_t)H * sizeof(double));
+    if (!wv) {
+#pragma omp atomic write
+      failed = 1;
+    }
+#pragma omp for schedule(static)
+    for (int64_t v = 0; v < V; ++v) {
+      if (!wv) continue;
+      for (int64_t k = 0; k < H; ++k) wv[k] = oracle_bf16_value(W[v * H + k]);
+      for (int64_t r = 0; r < rows; ++r) {
+        const double* h = hd + r * H;
+        double s = 0.0, sa = 0.0;
+        for (int64_t k = 0; k < H; ++k) {
+          double p = h[k] * wv[k];
+          s += p;
+          sa += fabs(p);
+        }
+        logits[r * V + v] = oracle_round_f32(a * s);
+        if (abs_sum) abs_sum[r * V + v] = fabs(a) * sa;
+      }
+    }
+    free(wv);
+  }
+  free(hd);
+  return failed ? 2 : 0;
+}
+
+/* ---------------------------------------------------------------- the NVFP4 W4A16 head */
+
+double oracle_nvfp4_weight(const uint8_t* packed, const uint8_t* scales, float g, int64_t H,
+                           int64_t v, int64_t k) {
+  uint8_t byte = packed[v * (H / 2) + k / 2];
+  uint8_t code = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0x0F);
+  uint8_t sc = scales[v * (H / 16) + k / 16];
+  return oracle_e2m1_value(code) * oracle_e4m3_value(sc) * (double)g;
+}
+
+int oracle_logits_w4a16_nvfp4(const uint16_t* hidden, int64_t rows, int64_t H,
+                              const uint8_t* packed, const uint8_t* scales, float g, int64_t V,
+                              float alpha, uint16_t* logits, double* abs_sum, int threads) {
+  if (rows < 0 || H <= 0 || V <= 0 || (H % 16) != 0) return 1;
+  if (rows == 0) return 0;
+  if (!hidden || !packed || !scales || !logits) return 1;
+  const double a = (double)alpha;
+  double* hd = (double*)malloc((size_t)rows * (size_t)H * sizeof(double));
+  if (!hd) return 2;
+  for (int64_t i = 0; i < rows * H; ++i) hd[i] = oracle_bf16_value(hidden[i]);
+  int failed = 0;
+#pragma omp parallel num_threads(threads > 0 ? threads : 1)
+  {
+    double* wv = (double*)malloc((size_t)H * sizeof(double));
+    if (!wv) {
+#pragma omp atomic write
+      failed = 1;
+    }
+#pragma omp for schedule(static)
+    for (int64_t v = 0; v < V; ++v) {
+      if (!wv) continue;
+      for (int64_t k = 0; k < H; ++k) wv[k] = oracle_nvfp4_weight(packed, scales, g, H, v, k);
+      for (int64_t r = 0; r < rows; ++r) {
+        const double* h = hd + r * H;
+        double s = 0.0, sa = 0.0;
+        for (int64_t k = 0; k < H; ++k) {
+          double p = h[k] * wv[k];
+          s += p;
+          sa += fabs(p);
+        }
+        logits[r * V + v] = oracle_round_bf16(a * s);
+        if (abs_sum) abs_sum[r * V + v] = fabs(a) * sa;
+      }
+    }
+    free(wv);
+  }
+  free(hd);
+  return failed ? 2 : 0;
+}

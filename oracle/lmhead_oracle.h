@@ -1,0 +1,50 @@
+/*
+ * CPU oracle for the LM-head logits projection -- TEST INFRASTRUCTURE ONLY (see
+ * lmhead_oracle.c for the definition it computes and the pages it follows). Nothing in the
+ * CUDA library includes this header.
+ */
+#ifndef LMHEAD_ORACLE_H
+#define LMHEAD_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exact value of one bf16 / E2M1 (low 4 bits of code) / E4M3fn encoding. */
+double oracle_bf16_value(uint16_t bits);
+double oracle_e2m1_value(uint8_t code);
+double oracle_e4m3_value(uint8_t code);
+
+/* One IEEE round-to-nearest-even from double. */
+float oracle_round_f32(double x);
+uint16_t oracle_round_bf16(double x);
+
+/* Decoded NVFP4 weight W[v, k] = e2m1 * e4m3 * g, exact in double. */
+double oracle_nvfp4_weight(const uint8_t* packed, const uint8_t* scales, float g, int64_t H,
+                           int64_t v, int64_t k);
+
+/*
+ * logits[r, v] = RN_fp32(alpha * sum_k hidden[r, k] * W[v, k]), all host arrays, row-major:
+ * hidden [rows, H] bf16 bits, W [V, H] bf16 bits, logits [rows, V] fp32. If abs_sum is not
+ * NULL it receives |alpha| * sum_k |hidden[r, k] * W[v, k]| (the error-bound scale).
+ * Returns 0 on success, 1 on bad arguments, 2 when host memory runs out.
+ */
+int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
+                           int64_t V, float alpha, float* logits, double* abs_sum, int threads);
+
+/*
+ * logits[r, v] = RN_bf16(alpha * sum_k hidden[r, k] * e2m1(code[v, k]) * e4m3(scale[v, k/16]) * g)
+ * packed [V, H/2] (element 2j = low nibble of byte j), scales [V, H/16] E4M3 bytes,
+ * logits [rows, V] bf16 bits. H must be a multiple of 16.
+ */
+int oracle_logits_w4a16_nvfp4(const uint16_t* hidden, int64_t rows, int64_t H,
+                              const uint8_t* packed, const uint8_t* scales, float g, int64_t V,
+                              float alpha, uint16_t* logits, double* abs_sum, int threads);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

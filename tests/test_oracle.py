@@ -1,0 +1,349 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself -- a library
+conversion, a closed form, exact integer arithmetic or a brute-force search -- so that a dropped
+term, a wrong sign or index, or a transposed operand in the oracle fails here.
+
+Formats and rules pinned: bf16 and E4M3fn decode (torch's own dtypes), E2M1 decode (the NVFP4
+value set +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}), one round-to-nearest-even from double to fp32 (numpy's
+cast) and to bf16 (brute-force nearest search), and the head
+    logits = RN(alpha * hidden @ W^T)
+from "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)" ("Purpose";
+"muP is folded into the fp32 GEMM") and lm_head_nvfp4_rows.rs (module doc).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp32_accumulate_lm_b200 import synth
+
+
+def bf16_bits_of_f32(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits through torch (round-to-nearest-even: a library routine)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def all_bf16_values() -> np.ndarray:
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    return torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).float().double().numpy()
+
+
+# ---------------------------------------------------------------- element decoders
+
+def test_bf16_decode_all_codes_match_torch_and_ieee_fields():
+    lib_vals = all_bf16_values()
+    for code in range(65536):
+        got = oracle.bf16_value(code)
+        want = lib_vals[code]
+        if math.isnan(want):
+            assert math.isnan(got), hex(code)
+            continue
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), hex(code)
+    # IEEE field reading on a few codes, independent of the bit-shift trick
+    for code in [0x0001, 0x007F, 0x0080, 0x3F80, 0x4049, 0xC2F7, 0x7F7F, 0x8001]:
+        s, e, m = code >> 15, (code >> 7) & 0xFF, code & 0x7F
+        mag = (m / 128.0) * 2.0 ** -126 if e == 0 else (1 + m / 128.0) * 2.0 ** (e - 127)
+        assert oracle.bf16_value(code) == (-mag if s else mag)
+    assert math.isinf(oracle.bf16_value(0x7F80)) and oracle.bf16_value(0xFF80) < 0
+
+
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_all_codes_match_value_set():
+    for code in range(16):
+        want = E2M1_TABLE[code & 7] * (-1.0 if code & 8 else 1.0)
+        got = oracle.e2m1_value(code)
+        assert got == want, code
+        assert math.copysign(1, got) == (-1 if code & 8 else 1), code  # 0x8 is -0
+
+
+def test_e2m1_decode_matches_torch_float4_where_supported():
+    packed = torch.arange(256, dtype=torch.uint8).view(torch.float4_e2m1fn_x2)
+    try:
+        vals = packed.to(torch.float32)
+    except Exception:
+        pytest.skip("this torch build cannot convert float4_e2m1fn_x2")
+    vals = vals.numpy().reshape(-1)
+    if vals.size != 512:
+        pytest.skip("float4_e2m1fn_x2 conversion does not unpack to two values per byte")
+    for byte in range(256):
+        lo, hi = oracle.e2m1_value(byte & 0xF), oracle.e2m1_value(byte >> 4)
+        assert {vals[2 * byte], vals[2 * byte + 1]} <= {lo, hi} | {-lo, -hi}
+
+
+def test_e4m3_decode_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for code in range(256):
+        got = oracle.e4m3_value(code)
+        if math.isnan(lib[code]):
+            assert math.isnan(got), hex(code)
+            assert code in (0x7F, 0xFF)
+        else:
+            assert got == lib[code], hex(code)
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6
+
+
+def test_e2m1_times_e4m3_is_exact_in_bf16():
+    """Every E2M1 x E4M3 product (all 8 x 127 non-negative, non-NaN pairs) round-trips through
+    bf16 unchanged -- the reason a dequantised NVFP4 weight tile can be held in bf16 exactly."""
+    for q in range(8):
+        for s in range(0x7F):
+            p = oracle.e2m1_value(q) * oracle.e4m3_value(s)
+            assert oracle.bf16_value(oracle.round_bf16(p)) == p
+            assert bf16_bits_of_f32(np.array([p], np.float32))[0] == oracle.round_bf16(p)
+
+
+# ---------------------------------------------------------------- rounding
+
+def _bf16_nearest_bruteforce(x: float, finite_sorted: np.ndarray, codes_sorted: np.ndarray) -> int:
+    """Nearest finite bf16 by search, ties to the even code, overflow to infinity."""
+    maxf = finite_sorted[-1]
+    if abs(x) >= maxf + (2.0 ** 128 - maxf) / 2:
+        return 0x7F80 | (0x8000 if x < 0 else 0)
+    i = int(np.searchsorted(finite_sorted, x))
+    cands = [j for j in (i - 1, i) if 0 <= j < len(finite_sorted)]
+    best = min(abs(finite_sorted[j] - x) for j in cands)
+    ties = [int(codes_sorted[j]) for j in cands if abs(finite_sorted[j] - x) == best]
+    if len(ties) == 1:
+        return ties[0]
+    even = [c for c in ties if c % 2 == 0]
+    return even[0]
+
+
+def test_round_bf16_matches_bruteforce_nearest_even():
+    vals = all_bf16_values()
+    codes = np.arange(65536)
+    finite = np.isfinite(vals) & ~((vals == 0) & (codes >= 0x8000))  # drop NaN/inf and -0
+    order = np.argsort(vals[finite], kind="stable")
+    fs, cs = vals[finite][order], codes[finite][order]
+    rng = np.random.default_rng(7)
+    xs = list(rng.standard_normal(2000) * 10.0 ** rng.integers(-45, 39, 2000))
+    # exact midpoints between neighbours (ties), subnormal region, overflow boundary
+    for c in [0x0001, 0x0002, 0x3F80, 0x3F81, 0x4000, 0x7F7E, 0x007F, 0x0080]:
+        a, b = oracle.bf16_value(c), oracle.bf16_value(c + 1)
+        xs += [(a + b) / 2, -(a + b) / 2, np.nextafter((a + b) / 2, 0), np.nextafter((a + b) / 2, 1e300)]
+    maxf = oracle.bf16_value(0x7F7F)
+    xs += [maxf, np.nextafter(maxf + 2.0 ** 119, 0), maxf + 2.0 ** 119, 1e300, -1e300, 1e-300]
+    for x in xs:
+        x = float(x)
+        got = oracle.round_bf16(x)
+        want = _bf16_nearest_bruteforce(x, fs, cs)
+        if x != 0 and abs(x) < oracle.bf16_value(0x0001) / 2 + 1e-320:  # rounds to a signed zero
+            assert got & 0x7FFF == want & 0x7FFF
+        else:
+            assert got == want, (x, hex(got), hex(want))
+    assert oracle.round_bf16(0.0) == 0x0000 and oracle.round_bf16(-0.0) == 0x8000
+    assert oracle.round_bf16(float("inf")) == 0x7F80
+    assert (oracle.round_bf16(float("nan")) & 0x7FFF) > 0x7F80
+
+
+def test_round_bf16_matches_torch_on_float32_inputs():
+    """Where the double is already a float32, torch's float32 -> bf16 RNE is one rounding."""
+    rng = np.random.default_rng(11)
+    xs = (rng.standard_normal(5000) * 10.0 ** rng.integers(-30, 30, 5000)).astype(np.float32)
+    lib = bf16_bits_of_f32(xs)
+    for x, want in zip(xs, lib):
+        assert oracle.round_bf16(float(x)) == int(want)
+
+
+def test_round_f32_matches_numpy_cast():
+    rng = np.random.default_rng(3)
+    xs = rng.standard_normal(5000) * 10.0 ** rng.integers(-40, 40, 5000)
+    with np.errstate(over="ignore"):
+        for x in xs:
+            assert np.float32(oracle.round_f32(float(x))) == np.float32(x)
+
+
+# ---------------------------------------------------------------- the fp32 head
+
+def test_hand_computed_dot_products():
+    # H = 16, small integers: closed forms written out
+    H = 16
+    h = np.zeros((2, H), np.float32)
+    w = np.zeros((3, H), np.float32)
+    h[0] = 1.0                         # row of ones
+    h[1] = np.arange(H)                # 0..15
+    w[0] = np.arange(H)                # sum k = 120 ; sum k^2 = 1240
+    w[1] = -2.0                        # -2 * 16 = -32 ; -2 * 120 = -240
+    w[2, 3] = 0.5                      # picks element 3: 0.5 ; 1.5
+    out, absum = oracle.logits_bf16_f32(bf16_bits_of_f32(h), bf16_bits_of_f32(w), 1.0)
+    assert out.tolist() == [[120.0, -32.0, 0.5], [1240.0, -240.0, 1.5]]
+    assert absum.tolist() == [[120.0, 32.0, 0.5], [1240.0, 240.0, 1.5]]
+    out, _ = oracle.logits_bf16_f32(bf16_bits_of_f32(h), bf16_bits_of_f32(w), 0.25)
+    assert out.tolist() == [[30.0, -8.0, 0.125], [310.0, -60.0, 0.375]]
+
+
+def test_integer_inputs_equal_exact_integer_matmul():
+    """Small-integer operands: every partial sum is an exact integer below 2^24, so the result
+    must equal int64 arithmetic bit-for-bit (any sign or index error shows up here)."""
+    rng = np.random.default_rng(5)
+    rows, H, V = 5, 96, 37
+    hi = rng.integers(-8, 9, (rows, H))
+    wi = rng.integers(-8, 9, (V, H))
+    out, _ = oracle.logits_bf16_f32(bf16_bits_of_f32(hi.astype(np.float32)),
+                                    bf16_bits_of_f32(wi.astype(np.float32)), 1.0)
+    want = (hi.astype(np.int64) @ wi.astype(np.int64).T).astype(np.float32)
+    assert np.array_equal(out, want)
+    # non-square shapes with rows != V catch a transposed operand
+    out2, _ = oracle.logits_bf16_f32(bf16_bits_of_f32(hi[:2].astype(np.float32)),
+                                     bf16_bits_of_f32(wi.astype(np.float32)), 0.5)
+    assert np.array_equal(out2, (want[:2] * 0.5).astype(np.float32))
+
+
+def test_one_hot_rows_pick_columns_of_w():
+    H, V = 256, 1024
+    w_bits = synth.weight(V, H, 0.02, synth.SEED_TINY)
+    wf = synth.bf16_bits_to_f32(w_bits).astype(np.float64)
+    ks = [0, 1, 17, 255]
+    h = np.zeros((len(ks), H), np.float32)
+    for i, k in enumerate(ks):
+        h[i, k] = 1.0
+    for alpha in (1.0, 0.25, 1.0 / 3.0):
+        out, _ = oracle.logits_bf16_f32(bf16_bits_of_f32(h), w_bits, alpha)
+        for i, k in enumerate(ks):
+            want = (np.float64(np.float32(alpha)) * wf[:, k]).astype(np.float32)
+            assert np.array_equal(out[i], want)
+
+
+def test_zero_and_identity_block_weights():
+    rows, H, V = 3, 64, 80
+    h_bits = synth.hidden(rows, H, 99)
+    hf = synth.bf16_bits_to_f32(h_bits)
+    out, _ = oracle.logits_bf16_f32(h_bits, np.zeros((V, H), np.uint16), 0.125)
+    assert np.all(out == 0) and not np.any(np.signbit(out))
+    eye = np.zeros((V, H), np.float32)
+    eye[np.arange(H), np.arange(H)] = 1.0
+    out, _ = oracle.logits_bf16_f32(h_bits, bf16_bits_of_f32(eye), 0.125)
+    assert np.array_equal(out[:, :H], (hf * np.float32(0.125)).astype(np.float32))
+    assert np.all(out[:, H:] == 0)
+
+
+def test_alpha_fold_against_separate_multiply():
+    """RN(alpha*S) vs RN(RN(S)*alpha): equal for power-of-two alpha, within one fp32 ulp else
+    (page 1's fold claim, with the double rounding a separate multiply adds)."""
+    rows, H, V = 4, 256, 1024
+    h = synth.hidden(rows, H, synth.SEED_TINY)
+    w = synth.weight(V, H, 0.02, synth.SEED_TINY)
+    base, _ = oracle.logits_bf16_f32(h, w, 1.0)
+    for alpha in (0.25, 0.125, 1.0 / 16):
+        fused, _ = oracle.logits_bf16_f32(h, w, alpha)
+        assert np.array_equal(fused, (base * np.float32(alpha)).astype(np.float32))
+    for alpha in (1.0 / 3.0, 1.0 / 6.0, 0.7):
+        fused, _ = oracle.logits_bf16_f32(h, w, alpha)
+        sep = (base * np.float32(alpha)).astype(np.float32)
+        ulp = np.spacing(np.abs(fused))
+        assert np.all(np.abs(fused.astype(np.float64) - sep) <= ulp)
+
+
+def test_matches_library_double_matmul():
+    """numpy's float64 matmul (BLAS) on the decoded operands: the same real number up to the
+    double summation order, so after one fp32 rounding the two agree to within one ulp."""
+    for rows, H, V, seed in [(4, 256, 1024, synth.SEED_TINY), (3, 2048, 512, 77)]:
+        h = synth.hidden(rows, H, seed)
+        w = synth.weight(V, H, 0.02, seed)
+        alpha = 0.25
+        out, absum = oracle.logits_bf16_f32(h, w, alpha)
+        hd = synth.bf16_bits_to_f32(h).astype(np.float64)
+        wd = synth.bf16_bits_to_f32(w).astype(np.float64)
+        ref = (np.float64(np.float32(alpha)) * (hd @ wd.T)).astype(np.float32)
+        diff = np.abs(out.astype(np.float64) - ref)
+        assert np.all(diff <= np.spacing(np.abs(ref))), diff.max()
+        assert np.mean(out == ref) > 0.99
+        assert np.allclose(absum, abs(alpha) * (np.abs(hd) @ np.abs(wd).T), rtol=1e-12)
+
+
+def test_empty_rows():
+    out, absum = oracle.logits_bf16_f32(np.zeros((0, 64), np.uint16), np.zeros((8, 64), np.uint16), 1.0)
+    assert out.shape == (0, 8) and absum.shape == (0, 8)
+
+
+# ---------------------------------------------------------------- the NVFP4 head
+
+def _dequant_with_torch(packed, scales, g):
+    """Independent dequantisation through torch's float8_e4m3fn and the NVFP4 value set."""
+    V, Hh = packed.shape
+    lo, hi = packed & 0xF, packed >> 4
+    codes = np.empty((V, 2 * Hh), np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = lo, hi
+    mags = np.array(E2M1_TABLE)[codes & 7]
+    q = np.where(codes & 8, -mags, mags)
+    s = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).double().numpy()
+    return q * np.repeat(s, 16, axis=1) * np.float64(np.float32(g))
+
+
+def test_nvfp4_weight_decode_matches_torch_dequant():
+    V, H = 40, 64
+    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 123)
+    ref = _dequant_with_torch(packed, scales, g)
+    for v in range(V):
+        for k in range(H):
+            assert oracle.nvfp4_weight(packed, scales, g, v, k) == ref[v, k]
+
+
+def test_nvfp4_head_one_hot_and_integer_cases():
+    V, H = 48, 64
+    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 321)
+    wq = _dequant_with_torch(packed, scales, g)
+    ks = [0, 1, 15, 16, 63]
+    h = np.zeros((len(ks), H), np.float32)
+    for i, k in enumerate(ks):
+        h[i, k] = 1.0
+    out, _ = oracle.logits_w4a16_nvfp4(bf16_bits_of_f32(h), packed, scales, g, 0.5)
+    for i, k in enumerate(ks):
+        want = np.array([oracle.round_bf16(0.5 * wq[v, k]) for v in range(V)], np.uint16)
+        assert np.array_equal(out[i], want)
+        # power-of-two alpha: the bf16 of the exact product, via torch's float32 path (exact here)
+        assert np.array_equal(out[i], bf16_bits_of_f32((0.5 * wq[:, k]).astype(np.float32)))
+    # integer codes, unit scale (E4M3 0x38 = 1.0), g = 1: exact small sums
+    rng = np.random.default_rng(9)
+    codes = rng.integers(0, 16, (V, H)).astype(np.uint8)
+    pk = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    sc = np.full((V, H // 16), 0x38, np.uint8)
+    hi = rng.integers(-4, 5, (3, H)).astype(np.float32)
+    out, _ = oracle.logits_w4a16_nvfp4(bf16_bits_of_f32(hi), pk, sc, 1.0, 1.0)
+    qv = np.array(E2M1_TABLE)[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    exact = hi.astype(np.float64) @ qv.T  # sums of multiples of 0.5 below 2^8: exact
+    assert np.array_equal(out, bf16_bits_of_f32(exact.astype(np.float32)))
+
+
+def test_nvfp4_head_matches_library_double_matmul():
+    rows, H, V = 5, 256, 300
+    h = synth.hidden(rows, H, 31)
+    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 32)
+    out, _ = oracle.logits_w4a16_nvfp4(h, packed, scales, g, 0.125)
+    wq = _dequant_with_torch(packed, scales, g)
+    ref = 0.125 * (synth.bf16_bits_to_f32(h).astype(np.float64) @ wq.T)
+    got = synth.bf16_bits_to_f32(out).astype(np.float64)
+    # one bf16 rounding of the same real number (BLAS sums in another order): within 1 ulp
+    assert np.all(np.abs(got - ref) <= np.spacing(np.abs(ref).astype(np.float32)) * 2 ** 16)
+    assert np.mean(bf16_bits_of_f32(ref.astype(np.float32)) == out) > 0.98
+
+
+def test_nvfp4_quantiser_round_trip_bounds():
+    """The test-weight generator: decoded NVFP4 is within half an E2M1 step (relative to the block
+    scale) of the bf16 weights it came from, and block maxima land on +-6 * s * g within E4M3
+    rounding."""
+    V, H = 64, 256
+    w_bits = synth.weight(V, H, 0.02, 44)
+    wf = synth.bf16_bits_to_f32(w_bits).astype(np.float64)
+    packed, scales, g = synth.nvfp4_quantize(w_bits)
+    wq = _dequant_with_torch(packed, scales, g)
+    s = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).double().numpy()
+    step = np.repeat(s, 16, axis=1) * g  # the value of one E2M1 unit in this block
+    # largest gap in the E2M1 grid is 2 (between 4 and 6): error <= 1 unit, and <= 0.25 near 0
+    assert np.all(np.abs(wq - wf) <= 1.0 * step + 1e-30)
+    assert np.max(np.abs(wq)) <= 6 * 448 * g * (1 + 1e-12)
+
+
+def test_synth_e4m3_table_matches_torch():
+    """The generator's E4M3 encode table is ascending and equals torch's decode."""
+    vals = synth._E4M3_POS_VALUES
+    lib = torch.from_numpy(synth._E4M3_POS_CODES.copy()).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(vals, lib)
+    assert np.all(np.diff(vals) > 0)
