@@ -1,0 +1,171 @@
+"""B200 (sm_100a) LM-head logits projection: Python binding of the C ABI in include/lmhead.h.
+
+    logits[rows, V] = alpha * (hidden[rows, H] @ W[V, H]^T)
+
+``logits_bf16_f32`` takes bf16 operands and returns fp32 logits (fp32 accumulation, alpha folded
+into the epilogue -- "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)",
+"muP is folded into the fp32 GEMM"); ``logits_w4a16_nvfp4`` is the W4A16 NVFP4 head with bf16
+logits (lm_head_nvfp4_rows.rs, lm_head_nvfp4_rows_run).
+
+This module only marshals arguments: every step of the computation runs in the CUDA library
+``liblmhead.so`` built in-tree by ``fp32_accumulate_lm_b200._build``. If that library is
+missing or fails to load, every call raises; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_w4a16_nvfp4",
+    "lmhead_logits_bf16_f32", "lmhead_logits_w4a16_nvfp4", "status_string", "device_status",
+    "version", "set_fault_injection", "STATUS",
+]
+
+STATUS = {
+    0: "LMHEAD_OK", 1: "LMHEAD_ERR_NULL", 2: "LMHEAD_ERR_SHAPE", 3: "LMHEAD_ERR_ALIGN",
+    4: "LMHEAD_ERR_ARCH", 5: "LMHEAD_ERR_LAUNCH", 6: "LMHEAD_ERR_TIMEOUT", 7: "LMHEAD_ERR_ALIAS",
+}
+LMHEAD_OK = 0
+LMHEAD_ERR_TIMEOUT = 6
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblmhead.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class LmheadError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load liblmhead.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m fp32_accumulate_lm_b200._build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+        lib.lmhead_logits_bf16_f32.argtypes = [vp, i64, i64, vp, i64, f32, vp, vp]
+        lib.lmhead_logits_bf16_f32.restype = i32
+        lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
+        lib.lmhead_logits_w4a16_nvfp4.restype = i32
+        lib.lmhead_status_string.argtypes = [i32]
+        lib.lmhead_status_string.restype = ctypes.c_char_p
+        lib.lmhead_device_status.argtypes = [i32]
+        lib.lmhead_device_status.restype = i32
+        lib.lmhead_version.argtypes = []
+        lib.lmhead_version.restype = i32
+        lib.lmhead_debug_set_fault_injection.argtypes = [i32, ctypes.c_uint64]
+        lib.lmhead_debug_set_fault_injection.restype = None
+        _lib = lib
+        return lib
+
+
+# ---------------------------------------------------------------- raw C-ABI (integers in, status out)
+
+def lmhead_logits_bf16_f32(hidden_ptr: int, rows: int, H: int, w_ptr: int, V: int, alpha: float,
+                           logits_ptr: int, stream: int = 0) -> int:
+    return load_library().lmhead_logits_bf16_f32(hidden_ptr, rows, H, w_ptr, V, alpha,
+                                                  logits_ptr, stream)
+
+
+def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
+                              scales_ptr: int, w_global_scale: float, V: int, alpha: float,
+                              logits_ptr: int, stream: int = 0) -> int:
+    return load_library().lmhead_logits_w4a16_nvfp4(hidden_ptr, rows, H, packed_ptr, scales_ptr,
+                                                     w_global_scale, V, alpha, logits_ptr, stream)
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().lmhead_status_string(int(status)).decode()
+    except RuntimeError:
+        return STATUS.get(status, "unknown status")
+
+
+def device_status(clear: bool = False) -> int:
+    """Status word of the current device (0, or LMHEAD_ERR_TIMEOUT | role << 8)."""
+    return load_library().lmhead_device_status(1 if clear else 0)
+
+
+def version() -> int:
+    return load_library().lmhead_version()
+
+
+def set_fault_injection(starve_loads: bool, wait_limit_ns: int = 0) -> None:
+    """Test-only: make launches issue no loads so their waits time out after wait_limit_ns."""
+    load_library().lmhead_debug_set_fault_injection(1 if starve_loads else 0, int(wait_limit_ns))
+
+
+# ---------------------------------------------------------------- torch-tensor convenience wrappers
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def logits_bf16_f32(hidden, W, alpha: float = 1.0, out=None, stream=None):
+    """fp32 logits[rows, V] = alpha * hidden @ W^T for bf16 CUDA tensors hidden [rows, H] and
+    W [V, H]. Runs asynchronously on ``stream`` (default: torch's current stream)."""
+    import torch
+    _check(hidden.dtype == torch.bfloat16 and W.dtype == torch.bfloat16, "bf16 operands required")
+    _check(hidden.dim() == 2 and W.dim() == 2 and hidden.shape[1] == W.shape[1], "shape mismatch")
+    _check(hidden.is_cuda and W.is_cuda, "CUDA tensors required")
+    _check(hidden.is_contiguous() and W.is_contiguous(), "contiguous tensors required")
+    rows, H = hidden.shape
+    V = W.shape[0]
+    if out is None:
+        out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
+    _check(out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (rows, V),
+           "out must be a contiguous fp32 [rows, V] tensor")
+    st = lmhead_logits_bf16_f32(hidden.data_ptr(), rows, H, W.data_ptr(), V, float(alpha),
+                                out.data_ptr(), _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logits_bf16_f32")
+    return out
+
+
+def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha: float = 1.0,
+                       out=None, stream=None):
+    """bf16 logits[rows, V] for the NVFP4 head: w_packed uint8 [V, H/2], w_scales uint8
+    (E4M3) [V, H/16], bf16 hidden [rows, H]."""
+    import torch
+    _check(hidden.dtype == torch.bfloat16, "bf16 hidden required")
+    _check(w_packed.dtype == torch.uint8 and w_scales.dtype == torch.uint8, "uint8 codes/scales")
+    rows, H = hidden.shape
+    V = w_packed.shape[0]
+    _check(tuple(w_packed.shape) == (V, H // 2) and tuple(w_scales.shape) == (V, H // 16),
+           "w_packed must be [V, H/2] and w_scales [V, H/16]")
+    _check(all(t.is_cuda and t.is_contiguous() for t in (hidden, w_packed, w_scales)),
+           "contiguous CUDA tensors required")
+    if out is None:
+        out = torch.empty((rows, V), dtype=torch.bfloat16, device=hidden.device)
+    _check(out.dtype == torch.bfloat16 and out.is_contiguous() and tuple(out.shape) == (rows, V),
+           "out must be a contiguous bf16 [rows, V] tensor")
+    st = lmhead_logits_w4a16_nvfp4(hidden.data_ptr(), rows, H, w_packed.data_ptr(),
+                                   w_scales.data_ptr(), float(w_global_scale), V, float(alpha),
+                                   out.data_ptr(), _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logits_w4a16_nvfp4")
+    return out

@@ -1,0 +1,308 @@
+// C ABI of the LM-head library (declared in include/lmhead.h): argument validation, TMA
+// descriptor set-up and the launch of one kernel per call on the caller's stream.
+//
+// The operation: logits = alpha * hidden @ W^T with bf16 inputs, fp32 accumulation and alpha in
+// the epilogue ("[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)",
+// "muP is folded into the fp32 GEMM"; "FP32 LM head skip FP32 cast", implementation breakdown),
+// and the W4A16 NVFP4 head with bf16 logits (lm_head_nvfp4_rows.rs, lm_head_nvfp4_rows_run).
+// As on that page, a call that cannot run launches nothing and reports why.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "lmhead.h"
+#include "lmhead_bf16.cuh"
+#include "lmhead_nvfp4.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+constexpr int kMaxStages = 16;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
+
+std::atomic<int> g_starve_loads{0};
+std::atomic<uint64_t> g_wait_limit_ns{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  bool probed = false;
+  bool arch_ok = false;
+  bool attrs_set = false;
+  int num_sms = 0;
+  int smem_optin = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_devices[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  });
+  return g_encode;
+}
+
+// Probe the current device once: architecture, SM count, shared-memory opt-in; raise the
+// kernels' dynamic shared-memory limit.
+int current_device(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMHEAD_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess) {
+      return LMHEAD_ERR_LAUNCH;
+    }
+    d.arch_ok = (major == 10 && minor == 0);
+    d.probed = true;
+  }
+  if (!d.arch_ok) return LMHEAD_ERR_ARCH;
+  if (!d.attrs_set) {
+    if (cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(lmh::lmhead_w4a16_nvfp4_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess) {
+      return LMHEAD_ERR_LAUNCH;
+    }
+    d.attrs_set = true;
+  }
+  *out = d;
+  return LMHEAD_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + (uintptr_t)bbytes && b0 < a0 + (uintptr_t)abytes;
+}
+
+// Row-major [outer, inner] tensor, tile box [box_outer, box_inner], 128-byte swizzle.
+int encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base,
+              int64_t inner, int64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return LMHEAD_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)(inner * elem_bytes)};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+// Packed NVFP4 codes as a [V, H/2] byte matrix, box [128 rows x 32 bytes] (one K step of 64),
+// no swizzle: the dequantisers read it as plain row-major bytes.
+int encode_nvfp4_codes(CUtensorMap* map, const void* base, int64_t row_bytes, int64_t V) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return LMHEAD_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)V};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(lmh::kBK / 2), (cuuint32_t)lmh::kBM};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+lmh::WaitCfg wait_cfg() {
+  lmh::WaitCfg w;
+  const uint64_t lim = g_wait_limit_ns.load(std::memory_order_relaxed);
+  w.limit_ns = lim ? lim : kDefaultWaitLimitNs;
+  w.starve_loads = g_starve_loads.load(std::memory_order_relaxed);
+  return w;
+}
+
+// Rows per tile: the padded row count up to 256, else 256. Every choice runs the same
+// per-element MMA chain over K, so it affects speed only, never a row's bits.
+int32_t pick_bn(int64_t rows) { return rows >= 256 ? 256 : (int32_t)((rows + 15) / 16 * 16); }
+
+uint32_t tmem_cols_for(int32_t bn) {
+  uint32_t need = 2u * (uint32_t)bn, c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
+
+constexpr int kInt32Max = 0x7fffffff;
+
+}  // namespace
+
+extern "C" {
+
+int lmhead_version(void) { return kVersion; }
+
+const char* lmhead_status_string(int status) {
+  switch (status) {
+    case LMHEAD_OK: return "ok";
+    case LMHEAD_ERR_NULL: return "a required pointer is NULL";
+    case LMHEAD_ERR_SHAPE: return "unsupported or invalid size";
+    case LMHEAD_ERR_ALIGN: return "pointer or row pitch misaligned";
+    case LMHEAD_ERR_ARCH: return "current device is not an sm_100 GPU";
+    case LMHEAD_ERR_LAUNCH: return "CUDA runtime refused a set-up call or the launch";
+    case LMHEAD_ERR_TIMEOUT: return "a kernel timed out waiting on one of its barriers";
+    case LMHEAD_ERR_ALIAS: return "output overlaps an input";
+    default: return "unknown status";
+  }
+}
+
+void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) {
+  g_starve_loads.store(starve_loads ? 1 : 0);
+  g_wait_limit_ns.store(wait_limit_ns);
+}
+
+int lmhead_device_status(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lmh::g_lmhead_status, sizeof v) != cudaSuccess)
+    return LMHEAD_ERR_LAUNCH;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(lmh::g_lmhead_status, &z, sizeof z) != cudaSuccess)
+      return LMHEAD_ERR_LAUNCH;
+  }
+  return (int)v;
+}
+
+int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const void* W, int64_t V,
+                           float alpha, float* logits, lmhead_stream_t stream) {
+  if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 8 != 0) return LMHEAD_ERR_ALIGN;
+  if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (hidden == nullptr || W == nullptr || logits == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(logits, 4)) return LMHEAD_ERR_ALIGN;
+  if (overlaps(logits, rows * V * 4, hidden, rows * H * 2) ||
+      overlaps(logits, rows * V * 4, W, V * H * 2)) {
+    return LMHEAD_ERR_ALIAS;
+  }
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+
+  lmh::Bf16HeadParams p;
+  p.rows = rows;
+  p.H = H;
+  p.V = V;
+  p.out = logits;
+  p.alpha = alpha;
+  p.bn = pick_bn(rows);
+  p.n_rtiles = (int32_t)((rows + p.bn - 1) / p.bn);
+  p.n_vtiles = (int32_t)((V + lmh::kBM - 1) / lmh::kBM);
+  const int64_t tiles = (int64_t)p.n_rtiles * p.n_vtiles;
+  if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
+  p.num_tiles = (int32_t)tiles;
+  p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
+  p.stage_bytes = (uint32_t)(lmh::kBM * lmh::kBK * 2 + p.bn * lmh::kBK * 2);
+  const int reserve = 1024 + 512;  // alignment slack + barriers
+  int stages = (dev.smem_optin - reserve) / (int)p.stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return LMHEAD_ERR_SHAPE;
+  p.stages = stages;
+  p.tmem_cols = tmem_cols_for(p.bn);
+  p.wait = wait_cfg();
+
+  CUtensorMap tmap_w, tmap_h;
+  st = encode_2d(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, H, V, lmh::kBK, lmh::kBM);
+  if (st != LMHEAD_OK) return st;
+  st = encode_2d(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H, rows, lmh::kBK,
+                 (uint32_t)p.bn);
+  if (st != LMHEAD_OK) return st;
+
+  const int grid = p.num_tiles < dev.num_sms ? p.num_tiles : dev.num_sms;
+  const size_t smem = (size_t)reserve + (size_t)stages * p.stage_bytes;
+  lmh::lmhead_bf16_f32_kernel<<<grid, lmh::kHeadThreads, smem, (cudaStream_t)stream>>>(
+      tmap_w, tmap_h, p);
+  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,
+                              const uint8_t* w_scales, float w_global_scale, int64_t V,
+                              float alpha, void* logits, lmhead_stream_t stream) {
+  if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 64 != 0) return LMHEAD_ERR_ALIGN;
+  if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (hidden == nullptr || w_packed == nullptr || w_scales == nullptr || logits == nullptr)
+    return LMHEAD_ERR_NULL;
+  if (!aligned(hidden, 16) || !aligned(w_packed, 16) || !aligned(w_scales, 4) ||
+      !aligned(logits, 2)) {
+    return LMHEAD_ERR_ALIGN;
+  }
+  const int64_t out_bytes = rows * V * 2;
+  if (overlaps(logits, out_bytes, hidden, rows * H * 2) ||
+      overlaps(logits, out_bytes, w_packed, V * H / 2) ||
+      overlaps(logits, out_bytes, w_scales, V * H / 16)) {
+    return LMHEAD_ERR_ALIAS;
+  }
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+
+  lmh::Nvfp4HeadParams p;
+  p.rows = rows;
+  p.H = H;
+  p.V = V;
+  p.out = reinterpret_cast<uint16_t*>(logits);
+  p.scales = w_scales;
+  p.alpha = alpha;
+  p.gscale = w_global_scale;
+  p.bn = pick_bn(rows);
+  p.n_rtiles = (int32_t)((rows + p.bn - 1) / p.bn);
+  p.n_vtiles = (int32_t)((V + lmh::kBM - 1) / lmh::kBM);
+  const int64_t tiles = (int64_t)p.n_rtiles * p.n_vtiles;
+  if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
+  p.num_tiles = (int32_t)tiles;
+  p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
+  p.raw_bytes = (uint32_t)(lmh::kBM * lmh::kBK / 2);        // packed nibbles of one K step
+  p.a_bytes = (uint32_t)(lmh::kBM * lmh::kBK * 2);          // dequantised bf16 tile
+  p.b_bytes = (uint32_t)(p.bn * lmh::kBK * 2);              // hidden tile
+  const int reserve = 1024 + 1024;
+  const int per_stage = (int)lmh::nvfp4_stage_bytes(p.bn);
+  int stages = (dev.smem_optin - reserve) / per_stage;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return LMHEAD_ERR_SHAPE;
+  p.stages = stages;
+  p.tmem_cols = tmem_cols_for(p.bn);
+  p.wait = wait_cfg();
+
+  CUtensorMap tmap_q, tmap_h;
+  // Packed codes as a [V, H/2] byte matrix: a K step of 64 elements is 32 bytes of a row.
+  st = encode_nvfp4_codes(&tmap_q, w_packed, H / 2, V);
+  if (st != LMHEAD_OK) return st;
+  st = encode_2d(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H, rows, lmh::kBK,
+                 (uint32_t)p.bn);
+  if (st != LMHEAD_OK) return st;
+
+  const int grid = p.num_tiles < dev.num_sms ? p.num_tiles : dev.num_sms;
+  const size_t smem = (size_t)reserve + (size_t)stages * per_stage;
+  lmh::lmhead_w4a16_nvfp4_kernel<<<grid, lmh::kNvfp4Threads, smem, (cudaStream_t)stream>>>(
+      tmap_q, tmap_h, p);
+  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+}  // extern "C"

@@ -1,0 +1,230 @@
+// fp32-accumulate LM head, bf16 operands: logits[r, v] = fl32(alpha * sum_k h[r, k] * W[v, k]).
+//
+// One persistent, warp-specialised tcgen05 kernel serves every row count (decode, speculative
+// verify and prefill alike), so a row's reduction order never depends on how many rows a call
+// carries ("A row's logits here do not depend on the row count", lm_head_nvfp4_rows.rs, module
+// doc -- applied here to the bf16 head as well).
+//
+// Orientation ("swap-AB"): W supplies the MMA's M = 128 side and the hidden rows the N side, so
+// a handful of decode rows pads N (16..256 in steps of 16), never M, and each TMEM lane holds one
+// vocab entry: the epilogue's 32 lanes of a warp write 32 consecutive logits of one row.
+//
+// Roles (192 threads):
+//   warp 0     TMA producer: W tile [128 x 64] and hidden tile [BN x 64] per K step into a
+//              ring of shared-memory stages (128-byte swizzle), completion on full[s].
+//   warp 1     TMEM allocator and MMA issuer: 4 x tcgen05.mma (K = 16 each) per stage into one of
+//              two TMEM accumulators, tcgen05.commit frees the stage (empty[s]) and, after the
+//              last K step, hands the accumulator to the epilogue (tmem_full[a]).
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, one IEEE fp32 multiply by alpha, store.
+// Tiles (v-tile, row-tile) are walked v-major with a static stride of gridDim.x, so CTAs that
+// run at the same time share W tiles through L2 in the many-row case.
+#pragma once
+
+#include "lmhead_common.cuh"
+
+namespace lmh {
+
+struct Bf16HeadParams {
+  int64_t rows, H, V;
+  float* out;
+  float alpha;
+  int32_t bn;        // rows per tile: multiple of 16 in [16, 256]
+  int32_t n_rtiles;  // ceil(rows / bn)
+  int32_t n_vtiles;  // ceil(V / 128)
+  int32_t num_tiles;
+  int32_t num_kb;    // ceil(H / 64)
+  int32_t stages;
+  uint32_t tmem_cols;
+  uint32_t stage_bytes;
+  WaitCfg wait;
+};
+
+__global__ void __launch_bounds__(kHeadThreads, 1)
+    lmhead_bf16_f32_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_h, const Bf16HeadParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_up_1024(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = p.stages;
+
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + S);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S);
+  const uint32_t tempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t done_bar = smem_u32(bars + 2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, kEpilogueThreads);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_h);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const uint32_t a_bytes = kBM * kBK * 2;
+  const uint32_t tx_bytes = a_bytes + (uint32_t)p.bn * kBK * 2;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    const uint64_t pol_w = l2_policy_evict_first();  // W is streamed (re-read via L2 only
+    const uint64_t pol_h = l2_policy_evict_last();   // by CTAs sharing a v-tile); hidden stays
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      const int vt = tile / p.n_rtiles;
+      const int rt = tile - vt * p.n_rtiles;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(empty0 + 8 * stage, phase ^ 1u, p.wait, abort_flag)) {
+          fail(kRoleProducer, abort_flag);
+          ok = false;
+          break;
+        }
+        if (lane == 0 && !p.wait.starve_loads) {
+          const uint32_t full = full0 + 8 * stage;
+          uint8_t* sa = stage_base + (size_t)stage * p.stage_bytes;
+          mbar_arrive_expect_tx(full, tx_bytes);
+          tma_load_2d(smem_u32(sa), &tmap_w, full, kb * kBK, vt * kBM, pol_w);
+          tma_load_2d(smem_u32(sa + a_bytes), &tmap_h, full, kb * kBK, rt * p.bn, pol_h);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Drain: wait until every load this CTA issued has landed before the CTA may exit.
+    if (!p.wait.starve_loads) {
+      const int outstanding = issued < S ? issued : S;
+      for (int i = 0; i < outstanding; ++i) {
+        if (--stage < 0) {
+          stage = S - 1;
+          phase ^= 1u;
+        }
+        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, nullptr)) {
+          fail(kRoleDrain, abort_flag);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      if (!wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, p.wait, abort_flag)) {
+        fail(kRoleMma, abort_flag);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, abort_flag)) {
+          fail(kRoleMma, abort_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(stage_base + (size_t)stage * p.stage_bytes);
+          const uint32_t sb = sa + a_bytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k) {
+            mma_bf16_ss(d_tmem, sdesc_kmajor_sw128(sa + k * kUK * 2),
+                        sdesc_kmajor_sw128(sb + k * kUK * 2), idesc, (kb | k) != 0);
+          }
+          mma_commit(empty0 + 8 * stage);
+        }
+        __syncwarp();
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(tfull0 + 8 * acc);
+      __syncwarp();
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    // Every MMA this thread issued must finish before TMEM is released.
+    if (lane == 0) mma_commit(done_bar);
+    __syncwarp();
+    if (!wait_bounded(done_bar, 0, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int v_local = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int vt = tile / p.n_rtiles;
+      const int rt = tile - vt * p.n_rtiles;
+      if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag)) {
+        fail(kRoleEpilogue, abort_flag);
+        break;
+      }
+      tc_fence_after_sync();
+      const int64_t v = (int64_t)vt * kBM + v_local;
+      const int64_t r0 = (int64_t)rt * p.bn;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.bn);
+      const bool v_ok = v < p.V;
+      for (int c = 0; c < p.bn; c += 16) {
+        if (r0 + c >= p.rows) break;  // warp-uniform
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)c, r);
+        tmem_ld_wait();
+        if (v_ok) {
+          float* dst = p.out + (r0 + c) * p.V + v;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (r0 + c + j < p.rows) __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
+          }
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace lmh

@@ -1,0 +1,129 @@
+/*
+ * lmhead -- LM-head logits projection for NVIDIA B200 (sm_100a), C ABI.
+ *
+ *   logits[rows, V] = alpha * (hidden[rows, H] @ W[V, H]^T)
+ *
+ * Entry 1 takes bf16 hidden and W, accumulates in fp32 and writes fp32 logits; no fp32 copy of
+ * either operand is ever made. Entry 2 is the W4A16 NVFP4 head: E2M1 weights with per-16 E4M3
+ * block scales and one fp32 per-tensor scale, bf16 activations that are never quantised, bf16
+ * logits.
+ *
+ * The operation comes from these pages:
+ *  - "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)", "Purpose" and
+ *    "muP is folded into the fp32 GEMM (not a bypass)": out = alpha * (hidden @ w.t()) with
+ *    alpha = 1/mup, bf16 inputs accumulated into fp32 without materialising an fp32 weight copy,
+ *    alpha applied in the GEMM epilogue, bit-identical to the projection followed by a separate
+ *    fp32 multiply by alpha.
+ *  - "FP32 LM head skip FP32 cast" (SGLang PR #32370 summary), implementation breakdown:
+ *    torch.mm(hidden, W.T, out_dtype=float32) -- bf16 x bf16 -> fp32 with an fp32 accumulator,
+ *    replacing a cast of both operands to fp32.
+ *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head at its
+ *    declared W4A16 precision, bf16 logits[rows, vocab], row-major hidden and logits, launching
+ *    nothing unless the head can run, and a row's logits that do not depend on the row count.
+ *
+ * Conventions for every entry point:
+ *  - All array arguments are DEVICE pointers owned by the caller. The library keeps no reference
+ *    after the call returns; buffers must stay alive until the work on `stream` has finished.
+ *  - Matrices are row-major and contiguous: hidden [rows, H], W [V, H] (used transposed), logits
+ *    [rows, V].
+ *  - A call validates its arguments synchronously on the host and launches nothing on error; it
+ *    then enqueues ONE kernel on `stream` and returns without waiting. Faults surface at the
+ *    caller's next synchronisation. There is no fallback path of any kind.
+ *  - rows == 0 is valid and launches nothing.
+ *  - Determinism: the same inputs give the same bits on every run (no atomics, no split-K). Each
+ *    output element is one fp32 accumulator chain over k in ascending 16-element steps, the same
+ *    for every row count, row position and tile, so a row's logits are bit-identical whether it
+ *    is computed alone or with any other rows.
+ *  - Outputs must not overlap inputs (LMHEAD_ERR_ALIAS).
+ *  - Functions are thread-safe; calls on different streams may run concurrently.
+ */
+#ifndef LMHEAD_H
+#define LMHEAD_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* The same type as cudaStream_t / CUstream. NULL is the legacy default stream. */
+typedef struct CUstream_st* lmhead_stream_t;
+
+typedef enum {
+  LMHEAD_OK = 0,
+  LMHEAD_ERR_NULL = 1,    /* a required pointer is NULL */
+  LMHEAD_ERR_SHAPE = 2,   /* a size is negative, zero where it must not be, or unsupported */
+  LMHEAD_ERR_ALIGN = 3,   /* a pointer or row pitch breaks the alignment rules below */
+  LMHEAD_ERR_ARCH = 4,    /* the current device is not an sm_100 (B200-class) GPU */
+  LMHEAD_ERR_LAUNCH = 5,  /* the CUDA runtime refused the launch or a setup call */
+  LMHEAD_ERR_TIMEOUT = 6, /* a kernel gave up waiting on one of its own barriers (see below) */
+  LMHEAD_ERR_ALIAS = 7    /* the output range overlaps an input range */
+} lmhead_status;
+
+/*
+ * Entry 1: fp32 logits from bf16 operands.
+ *   logits[r, v] = fl32(alpha * acc[r, v]),  acc[r, v] = sum_k hidden[r, k] * W[v, k] in fp32.
+ * The multiply by alpha is one IEEE round-to-nearest fp32 multiply of the finished accumulator
+ * (no FMA contraction, no flush to zero), so lmhead_logits_bf16_f32(alpha) equals
+ * fl32(lmhead_logits_bf16_f32(1.0f) * alpha) bit for bit. alpha = 1.0f gives the plain head.
+ *
+ *   hidden  bf16 [rows, H], 16-byte aligned          rows >= 0
+ *   W       bf16 [V, H],    16-byte aligned          H > 0, H % 8 == 0 (16-byte row pitch)
+ *   logits  fp32 [rows, V], 4-byte aligned           V > 0
+ * Returns an lmhead_status.
+ */
+int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const void* W, int64_t V,
+                           float alpha, float* logits, lmhead_stream_t stream);
+
+/*
+ * Entry 2: bf16 logits from the W4A16 NVFP4 head.
+ *   W[v, k]      = e2m1(code[v, k]) * e4m3(w_scales[v, k / 16])      (exact in bf16)
+ *   logits[r, v] = bf16_rn( fl32( fl32(acc[r, v] * w_global_scale) * alpha ) ),
+ *   acc[r, v]    = sum_k hidden[r, k] * W[v, k] in fp32.
+ * Layouts: w_packed is [V, H/2] bytes, element 2j of a row in the LOW nibble of byte j and
+ * element 2j+1 in the high nibble; each E2M1 code is sign (bit 3), exponent (bits 2..1, bias 1),
+ * mantissa (bit 0). w_scales is a plain row-major [V, H/16] array of E4M3 (fn variant) bytes;
+ * scale j of row v covers k in [16j, 16j + 16). NaN scales give unspecified logits.
+ * w_global_scale is the decode multiplier (w = code * scale * w_global_scale).
+ *
+ *   hidden    bf16 [rows, H], 16-byte aligned        rows >= 0
+ *   w_packed  u8 [V, H/2],    16-byte aligned        H > 0, H % 64 == 0
+ *   w_scales  u8 [V, H/16],   4-byte aligned
+ *   logits    bf16 [rows, V], 2-byte aligned         V > 0
+ * (H % 64 == 0 makes every scale row a whole number of 4-byte words.)
+ * Returns an lmhead_status.
+ */
+int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,
+                              const uint8_t* w_scales, float w_global_scale, int64_t V,
+                              float alpha, void* logits, lmhead_stream_t stream);
+
+/* A static English description of a status code. Never NULL. */
+const char* lmhead_status_string(int status);
+
+/*
+ * Every wait inside the kernels is bounded. When one runs out (the default limit is 2 s of wall
+ * time per wait) the kernel records LMHEAD_ERR_TIMEOUT, and where it gave up, in a per-device
+ * status word, stops its work and exits cleanly, so the CUDA context stays usable; the logits
+ * of that call are then undefined. Read the word after synchronising the stream:
+ * returns the recorded status of the CURRENT device (LMHEAD_OK if none) and, when `clear` is
+ * non-zero, resets it. The low byte is the lmhead_status; bits 8..15 name the waiting role.
+ */
+int lmhead_device_status(int clear);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+int lmhead_version(void);
+
+/*
+ * Fault-injection knob for tests of the timeout path (host side, per process). When
+ * `starve_loads` is non-zero, subsequent launches issue no weight/activation loads, so their
+ * consumers wait on barriers that never complete and must time out after `wait_limit_ns`
+ * nanoseconds. wait_limit_ns == 0 restores the default limit. Not for production use.
+ */
+void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMHEAD_H */

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads, exports every
+function include/lmhead.h declares, and rejects bad arguments synchronously -- launching
+nothing, as lm_head_nvfp4_rows.rs's lm_head_nvfp4_rows_run does when its head cannot run."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import fp32_accumulate_lm_b200 as lm
+from fp32_accumulate_lm_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lmhead.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return lm.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lmhead_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_two_entry_points():
+    names = declared_functions()
+    assert "lmhead_logits_bf16_f32" in names and "lmhead_logits_w4a16_nvfp4" in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lm.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing from the statically linked CUDA runtime leaks out
+    assert not any(s.startswith("cuda") for s in exported)
+
+
+def test_header_compiles_as_c():
+    src = f'#include "{HEADER}"\nint main(void) {{ return lmhead_version() < 0; }}\n'
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-x", "c", "-"],
+                         input=src, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+
+
+def test_status_strings_and_version(lib):
+    for code in range(8):
+        assert lm.status_string(code) and lm.status_string(code) != "unknown status"
+    assert lm.status_string(99) == "unknown status"
+    assert lm.version() >= 100
+
+
+# Pointer values below are never dereferenced: every case fails validation first.
+A16 = 0x10000  # 16-byte aligned fake device addresses
+B16 = 0x20000000
+C16 = 0x40000000
+
+
+@pytest.mark.parametrize("rows,H,V,want", [
+    (-1, 64, 128, 2), (4, 0, 128, 2), (4, 64, 0, 2), (4, -8, 128, 2),
+    (4, 60, 128, 3),            # H % 8 != 0: 16-byte row pitch impossible
+    (2 ** 31, 64, 128, 2),      # beyond the int32 tile coordinates
+])
+def test_bf16_shape_errors(lib, rows, H, V, want):
+    assert lm.lmhead_logits_bf16_f32(A16, rows, H, B16, V, 1.0, C16, 0) == want
+
+
+def test_bf16_null_align_alias(lib):
+    assert lm.lmhead_logits_bf16_f32(0, 4, 64, B16, 128, 1.0, C16, 0) == 1
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, 0, 128, 1.0, C16, 0) == 1
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, 0, 0) == 1
+    assert lm.lmhead_logits_bf16_f32(A16 + 8, 4, 64, B16, 128, 1.0, C16, 0) == 3
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16 + 2, 128, 1.0, C16, 0) == 3
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, C16 + 2, 0) == 3
+    # logits overlapping W or hidden
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, B16 + 64, 0) == 7
+    assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, A16 - 16, 0) == 7
+
+
+def test_rows_zero_launches_nothing(lib):
+    # rows == 0 is a no-op even with NULL pointers (no CUDA call is made)
+    assert lm.lmhead_logits_bf16_f32(0, 0, 64, 0, 128, 1.0, 0, 0) == 0
+    assert lm.lmhead_logits_w4a16_nvfp4(0, 0, 64, 0, 0, 1.0, 128, 1.0, 0, 0) == 0
+
+
+def test_nvfp4_argument_errors(lib):
+    f = lm.lmhead_logits_w4a16_nvfp4
+    assert f(A16, 4, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) != 2  # valid shape gets past
+    assert f(A16, -1, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 2
+    assert f(A16, 4, 96, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 3   # H % 64 != 0
+    assert f(A16, 4, 64, B16, C16, 1.0, 0, 1.0, 0x7000000, 0) == 2
+    assert f(0, 4, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 1
+    assert f(A16, 4, 64, 0, C16, 1.0, 128, 1.0, 0x7000000, 0) == 1
+    assert f(A16, 4, 64, B16, 0, 1.0, 128, 1.0, 0x7000000, 0) == 1
+    assert f(A16, 4, 64, B16 + 4, C16, 1.0, 128, 1.0, 0x7000000, 0) == 3
+    assert f(A16, 4, 64, B16, C16 + 2, 1.0, 128, 1.0, 0x7000000, 0) == 3
+    assert f(A16, 4, 64, B16, C16, 1.0, 128, 1.0, 0x7000001, 0) == 3
+    assert f(A16, 4, 64, B16, C16, 1.0, 128, 1.0, B16 + 16, 0) == 7   # logits over the codes
+    assert f(A16, 4, 64, B16, C16, 1.0, 128, 1.0, C16, 0) == 7        # logits over the scales
+
+
+def test_no_cpu_fallback_without_a_device(lib):
+    """On a host without a usable GPU a valid call must fail loudly, never compute on the CPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, C16, 0)
+    assert st in (4, 5)
+
+
+def test_torch_wrapper_rejects_wrong_dtypes():
+    import torch
+    h = torch.zeros(2, 64, dtype=torch.float32)
+    w = torch.zeros(8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lm.logits_bf16_f32(h, w, 1.0)
