@@ -24,6 +24,17 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxStages = 16;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 
+// L2 sector promotion of weight loads: 0 none, 1 64 B, 2 128 B, 3 256 B (build-time knob).
+#ifndef LMHEAD_WEIGHT_L2_PROMOTION
+#define LMHEAD_WEIGHT_L2_PROMOTION 3
+#endif
+// Force the bf16 head's K sub-tiles per stage (0 = choose by shared-memory room).
+#ifndef LMHEAD_FORCE_NSUB
+#define LMHEAD_FORCE_NSUB 0
+#endif
+constexpr CUtensorMapL2promotion kWeightPromo =
+    (CUtensorMapL2promotion)(CU_TENSOR_MAP_L2_PROMOTION_NONE + LMHEAD_WEIGHT_L2_PROMOTION);
+
 std::atomic<int> g_starve_loads{0};
 std::atomic<uint64_t> g_wait_limit_ns{0};
 
@@ -79,7 +90,13 @@ int current_device(DeviceInfo* out) {
   }
   if (!d.arch_ok) return LMHEAD_ERR_ARCH;
   if (!d.attrs_set) {
-    if (cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel,
+    if (cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              d.smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(lmh::lmhead_w4a16_nvfp4_kernel,
@@ -100,9 +117,12 @@ bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
   return a0 < b0 + (uintptr_t)bbytes && b0 < a0 + (uintptr_t)abytes;
 }
 
-// Row-major [outer, inner] tensor, tile box [box_outer, box_inner], 128-byte swizzle.
+// Row-major [outer, inner] tensor, tile box [box_outer, box_inner], 128-byte swizzle unless
+// `swizzle` says otherwise.
 int encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base,
-              int64_t inner, int64_t outer, uint32_t box_inner, uint32_t box_outer) {
+              int64_t inner, int64_t outer, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+              CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return LMHEAD_ERR_LAUNCH;
   const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
@@ -110,25 +130,28 @@ int encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
-// Packed NVFP4 codes as a [V, H/2] byte matrix, box [128 rows x 32 bytes] (one K step of 64),
-// no swizzle: the dequantisers read it as plain row-major bytes.
-int encode_nvfp4_codes(CUtensorMap* map, const void* base, int64_t row_bytes, int64_t V) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return LMHEAD_ERR_LAUNCH;
-  const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)V};
-  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  const cuuint32_t box[2] = {(cuuint32_t)(lmh::kBK / 2), (cuuint32_t)lmh::kBM};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+// Tensor map over a row-major [outer, inner_bytes / esize] matrix of esize-byte elements, box
+// [box_outer rows x box_bytes bytes]. With LMHEAD_TMA_WIDE the rows are described as 32-bit
+// elements (identical bytes in global and shared memory, a quarter or half as many elements).
+int encode_rows(CUtensorMap* map, CUtensorMapDataType natural, int esize, const void* base,
+                int64_t inner_bytes, int64_t outer, uint32_t box_bytes, uint32_t box_outer,
+                CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promo) {
+  if (LMHEAD_TMA_WIDE)
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, inner_bytes / 4, outer,
+                     box_bytes / 4, box_outer, swizzle, promo);
+  return encode_2d(map, natural, esize, base, inner_bytes / esize, outer, box_bytes / esize,
+                   box_outer, swizzle, promo);
+}
+
+// Rows of hidden one TMA box brings: the call's rows when they fit one row tile (the MMA still
+// spans bn columns; columns past the call's rows are never stored), else the tile height.
+int32_t hid_box_rows(int64_t rows, int32_t bn) {
+  return (LMHEAD_HID_BOX_EXACT && rows < bn) ? (int32_t)rows : bn;
 }
 
 lmh::WaitCfg wait_cfg() {
@@ -150,6 +173,29 @@ uint32_t tmem_cols_for(int32_t bn) {
 }
 
 constexpr int kInt32Max = 0x7fffffff;
+
+// Tile ownership (see TileSched) and grid size: one persistent CTA per SM at most.
+int make_sched(int64_t rows, int64_t V, int32_t bn, int num_sms, lmh::TileSched* s, int* grid) {
+  s->bn = bn;
+  s->n_rtiles = (int32_t)((rows + bn - 1) / bn);
+  const int64_t n_vtiles = (V + lmh::kBM - 1) / lmh::kBM;
+  const int64_t tiles = (int64_t)s->n_rtiles * n_vtiles;
+  if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
+  s->num_tiles = (int32_t)tiles;
+  *grid = s->num_tiles < num_sms ? s->num_tiles : num_sms;
+  return LMHEAD_OK;
+}
+
+// 64-wide K sub-tiles per pipeline stage of the bf16 head: the largest of 4, 2, 1 that still
+// leaves room for 3 stages. Longer per-stage bursts along each weight row read HBM faster.
+int pick_nsub(int32_t bn, int smem_budget) {
+  if (LMHEAD_FORCE_NSUB) return LMHEAD_FORCE_NSUB;
+  for (int nsub = 4; nsub > 1; nsub /= 2) {
+    const int stage = nsub * (lmh::kBM * lmh::kBK * 2 + bn * lmh::kBK * 2);
+    if (smem_budget / stage >= 3) return nsub;
+  }
+  return 1;
+}
 
 }  // namespace
 
@@ -211,14 +257,13 @@ int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const vo
   p.out = logits;
   p.alpha = alpha;
   p.bn = pick_bn(rows);
-  p.n_rtiles = (int32_t)((rows + p.bn - 1) / p.bn);
-  p.n_vtiles = (int32_t)((V + lmh::kBM - 1) / lmh::kBM);
-  const int64_t tiles = (int64_t)p.n_rtiles * p.n_vtiles;
-  if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
-  p.num_tiles = (int32_t)tiles;
-  p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
-  p.stage_bytes = (uint32_t)(lmh::kBM * lmh::kBK * 2 + p.bn * lmh::kBK * 2);
+  int grid = 0;
+  st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
+  if (st != LMHEAD_OK) return st;
   const int reserve = 1024 + 512;  // alignment slack + barriers
+  const int nsub = pick_nsub(p.bn, dev.smem_optin - reserve);
+  p.num_ks = (int32_t)((H + nsub * lmh::kBK - 1) / (nsub * lmh::kBK));
+  p.stage_bytes = (uint32_t)(nsub * (lmh::kBM * lmh::kBK * 2 + p.bn * lmh::kBK * 2));
   int stages = (dev.smem_optin - reserve) / (int)p.stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return LMHEAD_ERR_SHAPE;
@@ -227,16 +272,20 @@ int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const vo
   p.wait = wait_cfg();
 
   CUtensorMap tmap_w, tmap_h;
-  st = encode_2d(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, H, V, lmh::kBK, lmh::kBM);
+  st = encode_rows(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, H * 2, V, lmh::kBK * 2,
+                   lmh::kBM, CU_TENSOR_MAP_SWIZZLE_128B, kWeightPromo);
   if (st != LMHEAD_OK) return st;
-  st = encode_2d(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H, rows, lmh::kBK,
-                 (uint32_t)p.bn);
+  p.hid_rows = hid_box_rows(rows, p.bn);
+  st = encode_rows(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H * 2, rows,
+                   lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (st != LMHEAD_OK) return st;
 
-  const int grid = p.num_tiles < dev.num_sms ? p.num_tiles : dev.num_sms;
   const size_t smem = (size_t)reserve + (size_t)stages * p.stage_bytes;
-  lmh::lmhead_bf16_f32_kernel<<<grid, lmh::kHeadThreads, smem, (cudaStream_t)stream>>>(
-      tmap_w, tmap_h, p);
+  auto kernel = nsub == 4 ? lmh::lmhead_bf16_f32_kernel<4>
+                : nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2>
+                            : lmh::lmhead_bf16_f32_kernel<1>;
+  kernel<<<grid, lmh::kHeadThreads, smem, (cudaStream_t)stream>>>(tmap_w, tmap_h, p);
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
@@ -271,37 +320,43 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.scales = w_scales;
   p.alpha = alpha;
   p.gscale = w_global_scale;
-  p.bn = pick_bn(rows);
-  p.n_rtiles = (int32_t)((rows + p.bn - 1) / p.bn);
-  p.n_vtiles = (int32_t)((V + lmh::kBM - 1) / lmh::kBM);
-  const int64_t tiles = (int64_t)p.n_rtiles * p.n_vtiles;
-  if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
-  p.num_tiles = (int32_t)tiles;
-  p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
-  p.raw_bytes = (uint32_t)(lmh::kBM * lmh::kBK / 2);        // packed nibbles of one K step
-  p.a_bytes = (uint32_t)(lmh::kBM * lmh::kBK * 2);          // dequantised bf16 tile
-  p.b_bytes = (uint32_t)(p.bn * lmh::kBK * 2);              // hidden tile
-  const int reserve = 1024 + 1024;
-  const int per_stage = (int)lmh::nvfp4_stage_bytes(p.bn);
-  int stages = (dev.smem_optin - reserve) / per_stage;
-  if (stages > kMaxStages) stages = kMaxStages;
+  p.bn = pick_bn(rows) < lmh::kBnMax ? pick_bn(rows) : lmh::kBnMax;
+  int grid = 0;
+  st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
+  if (st != LMHEAD_OK) return st;
+  p.num_kb = (int32_t)(H / lmh::kBK);
+  const int reserve = 1024 + 512;
+  const int stage_bytes = (int)lmh::nvfp4_stage_bytes(p.bn);
+  int stages = (dev.smem_optin - reserve) / stage_bytes;
+  if (stages > 8) stages = 8;
   if (stages < 2) return LMHEAD_ERR_SHAPE;
   p.stages = stages;
-  p.tmem_cols = tmem_cols_for(p.bn);
+  // Block scales come by TMA when each scale row is a whole number of 16-byte units.
+  p.scale_tma = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? 1 : 0;
   p.wait = wait_cfg();
 
-  CUtensorMap tmap_q, tmap_h;
-  // Packed codes as a [V, H/2] byte matrix: a K step of 64 elements is 32 bytes of a row.
-  st = encode_nvfp4_codes(&tmap_q, w_packed, H / 2, V);
+  // Packed codes as a [V, H/2] byte matrix, boxes of [128 rows x 128 bytes] (4 K steps) with the
+  // 128-byte swizzle; scales as a [V, H/16] byte matrix, boxes of [128 rows x 16 bytes].
+  CUtensorMap tmap_q, tmap_s, tmap_h;
+  st = encode_rows(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_packed, H / 2, V,
+                   lmh::kRawK * lmh::kBK / 2, lmh::kBM, CU_TENSOR_MAP_SWIZZLE_128B, kWeightPromo);
   if (st != LMHEAD_OK) return st;
-  st = encode_2d(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H, rows, lmh::kBK,
-                 (uint32_t)p.bn);
+  if (p.scale_tma) {
+    st = encode_rows(&tmap_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_scales, H / 16, V,
+                     lmh::kRawK * 4, lmh::kBM, CU_TENSOR_MAP_SWIZZLE_NONE, kWeightPromo);
+    if (st != LMHEAD_OK) return st;
+  } else {
+    tmap_s = tmap_q;  // unused
+  }
+  p.hid_rows = hid_box_rows(rows, p.bn);
+  st = encode_rows(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H * 2, rows,
+                   lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (st != LMHEAD_OK) return st;
 
-  const int grid = p.num_tiles < dev.num_sms ? p.num_tiles : dev.num_sms;
-  const size_t smem = (size_t)reserve + (size_t)stages * per_stage;
+  const size_t smem = (size_t)reserve + (size_t)stages * stage_bytes;
   lmh::lmhead_w4a16_nvfp4_kernel<<<grid, lmh::kNvfp4Threads, smem, (cudaStream_t)stream>>>(
-      tmap_q, tmap_h, p);
+      tmap_q, tmap_s, tmap_h, p);
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 

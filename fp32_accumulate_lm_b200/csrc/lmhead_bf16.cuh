@@ -10,14 +10,13 @@
 // vocab entry: the epilogue's 32 lanes of a warp write 32 consecutive logits of one row.
 //
 // Roles (192 threads):
-//   warp 0     TMA producer: W tile [128 x 64] and hidden tile [BN x 64] per K step into a
-//              ring of shared-memory stages (128-byte swizzle), completion on full[s].
-//   warp 1     TMEM allocator and MMA issuer: 4 x tcgen05.mma (K = 16 each) per stage into one of
-//              two TMEM accumulators, tcgen05.commit frees the stage (empty[s]) and, after the
-//              last K step, hands the accumulator to the epilogue (tmem_full[a]).
+//   warp 0     TMA producer: per pipeline stage, NSUB sub-tiles of 64 K-elements each of W
+//              [128 x 64] and of the hidden rows [BN x 64] (128-byte swizzle), landing on full[s].
+//   warp 1     TMEM allocator and MMA issuer: 4 * NSUB tcgen05.mma (K = 16 each) per stage into
+//              one of two TMEM accumulators; tcgen05.commit frees the stage (empty[s]) and, after
+//              the last K step, hands the accumulator to the epilogue (tmem_full[a]).
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, one IEEE fp32 multiply by alpha, store.
-// Tiles (v-tile, row-tile) are walked v-major with a static stride of gridDim.x, so CTAs that
-// run at the same time share W tiles through L2 in the many-row case.
+// Tile ownership: see TileSched.
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -29,16 +28,16 @@ struct Bf16HeadParams {
   float* out;
   float alpha;
   int32_t bn;        // rows per tile: multiple of 16 in [16, 256]
-  int32_t n_rtiles;  // ceil(rows / bn)
-  int32_t n_vtiles;  // ceil(V / 128)
-  int32_t num_tiles;
-  int32_t num_kb;    // ceil(H / 64)
+  int32_t hid_rows;  // rows of hidden one TMA box brings (<= bn; MMA columns past it unused)
+  TileSched sched;
+  int32_t num_ks;    // pipeline stages per tile: ceil(H / (64 * NSUB))
   int32_t stages;
   uint32_t tmem_cols;
   uint32_t stage_bytes;
   WaitCfg wait;
 };
 
+template <int NSUB>
 __global__ void __launch_bounds__(kHeadThreads, 1)
     lmhead_bf16_f32_kernel(const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ CUtensorMap tmap_h, const Bf16HeadParams p) {
@@ -48,6 +47,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   const int lane = threadIdx.x & 31;
   const int S = p.stages;
 
+  // stage s: [A sub-tile 0 .. NSUB-1, 16 KB each][B sub-tile 0 .. NSUB-1, BN*128 bytes each]
+  constexpr uint32_t a_sub = kBM * kBK * 2;
+  const uint32_t b_sub = (uint32_t)p.bn * kBK * 2;
+  const uint32_t b_tx = (uint32_t)p.hid_rows * kBK * 2;
   uint8_t* stage_base = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
   const uint32_t full0 = smem_u32(bars);
@@ -83,22 +86,20 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-
-  const uint32_t a_bytes = kBM * kBK * 2;
-  const uint32_t tx_bytes = a_bytes + (uint32_t)p.bn * kBK * 2;
+  const int my_tiles = sched_count(p.sched);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    const uint64_t pol_w = l2_policy_evict_first();  // W is streamed (re-read via L2 only
-    const uint64_t pol_h = l2_policy_evict_last();   // by CTAs sharing a v-tile); hidden stays
+    const uint64_t pol_w = l2_policy_weights();
+    const uint64_t pol_h = l2_policy_evict_last();  // hidden rows are re-read per v-tile
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      const int vt = tile / p.n_rtiles;
-      const int rt = tile - vt * p.n_rtiles;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+    for (int t = 0; ok && t < my_tiles; ++t) {
+      const TileCoord tc = sched_tile(p.sched, p.V, t);
+      const uint32_t tx = (uint32_t)NSUB * (a_sub + b_tx);
+      for (int ks = 0; ks < p.num_ks; ++ks) {
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1u, p.wait, abort_flag)) {
           fail(kRoleProducer, abort_flag);
           ok = false;
@@ -106,10 +107,17 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         }
         if (lane == 0 && !p.wait.starve_loads) {
           const uint32_t full = full0 + 8 * stage;
-          uint8_t* sa = stage_base + (size_t)stage * p.stage_bytes;
-          mbar_arrive_expect_tx(full, tx_bytes);
-          tma_load_2d(smem_u32(sa), &tmap_w, full, kb * kBK, vt * kBM, pol_w);
-          tma_load_2d(smem_u32(sa + a_bytes), &tmap_h, full, kb * kBK, rt * p.bn, pol_h);
+          const uint32_t sa = smem_u32(stage_base + (size_t)stage * p.stage_bytes);
+          const uint32_t sb = sa + NSUB * a_sub;
+          mbar_arrive_expect_tx(full, tx);
+#pragma unroll
+          for (int j = 0; j < NSUB; ++j)
+            tma_load_2d(sa + j * a_sub, &tmap_w, full, tma_x((ks * NSUB + j) * kBK * 2, 2),
+                        (int32_t)tc.v0, pol_w);
+#pragma unroll
+          for (int j = 0; j < NSUB; ++j)
+            tma_load_2d(sb + j * b_sub, &tmap_h, full, tma_x((ks * NSUB + j) * kBK * 2, 2),
+                        (int32_t)tc.r0, pol_h);
         }
         __syncwarp();
         ++issued;
@@ -141,14 +149,14 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int t = 0; ok && t < my_tiles; ++t) {
       if (!wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, p.wait, abort_flag)) {
         fail(kRoleMma, abort_flag);
         break;
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int ks = 0; ks < p.num_ks; ++ks) {
         if (!wait_bounded(full0 + 8 * stage, phase, p.wait, abort_flag)) {
           fail(kRoleMma, abort_flag);
           ok = false;
@@ -157,11 +165,15 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         tc_fence_after_sync();
         if (lane == 0) {
           const uint32_t sa = smem_u32(stage_base + (size_t)stage * p.stage_bytes);
-          const uint32_t sb = sa + a_bytes;
+          const uint32_t sb = sa + NSUB * a_sub;
 #pragma unroll
-          for (int k = 0; k < kBK / kUK; ++k) {
-            mma_bf16_ss(d_tmem, sdesc_kmajor_sw128(sa + k * kUK * 2),
-                        sdesc_kmajor_sw128(sb + k * kUK * 2), idesc, (kb | k) != 0);
+          for (int j = 0; j < NSUB; ++j) {
+#pragma unroll
+            for (int k = 0; k < kBK / kUK; ++k) {
+              mma_bf16_ss(d_tmem, sdesc_kmajor_sw128(sa + j * a_sub + k * kUK * 2),
+                          sdesc_kmajor_sw128(sb + j * b_sub + k * kUK * 2), idesc,
+                          (ks | j | k) != 0);
+            }
           }
           mma_commit(empty0 + 8 * stage);
         }
@@ -187,18 +199,17 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     const int v_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int vt = tile / p.n_rtiles;
-      const int rt = tile - vt * p.n_rtiles;
-      if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag)) {
+    for (int t = 0; t < my_tiles; ++t) {
+      const TileCoord tc = sched_tile(p.sched, p.V, t);
+      if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag, kSleepHintNs)) {
         fail(kRoleEpilogue, abort_flag);
         break;
       }
       tc_fence_after_sync();
-      const int64_t v = (int64_t)vt * kBM + v_local;
-      const int64_t r0 = (int64_t)rt * p.bn;
+      const int64_t v = tc.v0 + v_local;
+      const int64_t r0 = tc.r0;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.bn);
-      const bool v_ok = v < p.V;
+      const bool v_ok = v_local < tc.vrows;
       for (int c = 0; c < p.bn; c += 16) {
         if (r0 + c >= p.rows) break;  // warp-uniform
         uint32_t r[16];
@@ -208,7 +219,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           float* dst = p.out + (r0 + c) * p.V + v;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (r0 + c + j < p.rows) __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
+            if (r0 + c + j < p.rows)
+              __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
           }
         }
       }

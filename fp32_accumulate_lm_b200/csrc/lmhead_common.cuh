@@ -7,7 +7,30 @@
 
 #include "sm100_ptx.cuh"
 
+// Build-time tuning knobs (defaults are the measured best on B200; see the design notes):
+//   LMHEAD_WEIGHT_L2_POLICY  L2 hint for weight loads: 0 none, 1 evict-first, 2 evict-normal
+//   LMHEAD_TMA_WIDE          1: tensor maps see rows as 32-bit elements (same bytes, fewer
+//                            elements per box); 0: their natural types (bf16 / bytes)
+//   LMHEAD_HID_BOX_EXACT     1: a single row tile loads only the call's rows of hidden, not
+//                            the padded tile height
+#ifndef LMHEAD_WEIGHT_L2_POLICY
+#define LMHEAD_WEIGHT_L2_POLICY 1
+#endif
+#ifndef LMHEAD_TMA_WIDE
+#define LMHEAD_TMA_WIDE 1
+#endif
+#ifndef LMHEAD_HID_BOX_EXACT
+#define LMHEAD_HID_BOX_EXACT 1
+#endif
+// Elements per 128-byte row of a TMA box, and the x coordinate of byte offset b in a row.
+
+
 namespace lmh {
+
+// TMA x coordinate of byte offset `bytes` within a row whose natural element is `esize` bytes.
+__host__ __device__ constexpr int32_t tma_x(int64_t bytes, int esize) {
+  return (int32_t)(LMHEAD_TMA_WIDE ? bytes / 4 : bytes / esize);
+}
 
 constexpr int kBM = 128;   // vocab rows per tile (MMA M)
 constexpr int kBK = 64;    // K elements per pipeline stage (one 128-byte swizzle row of bf16)
@@ -26,6 +49,10 @@ enum : unsigned {
 
 constexpr unsigned kStatusTimeout = 6;  // == LMHEAD_ERR_TIMEOUT
 
+// Waits that are expected to last (the epilogue waiting for a whole tile's MMAs) let the
+// hardware suspend the thread up to this long per try instead of spinning on issue slots.
+constexpr uint32_t kSleepHintNs = 2000;
+
 struct WaitCfg {
   uint64_t limit_ns;     // wall-time limit of one barrier wait
   int32_t starve_loads;  // test-only: issue no loads, so consumers must time out
@@ -42,12 +69,12 @@ __device__ __forceinline__ uint8_t* align_up_1024(uint8_t* p) {
 // this CTA has already given up. Every lane of the calling warp waits and the warp agrees on the
 // result, so control flow stays warp-uniform.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCfg& w,
-                                             volatile int* abort_flag) {
+                                             volatile int* abort_flag, uint32_t sleep_ns = 0) {
   bool ok = mbar_try_wait(bar, parity);
   if (!ok) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
-      if (mbar_try_wait(bar, parity)) {
+      if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) {
         ok = true;
         break;
       }
@@ -58,6 +85,52 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
     }
   }
   return __all_sync(0xffffffffu, ok);
+}
+
+// Which output tiles a CTA owns. Tile t = (v-tile, row-tile) = (t / n_rtiles, t % n_rtiles):
+// 128 vocab rows by bn hidden rows; CTA i of G takes t = i, i + G, i + 2G, ... At any moment the
+// G CTAs work on neighbouring v-tiles, which keeps the weight stream on few DRAM pages and, with
+// many row tiles, lets CTAs share each weight tile through L2. (Balanced per-CTA strips of W and
+// splitting the last partial wave into 16-row pieces were both measured slower on B200.)
+// Every tile runs the same MMA chain over K, so the schedule changes no output bit.
+struct TileSched {
+  int32_t n_rtiles;
+  int32_t num_tiles;
+  int32_t bn;
+};
+
+struct TileCoord {
+  int64_t v0;     // first vocab row
+  int32_t vrows;  // vocab rows that belong to this tile (<= 128; rows past V are zero-filled)
+  int64_t r0;     // first hidden row
+};
+
+__device__ __forceinline__ int sched_count(const TileSched& s) {
+  return blockIdx.x < (unsigned)s.num_tiles
+             ? (int)((s.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x) + 1
+             : 0;
+}
+
+__device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, int i) {
+  TileCoord c;
+  const int t = (int)blockIdx.x + i * (int)gridDim.x;
+  const int vt = t / s.n_rtiles;
+  const int rt = t - vt * s.n_rtiles;
+  c.v0 = (int64_t)vt * kBM;
+  const int64_t left = V - c.v0;
+  c.vrows = (int32_t)(left < kBM ? left : kBM);
+  c.r0 = (int64_t)rt * s.bn;
+  return c;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_weights() {
+#if LMHEAD_WEIGHT_L2_POLICY == 1
+  return l2_policy_evict_first();
+#elif LMHEAD_WEIGHT_L2_POLICY == 2
+  return l2_policy_evict_normal();
+#else
+  return 0;
+#endif
 }
 
 __device__ __forceinline__ void fail(unsigned role, volatile int* abort_flag) {

@@ -2,29 +2,55 @@
 // rows that are never quantised (lm_head_nvfp4_rows.rs, module doc: the declared W4A16 head on
 // tensor-core row tiles, bf16 logits, a row's logits independent of the row count).
 //
-// The weight tile is dequantised in registers to bf16 and fed to the same tcgen05 bf16 MMA
-// chain as the bf16 head. W[v, k] = e2m1 * e4m3 has at most 6 significant bits and lies in
-// [2^-10, 2688], so it is exact in bf16 and every product with a bf16 hidden value is exact in
-// the fp32 accumulator, as for the bf16 head. The per-tensor scale g and alpha are applied in
-// the epilogue: logits = bf16_rn(fl32(fl32(acc * g) * alpha)).
+// The weight tile is dequantised in registers and written to tensor memory, where the bf16
+// tcgen05 MMA reads it as its A operand; the hidden rows (B) come from shared memory as in the
+// bf16 head. Keeping A out of shared memory matters: at HBM speed the dequantised tile would
+// need more shared-memory bandwidth (write it, then read it back) than an SM has.
 //
-// Roles (448 threads):
-//   warp 0      producer: TMA of the packed codes [128 rows x 32 bytes] and the hidden tile
-//               [BN x 64] per K step of 64, plus 4-byte async copies of the block scales
-//               [128 rows x 4]; all land on full[s].
-//   warp 1      TMEM allocator and MMA issuer (waits on full[s] and deq_full[s]).
+// Exactness. The value placed in TMEM is w' = e2m1 * e4m3 * 2^-7: it has at most 6 significant
+// bits and lies in [2^-17, 21], so it is an exact normal bf16, and every product with a bf16
+// hidden value is exact in the fp32 accumulator. The accumulator therefore holds exactly 2^-7
+// times what unscaled weights would give (fp32 rounding commutes with a power-of-two scale away
+// from the subnormal range), and the epilogue restores it exactly:
+//   logits = bf16_rn( fl32( fl32( (acc * 2^7) * g ) * alpha ) ).
+//
+// Every hand-off covers 4 K steps (256 elements of K). The single-thread roles (TMA producer,
+// MMA issuer) share their SM sub-partitions with busy dequantiser warps, so each of their
+// instructions is slow; paying one wait and one commit per K step of 64 made them the
+// bottleneck.
+//   stage (shared memory) 4 K steps of: the packed codes [128 rows x 128 bytes] in one box,
+//         their block scales [128 rows x 16 bytes] (TMA when the scale pitch allows, 4-byte
+//         async copies otherwise) and the hidden rows [BN x 64] x 4.
+//   slot  (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; two slots.
+// Roles (192 + 128 * kDequantGroups threads):
+//   warp 0      producer: fills stages.
+//   warp 1      TMEM allocator and MMA issuer: per stage waits for it and for its weight slot,
+//               16 x tcgen05.mma with A from TMEM, one commit frees each.
 //   warps 2-5   epilogue.
-//   warps 6-13  dequantisers: codes + scales of stage s -> bf16 tile in the 128-byte swizzled
-//               K-major layout the MMA reads, then deq_full[s].
+//   warps 6-13  dequantisers: two groups of four warps (one per TMEM lane quarter); group g
+//               takes stages g, g + 2, ... into slot g. Each thread converts one weight row.
 #pragma once
 
 #include "lmhead_common.cuh"
 
 namespace lmh {
 
-constexpr int kNvfp4Threads = 448;
+// Dequantiser groups of four warps (build-time knob LMHEAD_NVFP4_DQ_GROUPS).
+#ifndef LMHEAD_NVFP4_DQ_GROUPS
+#define LMHEAD_NVFP4_DQ_GROUPS 2
+#endif
+constexpr int kDequantGroups = LMHEAD_NVFP4_DQ_GROUPS;  // groups take K steps in turn
 constexpr int kDequantWarp0 = 6;
-constexpr int kDequantThreads = 256;
+constexpr int kDequantThreads = 128;                    // threads that fill one K step
+constexpr int kNvfp4Threads = 32 * kDequantWarp0 + kDequantThreads * kDequantGroups;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAColBase = 256;  // TMEM columns [256, 512): two dequantised weight slots
+constexpr int kBnMax = 128;          // row tile cap: two accumulators of <= 128 columns
+
+constexpr int kRawK = 4;                                  // K steps per stage
+constexpr uint32_t kRawCodeBytes = kBM * kRawK * kBK / 2;  // 16 KB
+constexpr uint32_t kRawScaleBytes = kBM * kRawK * 4;       // 2 KB
+constexpr uint32_t kSlotCols = kRawK * kBK / 2;            // TMEM columns of one weight slot
 
 struct Nvfp4HeadParams {
   int64_t rows, H, V;
@@ -33,19 +59,21 @@ struct Nvfp4HeadParams {
   float alpha;
   float gscale;
   int32_t bn;
-  int32_t n_rtiles, n_vtiles, num_tiles;
-  int32_t num_kb;
+  int32_t hid_rows;       // rows of hidden one TMA box brings (<= bn; MMA columns past it unused)
+  TileSched sched;
+  int32_t num_kb;         // K steps of 64 per tile (H / 64)
   int32_t stages;
-  uint32_t tmem_cols;
-  uint32_t raw_bytes;  // packed codes of one stage
-  uint32_t a_bytes;    // bf16 weight tile
-  uint32_t b_bytes;    // bf16 hidden tile
+  int32_t scale_tma;      // 1: block scales by TMA (H % 256 == 0), 0: 4-byte async copies
   WaitCfg wait;
 };
 
-// Stage layout: [A bf16 16 KB][B hidden BN*128][codes 4 KB][scales 512 B][pad 512 B]
+// Shared-memory stage (4 K steps): [hidden: 4 sub-tiles of BN x 64 bf16, 128-byte swizzle]
+// [codes: 128 rows x 128 bytes, 128-byte swizzle][scales: 128 rows x 16 bytes]
+__host__ __device__ constexpr uint32_t nvfp4_hid_sub_bytes(int bn) {
+  return (uint32_t)(bn * kBK * 2);
+}
 __host__ __device__ constexpr uint32_t nvfp4_stage_bytes(int bn) {
-  return (uint32_t)(kBM * kBK * 2 + bn * kBK * 2 + kBM * kBK / 2 + 1024);
+  return (uint32_t)kRawK * nvfp4_hid_sub_bytes(bn) + kRawCodeBytes + kRawScaleBytes;
 }
 
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -58,71 +86,128 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
-// bf16x2 (s', s') with s' = e4m3(code) * 2^112, exact (at most 4 significant bits, exponent
-// within bf16's range).
-__device__ __forceinline__ uint32_t scale_bf16x2_shifted(uint32_t code) {
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// bf16x2 (s', s') with s' = e4m3(code) * 2^119: exact (4 significant bits) and inside bf16's
+// normal range for every finite E4M3 (2^-9 .. 448).
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t code) {
   const uint32_t both = code | (code << 8);
   uint32_t h2;
   asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
       : "=r"(h2)
       : "r"(both));
-  const float f = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))) * 0x1p112f;
+  const float f = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))) * 0x1p119f;
   uint32_t out;
   asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(out) : "f"(f));
   return out;
 }
 
-// Two E2M1 codes (one byte: element 2j low nibble, 2j+1 high nibble) times the block scale,
-// as bf16x2 (element 2j in the low half). All steps are exact:
-//   h = f16x2 of the codes; (h >> 3) & 0x0FFF0FFF keeps each magnitude's exponent and mantissa
-//   in bf16 position, which reads as |q| * 2^-112 (zero stays zero); one bf16x2 multiply by
-//   s * 2^112 gives |q| * s; the codes' sign bits are put back with an XOR.
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t byte, uint32_t s2) {
-  uint32_t h;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-      : "=r"(h)
-      : "r"(byte));
-  const uint32_t mag = (h >> 3) & 0x0FFF0FFFu;
-  uint32_t p;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p) : "r"(mag), "r"(s2));
-  return p ^ (h & 0x80008000u);
+// Eight E2M1 codes (one little-endian word: element i in nibble i) times the block scale, as
+// four bf16x2 words in natural order (elements 2j, 2j+1 in word j), each value e2m1*e4m3*2^-7.
+//   1. A multiply spreads each selected nibble twice: to bits 9..6 (its exponent and mantissa
+//      land on bf16 bits 8..6) and to bits 15..12 (its sign lands on bit 15); a mask keeps just
+//      those four bits. Read as bf16 that is +-q * 2^-126 -- a bf16 subnormal for q = 0.5,
+//      exactly as E2M1 is subnormal there -- and zero for codes 0 / 8. The multiply handles
+//      nibbles i and i + 4 together (16 bits apart).
+//   2. prmt re-pairs halves into (2j, 2j+1) order.
+//   3. One exact bf16x2 multiply by s * 2^119.
+__device__ __forceinline__ void dequant8(uint32_t x, uint32_t s2, uint32_t* w) {
+  const uint32_t x8 = x >> 8;
+  const uint32_t p04 = ((x & 0x000F000Fu) * 0x1040u) & 0x81C081C0u;   // nibbles 0, 4
+  const uint32_t p15 = ((x & 0x00F000F0u) * 0x104u) & 0x81C081C0u;    // nibbles 1, 5
+  const uint32_t p26 = ((x8 & 0x000F000Fu) * 0x1040u) & 0x81C081C0u;  // nibbles 2, 6
+  const uint32_t p37 = ((x8 & 0x00F000F0u) * 0x104u) & 0x81C081C0u;   // nibbles 3, 7
+  w[0] = mul_bf16x2(prmt(p04, p15, 0x5410u), s2);
+  w[1] = mul_bf16x2(prmt(p26, p37, 0x5410u), s2);
+  w[2] = mul_bf16x2(prmt(p04, p15, 0x7632u), s2);
+  w[3] = mul_bf16x2(prmt(p26, p37, 0x7632u), s2);
 }
 
 __global__ void __launch_bounds__(kNvfp4Threads, 1)
     lmhead_w4a16_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                              const __grid_constant__ CUtensorMap tmap_s,
                               const __grid_constant__ CUtensorMap tmap_h,
                               const Nvfp4HeadParams p) {
+  static_assert(kDequantGroups == 2, "one TMEM weight slot per dequantiser group");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_up_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int S = p.stages;
+  const uint32_t sub_bytes = nvfp4_hid_sub_bytes(p.bn);
   const uint32_t stage_bytes = nvfp4_stage_bytes(p.bn);
-  const uint32_t off_b = p.a_bytes;
-  const uint32_t off_q = p.a_bytes + p.b_bytes;
-  const uint32_t off_s = off_q + p.raw_bytes;
+  const uint32_t off_q = kRawK * sub_bytes;
+  const uint32_t off_s = off_q + kRawCodeBytes;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t deq0 = smem_u32(bars + S);
-  const uint32_t empty0 = smem_u32(bars + 2 * S);
-  const uint32_t tfull0 = smem_u32(bars + 3 * S);
-  const uint32_t tempty0 = smem_u32(bars + 3 * S + 2);
-  const uint32_t done_bar = smem_u32(bars + 3 * S + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  const uint32_t empty0 = smem_u32(bars + S);
+  const uint32_t afull0 = smem_u32(bars + 2 * S);
+  const uint32_t aempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S + 4);
+  const uint32_t tempty0 = smem_u32(bars + 2 * S + 6);
+  const uint32_t done_bar = smem_u32(bars + 2 * S + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full0 + 8 * s, 1 + 32);  // expect_tx arrive + 32 scale-copy arrivals
-      mbar_init(deq0 + 8 * s, kDequantThreads);
-      mbar_init(empty0 + 8 * s, 1);
+      // expect_tx arrive (+ 32 scale-copy arrivals when the scales come by async copies)
+      mbar_init(full0 + 8 * s, p.scale_tma ? 1 : 1 + 32);
+      // the dequantisers have read the codes and the MMAs have read the hidden rows
+      mbar_init(empty0 + 8 * s, kDequantThreads + 1);
     }
     for (int a = 0; a < 2; ++a) {
+      mbar_init(afull0 + 8 * a, kDequantThreads);
+      mbar_init(aempty0 + 8 * a, 1);
       mbar_init(tfull0 + 8 * a, 1);
       mbar_init(tempty0 + 8 * a, kEpilogueThreads);
     }
@@ -132,10 +217,11 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_q);
+    if (p.scale_tma) prefetch_tmap(&tmap_s);
     prefetch_tmap(&tmap_h);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -143,60 +229,69 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const int64_t scale_pitch = p.H / 16;
+  const int my_tiles = sched_count(p.sched);
+  const int n_raw = (p.num_kb + kRawK - 1) / kRawK;  // stages per tile
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_w = l2_policy_weights();
     const uint64_t pol_h = l2_policy_evict_last();
-    const uint32_t tx_bytes = p.raw_bytes + p.b_bytes;
-    int stage = 0;
-    uint32_t phase = 0;
-    int issued = 0;
+    const uint32_t hid_tx = (uint32_t)p.hid_rows * kBK * 2;
+    int gr = 0;  // stages issued so far
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      const int vt = tile / p.n_rtiles;
-      const int rt = tile - vt * p.n_rtiles;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!wait_bounded(empty0 + 8 * stage, phase ^ 1u, p.wait, abort_flag)) {
+    for (int t = 0; ok && t < my_tiles; ++t) {
+      const TileCoord tc = sched_tile(p.sched, p.V, t);
+      for (int r = 0; r < n_raw; ++r, ++gr) {
+        const int st = gr % S;
+        if (!wait_bounded(empty0 + 8 * st, ((uint32_t)(gr / S) & 1u) ^ 1u, p.wait,
+                          abort_flag)) {
           fail(kRoleProducer, abort_flag);
           ok = false;
           break;
         }
+        const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
         if (!p.wait.starve_loads) {
-          const uint32_t full = full0 + 8 * stage;
-          const uint32_t sbase = smem_u32(smem + (size_t)stage * stage_bytes);
+          const uint32_t full = full0 + 8 * st;
+          const uint32_t sbase = smem_u32(smem + (size_t)st * stage_bytes);
           if (lane == 0) {
-            mbar_arrive_expect_tx(full, tx_bytes);
-            tma_load_2d(sbase + off_q, &tmap_q, full, kb * (kBK / 2), vt * kBM, pol_w);
-            tma_load_2d(sbase + off_b, &tmap_h, full, kb * kBK, rt * p.bn, pol_h);
+            mbar_arrive_expect_tx(full, kRawCodeBytes + (p.scale_tma ? kRawScaleBytes : 0u) +
+                                            (uint32_t)nk * hid_tx);
+            tma_load_2d(sbase + off_q, &tmap_q, full, tma_x(r * (kRawK * kBK / 2), 1),
+                        (int32_t)tc.v0, pol_w);
+            if (p.scale_tma)
+              tma_load_2d(sbase + off_s, &tmap_s, full, tma_x(r * (kRawK * 4), 1),
+                          (int32_t)tc.v0, pol_w);
+            for (int j = 0; j < nk; ++j)
+              tma_load_2d(sbase + (uint32_t)j * sub_bytes, &tmap_h, full,
+                          tma_x((r * kRawK + j) * kBK * 2, 2), (int32_t)tc.r0, pol_h);
           }
-          // Block scales: 4 bytes (one K step) for each of the 128 rows, 4 rows per lane.
+          if (!p.scale_tma) {
+            // 4 rows per lane, 4 K steps of 4 bytes each; rows past V and K steps past H copy
+            // nothing (zero-filled).
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = lane * 4 + i;
-            const int64_t v = (int64_t)vt * kBM + row;
-            const bool in = v < p.V;
-            const uint8_t* src = p.scales + (in ? v : 0) * scale_pitch + (int64_t)kb * 4;
-            cp_async_4(sbase + off_s + (uint32_t)row * 4, src, in ? 4u : 0u);
+            for (int i = 0; i < 4; ++i) {
+              const int row = lane * 4 + i;
+              const bool in_row = tc.v0 + row < p.V;
+#pragma unroll
+              for (int j = 0; j < kRawK; ++j) {
+                const bool in = in_row && j < nk;
+                const uint8_t* src =
+                    p.scales +
+                    (in ? (tc.v0 + row) * scale_pitch + (int64_t)(r * kRawK + j) * 4 : 0);
+                cp_async_4(sbase + off_s + (uint32_t)(row * 16 + j * 4), src, in ? 4u : 0u);
+              }
+            }
+            cp_async_arrive_noinc(full);
           }
-          cp_async_arrive_noinc(full);
         }
         __syncwarp();
-        ++issued;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
     }
+    // Drain: wait for the loads of the last stages issued.
     if (!p.wait.starve_loads) {
-      const int outstanding = issued < S ? issued : S;
-      for (int i = 0; i < outstanding; ++i) {
-        if (--stage < 0) {
-          stage = S - 1;
-          phase ^= 1u;
-        }
-        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, nullptr)) {
+      for (int i = 1; i <= (gr < S ? gr : S); ++i) {
+        const int g = gr - i;
+        if (!wait_bounded(full0 + 8 * (g % S), (uint32_t)(g / S) & 1u, p.wait, nullptr)) {
           fail(kRoleDrain, abort_flag);
           break;
         }
@@ -205,41 +300,45 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
-    int stage = 0;
-    uint32_t phase = 0;
+    int gr = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int t = 0; ok && t < my_tiles; ++t) {
       if (!wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, p.wait, abort_flag)) {
         fail(kRoleMma, abort_flag);
         break;
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, abort_flag) ||
-            !wait_bounded(deq0 + 8 * stage, phase, p.wait, abort_flag)) {
+      for (int r = 0; r < n_raw; ++r, ++gr) {
+        const int st = gr % S;
+        const int slot = gr & 1;
+        if (!wait_bounded(full0 + 8 * st, (uint32_t)(gr / S) & 1u, p.wait, abort_flag) ||
+            !wait_bounded(afull0 + 8 * slot, (uint32_t)(gr >> 1) & 1u, p.wait, abort_flag)) {
           fail(kRoleMma, abort_flag);
           ok = false;
           break;
         }
         tc_fence_after_sync();
         if (lane == 0) {
-          const uint32_t sa = smem_u32(smem + (size_t)stage * stage_bytes);
-          const uint32_t sb = sa + off_b;
+          const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
+          const uint32_t sb = smem_u32(smem + (size_t)st * stage_bytes);
+          const uint64_t bdesc0 = sdesc_kmajor_sw128(sb);
+          const uint32_t a0 = tmem_base + kAColBase + (uint32_t)slot * kSlotCols;
+          for (int j = 0; j < nk; ++j) {
 #pragma unroll
-          for (int k = 0; k < kBK / kUK; ++k) {
-            mma_bf16_ss(d_tmem, sdesc_kmajor_sw128(sa + k * kUK * 2),
-                        sdesc_kmajor_sw128(sb + k * kUK * 2), idesc, (kb | k) != 0);
+            for (int k = 0; k < kBK / kUK; ++k) {
+              // descriptor start addresses are in 16-byte units
+              mma_bf16_ts(d_tmem, a0 + (uint32_t)(j * (kBK / 2) + k * (kUK / 2)),
+                          bdesc0 + (uint64_t)((j * sub_bytes + k * kUK * 2) >> 4), idesc,
+                          (r | j | k) != 0);
+            }
           }
-          mma_commit(empty0 + 8 * stage);
+          mma_commit(empty0 + 8 * st);
+          mma_commit(aempty0 + 8 * slot);
         }
         __syncwarp();
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
       if (!ok) break;
       if (lane == 0) mma_commit(tfull0 + 8 * acc);
@@ -256,18 +355,17 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     const int v_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int vt = tile / p.n_rtiles;
-      const int rt = tile - vt * p.n_rtiles;
-      if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag)) {
+    for (int t = 0; t < my_tiles; ++t) {
+      const TileCoord tc = sched_tile(p.sched, p.V, t);
+      if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag, kSleepHintNs)) {
         fail(kRoleEpilogue, abort_flag);
         break;
       }
       tc_fence_after_sync();
-      const int64_t v = (int64_t)vt * kBM + v_local;
-      const int64_t r0 = (int64_t)rt * p.bn;
+      const int64_t v = tc.v0 + v_local;
+      const int64_t r0 = tc.r0;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.bn);
-      const bool v_ok = v < p.V;
+      const bool v_ok = v_local < tc.vrows;
       for (int c = 0; c < p.bn; c += 16) {
         if (r0 + c >= p.rows) break;
         uint32_t r[16];
@@ -278,7 +376,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (r0 + c + j < p.rows) {
-              const float y = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), p.gscale), p.alpha);
+              const float a = __fmul_rn(__uint_as_float(r[j]), 128.0f);  // undo the 2^-7
+              const float y = __fmul_rn(__fmul_rn(a, p.gscale), p.alpha);
               dst[(int64_t)j * p.V] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
             }
           }
@@ -291,49 +390,53 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------------- dequantisers
-    // Thread -> (row, half): 16 rows per warp, two threads per row, each 32 elements (16 code
-    // bytes, two scale blocks). A quarter-warp covers 128 contiguous code bytes (no bank
-    // conflicts), and its 16-byte stores land in 8 distinct swizzled chunks.
-    const int dw = warp - kDequantWarp0;
-    const int row = dw * 16 + (lane >> 1);
-    const int half = lane & 1;
-    const uint32_t sw = (uint32_t)(row & 7);
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, abort_flag)) {
-          fail(kRoleDequant, abort_flag);
-          ok = false;
-          break;
-        }
-        uint8_t* sbase = smem + (size_t)stage * stage_bytes;
-        const uint4 codes = *reinterpret_cast<const uint4*>(sbase + off_q + row * 32 + half * 16);
-        const uint32_t sc = *reinterpret_cast<const uint16_t*>(sbase + off_s + row * 4 + half * 2);
-        const uint32_t s_lo = scale_bf16x2_shifted(sc & 0xFFu);
-        const uint32_t s_hi = scale_bf16x2_shifted(sc >> 8);
-        const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-        uint8_t* arow = sbase + row * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 16-byte chunk = 8 elements = 4 code bytes
-          const uint32_t s2 = q < 2 ? s_lo : s_hi;
-          uint4 o;
-          o.x = dequant_pair(cw[q] & 0xFFu, s2);
-          o.y = dequant_pair((cw[q] >> 8) & 0xFFu, s2);
-          o.z = dequant_pair((cw[q] >> 16) & 0xFFu, s2);
-          o.w = dequant_pair(cw[q] >> 24, s2);
-          const uint32_t chunk = (uint32_t)(half * 4 + q);
-          *reinterpret_cast<uint4*>(arow + ((chunk ^ sw) << 4)) = o;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(deq0 + 8 * stage);
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
+    // Group g converts stages g, g + 2, ... into TMEM weight slot g; each thread one weight
+    // row, 64 elements per K step. The stores of a stage are waited for once, at its end.
+    const int group = (warp - kDequantWarp0) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t sw = (uint32_t)(row & 7);  // 128-byte swizzle of the codes box
+    const uint32_t t_slot =
+        tmem_base + ((uint32_t)(quarter * 32) << 16) + kAColBase + (uint32_t)group * kSlotCols;
+    const int total_raw = my_tiles * n_raw;
+    for (int gr = group; gr < total_raw; gr += kDequantGroups) {
+      const int st = gr % S;
+      const int r = gr % n_raw;
+      const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
+      if (!wait_bounded(full0 + 8 * st, (uint32_t)(gr / S) & 1u, p.wait, abort_flag) ||
+          !wait_bounded(aempty0 + 8 * group, ((uint32_t)(gr >> 1) & 1u) ^ 1u, p.wait,
+                        abort_flag)) {
+        fail(kRoleDequant, abort_flag);
+        break;
       }
-      if (!ok) break;
+      tc_fence_after_sync();
+      const uint8_t* sbase = smem + (size_t)st * stage_bytes;
+      const uint8_t* crow = sbase + off_q + row * 128;
+      const uint4 sc4 = *reinterpret_cast<const uint4*>(sbase + off_s + row * 16);
+      const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+      for (int j = 0; j < nk; ++j) {
+        const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2u * j) ^ sw) << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2u * j + 1u) ^ sw) << 4));
+        const uint32_t sc = scw[j];
+        uint32_t w[32];
+        const uint32_t s0 = scale_bf16x2(sc & 0xFFu);
+        dequant8(c0.x, s0, w + 0);
+        dequant8(c0.y, s0, w + 4);
+        const uint32_t s1 = scale_bf16x2((sc >> 8) & 0xFFu);
+        dequant8(c0.z, s1, w + 8);
+        dequant8(c0.w, s1, w + 12);
+        const uint32_t s2 = scale_bf16x2((sc >> 16) & 0xFFu);
+        dequant8(c1.x, s2, w + 16);
+        dequant8(c1.y, s2, w + 20);
+        const uint32_t s3 = scale_bf16x2(sc >> 24);
+        dequant8(c1.z, s3, w + 24);
+        dequant8(c1.w, s3, w + 28);
+        tmem_st_32x32b_x32(t_slot + (uint32_t)j * (kBK / 2), w);
+      }
+      mbar_arrive(empty0 + 8 * st);  // this row's codes and scales are in registers
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(afull0 + 8 * group);
     }
   }
 
@@ -341,7 +444,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

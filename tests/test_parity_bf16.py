@@ -122,6 +122,21 @@ def test_row_count_and_position_invariance():
     assert np.array_equal(f32_bits(shuffled), f32_bits(full[perm]))
 
 
+def test_vocab_position_invariance():
+    """A vocab row's logits do not depend on where it sits in W (which TMEM lane of which tile,
+    full or partial): rolling W by rows that are not multiples of 16 or 128 rolls the logits."""
+    rows, H, V = 5, 192, 1000
+    h = synth.hidden(rows, H, 41)
+    w = synth.weight(V, H, 0.02, 41)
+    base = gpu_bf16_f32(h, w, 0.125)
+    for shift in (1, 37, 128 + 5, 500):
+        rolled = gpu_bf16_f32(h, np.roll(w, shift, axis=0), 0.125)
+        assert np.array_equal(f32_bits(rolled), f32_bits(np.roll(base, shift, axis=1))), shift
+    # the same rows inside a 300-row call (round-robin tiles) and a 5-row call (strips)
+    many = gpu_bf16_f32(np.concatenate([h, synth.hidden(295, H, 42)]), w, 0.125)
+    assert np.array_equal(f32_bits(many[:rows]), f32_bits(base))
+
+
 def test_deterministic_and_no_writes_outside_logits():
     rows, H, V = 70, 256, 333
     h = dev_bf16(synth.hidden(rows, H, 8))
