@@ -163,19 +163,21 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        if (lane == 0) {
+        {
           const uint32_t sa = smem_u32(stage_base + (size_t)stage * p.stage_bytes);
-          const uint32_t sb = sa + NSUB * a_sub;
+          const uint64_t adesc0 = sdesc_kmajor_sw128(sa);
+          const uint64_t bdesc0 = sdesc_kmajor_sw128(sa + NSUB * a_sub);
 #pragma unroll
           for (int j = 0; j < NSUB; ++j) {
 #pragma unroll
             for (int k = 0; k < kBK / kUK; ++k) {
-              mma_bf16_ss(d_tmem, sdesc_kmajor_sw128(sa + j * a_sub + k * kUK * 2),
-                          sdesc_kmajor_sw128(sb + j * b_sub + k * kUK * 2), idesc,
-                          (ks | j | k) != 0);
+              // descriptor start addresses are in 16-byte units
+              mma_bf16_ss_elect(d_tmem, adesc0 + (uint64_t)((j * a_sub + k * kUK * 2) >> 4),
+                                bdesc0 + (uint64_t)((j * b_sub + k * kUK * 2) >> 4), idesc,
+                                (ks | j | k) != 0);
             }
           }
-          mma_commit(empty0 + 8 * stage);
+          mma_commit_elect(empty0 + 8 * stage);
         }
         __syncwarp();
         if (++stage == S) {
@@ -184,13 +186,13 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         }
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(tfull0 + 8 * acc);
+      mma_commit_elect(tfull0 + 8 * acc);
       __syncwarp();
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    // Every MMA this thread issued must finish before TMEM is released.
-    if (lane == 0) mma_commit(done_bar);
+    // Every MMA this warp issued must finish before TMEM is released.
+    mma_commit_elect(done_bar);
     __syncwarp();
     if (!wait_bounded(done_bar, 0, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
   } else {

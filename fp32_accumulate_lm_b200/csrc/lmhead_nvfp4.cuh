@@ -86,13 +86,16 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate. Called by a whole converged
+// warp; one elected lane issues it, so the operands stay warp-uniform.
+__device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           break;
         }
         tc_fence_after_sync();
-        if (lane == 0) {
+        {
           const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
           const uint32_t sb = smem_u32(smem + (size_t)st * stage_bytes);
           const uint64_t bdesc0 = sdesc_kmajor_sw128(sb);
@@ -330,23 +333,23 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
 #pragma unroll
             for (int k = 0; k < kBK / kUK; ++k) {
               // descriptor start addresses are in 16-byte units
-              mma_bf16_ts(d_tmem, a0 + (uint32_t)(j * (kBK / 2) + k * (kUK / 2)),
-                          bdesc0 + (uint64_t)((j * sub_bytes + k * kUK * 2) >> 4), idesc,
-                          (r | j | k) != 0);
+              mma_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2) + k * (kUK / 2)),
+                                bdesc0 + (uint64_t)((j * sub_bytes + k * kUK * 2) >> 4), idesc,
+                                (r | j | k) != 0);
             }
           }
-          mma_commit(empty0 + 8 * st);
-          mma_commit(aempty0 + 8 * slot);
+          mma_commit_elect(empty0 + 8 * st);
+          mma_commit_elect(aempty0 + 8 * slot);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(tfull0 + 8 * acc);
+      mma_commit_elect(tfull0 + 8 * acc);
       __syncwarp();
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    if (lane == 0) mma_commit(done_bar);
+    mma_commit_elect(done_bar);
     __syncwarp();
     if (!wait_bounded(done_bar, 0, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
   } else if (warp < kDequantWarp0) {
