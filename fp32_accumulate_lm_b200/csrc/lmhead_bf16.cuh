@@ -169,13 +169,9 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           const uint64_t bdesc0 = sdesc_kmajor_sw128(sa + NSUB * a_sub);
 #pragma unroll
           for (int j = 0; j < NSUB; ++j) {
-#pragma unroll
-            for (int k = 0; k < kBK / kUK; ++k) {
-              // descriptor start addresses are in 16-byte units
-              mma_bf16_ss_elect(d_tmem, adesc0 + (uint64_t)((j * a_sub + k * kUK * 2) >> 4),
-                                bdesc0 + (uint64_t)((j * b_sub + k * kUK * 2) >> 4), idesc,
-                                (ks | j | k) != 0);
-            }
+            // descriptor start addresses are in 16-byte units
+            mma4_bf16_ss_elect(d_tmem, adesc0 + (uint64_t)((j * a_sub) >> 4),
+                               bdesc0 + (uint64_t)((j * b_sub) >> 4), idesc, (ks | j) != 0);
           }
           mma_commit_elect(empty0 + 8 * stage);
         }

@@ -100,6 +100,26 @@ __device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tm
       : "memory");
 }
 
+// One K step of 64 with A from TMEM: four K = 16 MMAs, A advancing 8 columns and B 32 bytes per
+// MMA; only the first may start a fresh accumulator. One elected lane of a converged warp
+// issues them.
+__device__ __forceinline__ void mma4_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "add.s32 a1, %1, 8;\n\tadd.s32 a2, %1, 16;\n\tadd.s32 a3, %1, 24;\n\t"
+      "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -330,13 +350,9 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           const uint64_t bdesc0 = sdesc_kmajor_sw128(sb);
           const uint32_t a0 = tmem_base + kAColBase + (uint32_t)slot * kSlotCols;
           for (int j = 0; j < nk; ++j) {
-#pragma unroll
-            for (int k = 0; k < kBK / kUK; ++k) {
-              // descriptor start addresses are in 16-byte units
-              mma_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2) + k * (kUK / 2)),
-                                bdesc0 + (uint64_t)((j * sub_bytes + k * kUK * 2) >> 4), idesc,
-                                (r | j | k) != 0);
-            }
+            // descriptor start addresses are in 16-byte units
+            mma4_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2)),
+                               bdesc0 + (uint64_t)((j * sub_bytes) >> 4), idesc, (r | j) != 0);
           }
           mma_commit_elect(empty0 + 8 * st);
           mma_commit_elect(aempty0 + 8 * slot);
