@@ -45,7 +45,37 @@ WORKLOAD_TEXT = {
     "prefill": "prefill LM head: rows=8192, H=4096, V=151936, bf16 in, fp32 out, alpha=1/8",
     "nvfp4": "NVFP4 W4A16 head: rows {1,16,64,65,256}, H=2048, V=151936, E2M1 + E4M3/16 + fp32 "
              "scale, bf16 hidden and logits, alpha=1/8",
+    "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
+                    "fp32 out, alpha=1/8",
 }
+
+
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources and the public header (what a traffic figure is tied to)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(_ROOT, "fp32_accumulate_lm_b200", "csrc", "*")) +
+                   glob.glob(os.path.join(_ROOT, "include", "*.h")))
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) from profiles/traffic.json, if it was captured from
+    the current kernel sources; None otherwise."""
+    try:
+        with open(os.path.join(_ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get(kernel, {}).get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
 
 
 def load_peaks() -> dict:
@@ -128,7 +158,8 @@ class Workload:
         rows_list, H, V, std, alpha = synth.WORKLOADS[name]
         self.rows_list, self.H, self.V, self.alpha = rows_list, H, V, alpha
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
-                "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4}[name]
+                "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
+                "prefill_2048": synth.SEED_PREFILL}[name]
         rmax = max(rows_list)
         self.hidden = synth.hidden(rmax, H, seed, device=device)
         self.nvfp4 = name == "nvfp4"
@@ -254,7 +285,7 @@ def run_ours(args) -> dict | None:
         tot_bytes += b
         tot_flops += fl
         tot_ms += mean_ms
-    tensor_bound = args.workload == "prefill"
+    tensor_bound = args.workload.startswith("prefill")
     if tensor_bound:
         achieved = tot_flops / (tot_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -266,9 +297,10 @@ def run_ours(args) -> dict | None:
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": f"HBM copy ({peaks['source']})"}
-    roof["traffic"] = None
-    roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
     roof["kernel"] = "lmhead_w4a16_nvfp4_kernel" if wl.nvfp4 else "lmhead_bf16_f32_kernel"
+    roof["traffic"] = recorded_traffic(roof["kernel"], args.workload)
+    roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
+    roof["source_hash"] = kernel_source_hash()
 
     # ---- end to end through the C ABI: pinned host hidden -> device, call, logits -> pinned host
     e2e = run_e2e(args, wl, world)

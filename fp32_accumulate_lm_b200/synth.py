@@ -38,6 +38,8 @@ WORKLOADS = {
     "spec_verify": ([128, 97, 32], 4096, 128256, 0.015, 1.0 / 16),
     "prefill": ([8192], 4096, 151936, 0.02, 1.0 / 8),
     "nvfp4": ([1, 16, 64, 65, 256], 2048, 151936, 0.02, 1.0 / 8),
+    # profiling case: the prefill kernel and tile shape on 2048 rows (a few GB on the device)
+    "prefill_2048": ([2048], 4096, 151936, 0.02, 1.0 / 8),
 }
 
 
