@@ -48,8 +48,19 @@ struct DeviceInfo {
   bool arch_ok = false;
   bool attrs_set = false;
   int num_sms = 0;
-  int smem_optin = 0;
+  int smem_optin = 0;        // per-block shared-memory opt-in limit (static + dynamic)
+  int nvfp4_static_smem = 0;  // static shared memory of the NVFP4 kernel
 };
+
+// Let `kernel` use every byte of shared memory the device allows beside its static part.
+template <typename K>
+bool raise_smem_limit(K kernel, int optin, int* static_bytes) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+  if (static_bytes) *static_bytes = (int)a.sharedSizeBytes;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - (int)a.sharedSizeBytes) == cudaSuccess;
+}
 
 std::mutex g_mu;
 DeviceInfo g_devices[kMaxDevices];
@@ -90,18 +101,11 @@ int current_device(DeviceInfo* out) {
   }
   if (!d.arch_ok) return LMHEAD_ERR_ARCH;
   if (!d.attrs_set) {
-    if (cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<1>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<2>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(lmh::lmhead_bf16_f32_kernel<4>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(lmh::lmhead_w4a16_nvfp4_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess) {
+    if (!raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<4>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel, d.smem_optin,
+                          &d.nvfp4_static_smem)) {
       return LMHEAD_ERR_LAUNCH;
     }
     d.attrs_set = true;
@@ -327,10 +331,11 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.num_kb = (int32_t)(H / lmh::kBK);
   const int reserve = 1024 + 512;
   const int stage_bytes = (int)lmh::nvfp4_stage_bytes(p.bn);
-  int stages = (dev.smem_optin - reserve) / stage_bytes;
+  int stages = (dev.smem_optin - dev.nvfp4_static_smem - reserve) / stage_bytes;
   if (stages > 8) stages = 8;
   if (stages < 2) return LMHEAD_ERR_SHAPE;
   p.stages = stages;
+  p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
   // Block scales come by TMA when each scale row is a whole number of 16-byte units.
   p.scale_tma = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? 1 : 0;
   p.wait = wait_cfg();

@@ -43,7 +43,9 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
                            const __grid_constant__ CUtensorMap tmap_h, const Bf16HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_up_1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
+  // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
+  // counters and descriptors in uniform registers.
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int S = p.stages;
 

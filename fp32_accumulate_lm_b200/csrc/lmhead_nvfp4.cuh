@@ -21,14 +21,17 @@
 //   stage (shared memory) 4 K steps of: the packed codes [128 rows x 128 bytes] in one box,
 //         their block scales [128 rows x 16 bytes] (TMA when the scale pitch allows, 4-byte
 //         async copies otherwise) and the hidden rows [BN x 64] x 4.
-//   slot  (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; two slots.
+//   slot  (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; a ring of 3
+//         slots (2 when the row tile is 128), so refilling a slot never waits for the MMAs
+//         that were just issued.
 // Roles (192 + 128 * kDequantGroups threads):
 //   warp 0      producer: fills stages.
 //   warp 1      TMEM allocator and MMA issuer: per stage waits for it and for its weight slot,
 //               16 x tcgen05.mma with A from TMEM, one commit frees each.
 //   warps 2-5   epilogue.
 //   warps 6-13  dequantisers: two groups of four warps (one per TMEM lane quarter); group g
-//               takes stages g, g + 2, ... into slot g. Each thread converts one weight row.
+//               takes stages g, g + 2, ...; stage i goes to slot i mod slots. Each thread
+//               converts one weight row.
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -44,7 +47,7 @@ constexpr int kDequantWarp0 = 6;
 constexpr int kDequantThreads = 128;                    // threads that fill one K step
 constexpr int kNvfp4Threads = 32 * kDequantWarp0 + kDequantThreads * kDequantGroups;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAColBase = 256;  // TMEM columns [256, 512): two dequantised weight slots
+constexpr int kMaxSlots = 3;         // dequantised weight slots at the top of TMEM
 constexpr int kBnMax = 128;          // row tile cap: two accumulators of <= 128 columns
 
 constexpr int kRawK = 4;                                  // K steps per stage
@@ -63,6 +66,7 @@ struct Nvfp4HeadParams {
   TileSched sched;
   int32_t num_kb;         // K steps of 64 per tile (H / 64)
   int32_t stages;
+  int32_t slots;          // TMEM weight slots: 3 when 2 * bn + 3 * 128 <= 512, else 2
   int32_t scale_tma;      // 1: block scales by TMA (H % 256 == 0), 0: 4-byte async copies
   WaitCfg wait;
 };
@@ -117,6 +121,55 @@ __device__ __forceinline__ void mma4_bf16_ts_elect(uint32_t d_tmem, uint32_t a_t
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, 1;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, 1;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// A whole stage (4 K steps of 64 = 16 MMAs) from one asm block: A advances 8 TMEM columns per
+// MMA, B 32 bytes per MMA within a sub-tile and `b_sub` bytes (>> 4 in `b_step`) per K step.
+// Only the very first MMA may start a fresh accumulator.
+__device__ __forceinline__ void mma16_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                    uint64_t b_desc, uint32_t b_step,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 a;\n\t.reg .b64 b, bk;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "cvt.u64.u32 bk, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
+      "add.s32 a, %1, 8;\n\tadd.s64 b, %2, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 16;\n\tadd.s64 b, %2, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 24;\n\tadd.s64 b, %2, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s64 b, %2, bk;\n\t"
+      "add.s32 a, %1, 32;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 40;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 48;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 56;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s64 bk, bk, bk;\n\tadd.s64 b, %2, bk;\n\t"
+      "add.s32 a, %1, 64;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 72;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 80;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 88;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "cvt.u64.u32 bk, %3;\n\tmul.lo.u64 bk, bk, 3;\n\tadd.s64 b, %2, bk;\n\t"
+      "add.s32 a, %1, 96;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 104;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 112;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t"
+      "add.s32 a, %1, 120;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(b_step), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -199,10 +252,12 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                               const __grid_constant__ CUtensorMap tmap_s,
                               const __grid_constant__ CUtensorMap tmap_h,
                               const Nvfp4HeadParams p) {
-  static_assert(kDequantGroups == 2, "one TMEM weight slot per dequantiser group");
   extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119
   uint8_t* smem = align_up_1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
+  // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
+  // counters and descriptors in uniform registers.
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int S = p.stages;
   const uint32_t sub_bytes = nvfp4_hid_sub_bytes(p.bn);
@@ -214,11 +269,13 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + S);
   const uint32_t afull0 = smem_u32(bars + 2 * S);
-  const uint32_t aempty0 = smem_u32(bars + 2 * S + 2);
-  const uint32_t tfull0 = smem_u32(bars + 2 * S + 4);
-  const uint32_t tempty0 = smem_u32(bars + 2 * S + 6);
-  const uint32_t done_bar = smem_u32(bars + 2 * S + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
+  const uint32_t aempty0 = smem_u32(bars + 2 * S + kMaxSlots);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S + 2 * kMaxSlots);
+  const uint32_t tempty0 = smem_u32(bars + 2 * S + 2 * kMaxSlots + 2);
+  const uint32_t done_bar = smem_u32(bars + 2 * S + 2 * kMaxSlots + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kMaxSlots + 5);
+  const int NA = p.slots;
+  const uint32_t slot_col0 = kTmemCols - (uint32_t)NA * kSlotCols;  // weight slots at the top
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -228,9 +285,11 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       // the dequantisers have read the codes and the MMAs have read the hidden rows
       mbar_init(empty0 + 8 * s, kDequantThreads + 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kMaxSlots; ++a) {
       mbar_init(afull0 + 8 * a, kDequantThreads);
       mbar_init(aempty0 + 8 * a, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
       mbar_init(tempty0 + 8 * a, kEpilogueThreads);
     }
@@ -247,6 +306,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) scale_lut[c] = scale_bf16x2((uint32_t)c);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -261,13 +321,13 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     const uint64_t pol_h = l2_policy_evict_last();
     const uint32_t hid_tx = (uint32_t)p.hid_rows * kBK * 2;
     int gr = 0;  // stages issued so far
+    int st = 0;
+    uint32_t ph = 0;
     bool ok = true;
     for (int t = 0; ok && t < my_tiles; ++t) {
       const TileCoord tc = sched_tile(p.sched, p.V, t);
       for (int r = 0; r < n_raw; ++r, ++gr) {
-        const int st = gr % S;
-        if (!wait_bounded(empty0 + 8 * st, ((uint32_t)(gr / S) & 1u) ^ 1u, p.wait,
-                          abort_flag)) {
+        if (!wait_bounded(empty0 + 8 * st, ph ^ 1u, p.wait, abort_flag)) {
           fail(kRoleProducer, abort_flag);
           ok = false;
           break;
@@ -308,13 +368,20 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           }
         }
         __syncwarp();
+        if (++st == S) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
     }
     // Drain: wait for the loads of the last stages issued.
     if (!p.wait.starve_loads) {
-      for (int i = 1; i <= (gr < S ? gr : S); ++i) {
-        const int g = gr - i;
-        if (!wait_bounded(full0 + 8 * (g % S), (uint32_t)(g / S) & 1u, p.wait, nullptr)) {
+      for (int i = 0; i < (gr < S ? gr : S); ++i) {
+        if (--st < 0) {
+          st = S - 1;
+          ph ^= 1u;
+        }
+        if (!wait_bounded(full0 + 8 * st, ph, p.wait, nullptr)) {
           fail(kRoleDrain, abort_flag);
           break;
         }
@@ -324,6 +391,10 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
     int gr = 0;
+    int st = 0;
+    uint32_t ph = 0;
+    int sl = 0;  // weight slot of stage gr, and its phase
+    uint32_t sph = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -335,10 +406,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
       for (int r = 0; r < n_raw; ++r, ++gr) {
-        const int st = gr % S;
-        const int slot = gr & 1;
-        if (!wait_bounded(full0 + 8 * st, (uint32_t)(gr / S) & 1u, p.wait, abort_flag) ||
-            !wait_bounded(afull0 + 8 * slot, (uint32_t)(gr >> 1) & 1u, p.wait, abort_flag)) {
+        if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag) ||
+            !wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag)) {
           fail(kRoleMma, abort_flag);
           ok = false;
           break;
@@ -348,16 +417,28 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
           const uint32_t sb = smem_u32(smem + (size_t)st * stage_bytes);
           const uint64_t bdesc0 = sdesc_kmajor_sw128(sb);
-          const uint32_t a0 = tmem_base + kAColBase + (uint32_t)slot * kSlotCols;
-          for (int j = 0; j < nk; ++j) {
-            // descriptor start addresses are in 16-byte units
-            mma4_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2)),
-                               bdesc0 + (uint64_t)((j * sub_bytes) >> 4), idesc, (r | j) != 0);
+          const uint32_t a0 = tmem_base + slot_col0 + (uint32_t)sl * kSlotCols;
+          // descriptor start addresses are in 16-byte units
+          if (nk == kRawK) {
+            mma16_bf16_ts_elect(d_tmem, a0, bdesc0, sub_bytes >> 4, idesc, r != 0);
+          } else {
+            for (int j = 0; j < nk; ++j)
+              mma4_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2)),
+                                 bdesc0 + (uint64_t)((j * sub_bytes) >> 4), idesc,
+                                 (r | j) != 0);
           }
           mma_commit_elect(empty0 + 8 * st);
-          mma_commit_elect(aempty0 + 8 * slot);
+          mma_commit_elect(aempty0 + 8 * sl);
         }
         __syncwarp();
+        if (++st == S) {
+          st = 0;
+          ph ^= 1u;
+        }
+        if (++sl == NA) {
+          sl = 0;
+          sph ^= 1u;
+        }
       }
       if (!ok) break;
       mma_commit_elect(tfull0 + 8 * acc);
@@ -409,22 +490,24 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------------- dequantisers
-    // Group g converts stages g, g + 2, ... into TMEM weight slot g; each thread one weight
-    // row, 64 elements per K step. The stores of a stage are waited for once, at its end.
+    // Group g converts stages g, g + 2, ...; stage i goes to TMEM weight slot i mod slots. Each
+    // thread converts one weight row, 64 elements per K step; the stores of a stage are waited
+    // for once, at its end.
     const int group = (warp - kDequantWarp0) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t sw = (uint32_t)(row & 7);  // 128-byte swizzle of the codes box
-    const uint32_t t_slot =
-        tmem_base + ((uint32_t)(quarter * 32) << 16) + kAColBase + (uint32_t)group * kSlotCols;
+    const uint32_t t_slots = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot_col0;
     const int total_raw = my_tiles * n_raw;
+    int st = group % S;             // stage and phase of stage index gr, advanced by the group
+    uint32_t ph = (uint32_t)(group / S) & 1u;  // count each iteration (no divisions in the loop)
+    int r = group % n_raw;          // stage within its tile
+    int sl = group % NA;            // weight slot of stage gr, and its phase
+    uint32_t sph = (uint32_t)(group / NA) & 1u;
     for (int gr = group; gr < total_raw; gr += kDequantGroups) {
-      const int st = gr % S;
-      const int r = gr % n_raw;
       const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
-      if (!wait_bounded(full0 + 8 * st, (uint32_t)(gr / S) & 1u, p.wait, abort_flag) ||
-          !wait_bounded(aempty0 + 8 * group, ((uint32_t)(gr >> 1) & 1u) ^ 1u, p.wait,
-                        abort_flag)) {
+      if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag) ||
+          !wait_bounded(aempty0 + 8 * sl, sph ^ 1u, p.wait, abort_flag)) {
         fail(kRoleDequant, abort_flag);
         break;
       }
@@ -438,24 +521,36 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2u * j + 1u) ^ sw) << 4));
         const uint32_t sc = scw[j];
         uint32_t w[32];
-        const uint32_t s0 = scale_bf16x2(sc & 0xFFu);
+        const uint32_t s0 = scale_lut[sc & 0xFFu];
         dequant8(c0.x, s0, w + 0);
         dequant8(c0.y, s0, w + 4);
-        const uint32_t s1 = scale_bf16x2((sc >> 8) & 0xFFu);
+        const uint32_t s1 = scale_lut[(sc >> 8) & 0xFFu];
         dequant8(c0.z, s1, w + 8);
         dequant8(c0.w, s1, w + 12);
-        const uint32_t s2 = scale_bf16x2((sc >> 16) & 0xFFu);
+        const uint32_t s2 = scale_lut[(sc >> 16) & 0xFFu];
         dequant8(c1.x, s2, w + 16);
         dequant8(c1.y, s2, w + 20);
-        const uint32_t s3 = scale_bf16x2(sc >> 24);
+        const uint32_t s3 = scale_lut[sc >> 24];
         dequant8(c1.z, s3, w + 24);
         dequant8(c1.w, s3, w + 28);
-        tmem_st_32x32b_x32(t_slot + (uint32_t)j * (kBK / 2), w);
+        tmem_st_32x32b_x32(t_slots + (uint32_t)sl * kSlotCols + (uint32_t)j * (kBK / 2), w);
       }
       mbar_arrive(empty0 + 8 * st);  // this row's codes and scales are in registers
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(afull0 + 8 * group);
+      mbar_arrive(afull0 + 8 * sl);
+      sl += kDequantGroups;
+      while (sl >= NA) {
+        sl -= NA;
+        sph ^= 1u;
+      }
+      st += kDequantGroups;
+      if (st >= S) {
+        st -= S;
+        ph ^= 1u;
+      }
+      r += kDequantGroups;
+      while (r >= n_raw) r -= n_raw;
     }
   }
 
