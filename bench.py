@@ -196,7 +196,8 @@ class Workload:
         return 2 * r * self.H * self.V
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun env). `backend` "gloo" runs the same plumbing on CPU."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -204,21 +205,29 @@ def dist_setup(n_gpus: int):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
 
-def barrier(world: int):
+def _device_sync():
     import torch
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
+
+
+def barrier(world: int):
+    """Device idle on every rank, then a process-group barrier, then idle again."""
     import torch.distributed as dist
-    torch.cuda.synchronize()
+    _device_sync()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    _device_sync()
 
 
 def max_over_ranks(x: float, world: int) -> float:
@@ -226,9 +235,15 @@ def max_over_ranks(x: float, world: int) -> float:
     import torch.distributed as dist
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_us_per_call(elapsed_ms: float, steps: int, calls_per_step: int, world: int) -> float:
+    """Whole-job time per call: the slowest rank's elapsed time over every rank's calls."""
+    return elapsed_ms * 1e3 / (steps * calls_per_step * world)
 
 
 def run_ours(args) -> dict | None:
@@ -305,7 +320,7 @@ def run_ours(args) -> dict | None:
     # ---- end to end through the C ABI: pinned host hidden -> device, call, logits -> pinned host
     e2e = run_e2e(args, wl, world)
 
-    value = elapsed_ms * 1e3 / (args.steps * calls_per_step * world)
+    value = job_us_per_call(elapsed_ms, args.steps, calls_per_step, world)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,

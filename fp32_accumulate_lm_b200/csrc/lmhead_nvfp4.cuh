@@ -38,16 +38,15 @@
 
 namespace lmh {
 
-// Dequantiser groups of four warps (build-time knob LMHEAD_NVFP4_DQ_GROUPS).
-#ifndef LMHEAD_NVFP4_DQ_GROUPS
-#define LMHEAD_NVFP4_DQ_GROUPS 2
-#endif
-constexpr int kDequantGroups = LMHEAD_NVFP4_DQ_GROUPS;  // groups take K steps in turn
+// Two dequantiser groups of four warps take stages in turn. The slot ring's phase waits assume
+// no more groups than TMEM weight slots (a group is never two uses of a slot ahead).
+constexpr int kDequantGroups = 2;
 constexpr int kDequantWarp0 = 6;
 constexpr int kDequantThreads = 128;                    // threads that fill one K step
 constexpr int kNvfp4Threads = 32 * kDequantWarp0 + kDequantThreads * kDequantGroups;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 3;         // dequantised weight slots at the top of TMEM
+static_assert(kDequantGroups <= 2, "the slot ring may have only 2 slots");
 constexpr int kBnMax = 128;          // row tile cap: two accumulators of <= 128 columns
 
 constexpr int kRawK = 4;                                  // K steps per stage
