@@ -20,7 +20,7 @@ import threading
 __all__ = [
     "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_w4a16_nvfp4",
     "lmhead_logits_bf16_f32", "lmhead_logits_w4a16_nvfp4", "status_string", "device_status",
-    "version", "set_fault_injection", "STATUS",
+    "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS",
 ]
 
 STATUS = {
@@ -69,6 +69,8 @@ def load_library():
         lib.lmhead_version.restype = i32
         lib.lmhead_debug_set_fault_injection.argtypes = [i32, ctypes.c_uint64]
         lib.lmhead_debug_set_fault_injection.restype = None
+        lib.lmhead_debug_set_nvfp4_conversion.argtypes = [i32]
+        lib.lmhead_debug_set_nvfp4_conversion.restype = None
         _lib = lib
         return lib
 
@@ -102,6 +104,11 @@ def device_status(clear: bool = False) -> int:
 
 def version() -> int:
     return load_library().lmhead_version()
+
+
+def set_nvfp4_conversion(path: int) -> None:
+    """Test hook: 1 pair table, 2 integer spreading, 0 automatic (same bits either way)."""
+    load_library().lmhead_debug_set_nvfp4_conversion(int(path))
 
 
 def set_fault_injection(starve_loads: bool, wait_limit_ns: int = 0) -> None:

@@ -36,6 +36,7 @@ constexpr CUtensorMapL2promotion kWeightPromo =
     (CUtensorMapL2promotion)(CU_TENSOR_MAP_L2_PROMOTION_NONE + LMHEAD_WEIGHT_L2_PROMOTION);
 
 std::atomic<int> g_starve_loads{0};
+std::atomic<int> g_nvfp4_path{0};  // 0: automatic, 1: pair table, 2: spread (test hook)
 std::atomic<uint64_t> g_wait_limit_ns{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -49,7 +50,8 @@ struct DeviceInfo {
   bool attrs_set = false;
   int num_sms = 0;
   int smem_optin = 0;        // per-block shared-memory opt-in limit (static + dynamic)
-  int nvfp4_static_smem = 0;  // static shared memory of the NVFP4 kernel
+  int nvfp4_static_smem = 0;  // static shared memory of the NVFP4 kernels
+  int smem_reserved = 0;      // shared memory the system reserves per block
 };
 
 // Let `kernel` use every byte of shared memory the device allows beside its static part.
@@ -93,6 +95,8 @@ int current_device(DeviceInfo* out) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
             cudaSuccess) {
       return LMHEAD_ERR_LAUNCH;
     }
@@ -104,8 +108,9 @@ int current_device(DeviceInfo* out) {
     if (!raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<4>, d.smem_optin, nullptr) ||
-        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel, d.smem_optin,
-                          &d.nvfp4_static_smem)) {
+        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<true>, d.smem_optin,
+                          &d.nvfp4_static_smem) ||
+        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<false>, d.smem_optin, nullptr)) {
       return LMHEAD_ERR_LAUNCH;
     }
     d.attrs_set = true;
@@ -150,6 +155,27 @@ int encode_rows(CUtensorMap* map, CUtensorMapDataType natural, int esize, const 
                      box_bytes / 4, box_outer, swizzle, promo);
   return encode_2d(map, natural, esize, base, inner_bytes / esize, outer, box_bytes / esize,
                    box_outer, swizzle, promo);
+}
+
+// Tensor map over hidden [rows, H] bf16 seen as [H/64 K steps][rows][64 elements]: one box
+// brings `box_k` K steps of `box_rows` rows, each K step a 128-byte-swizzled [box_rows x 128 B]
+// sub-tile, the sub-tiles back to back.
+int encode_hidden_ksteps(CUtensorMap* map, const void* hidden, int64_t rows, int64_t H,
+                         uint32_t box_rows, uint32_t box_k) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return LMHEAD_ERR_LAUNCH;
+  const int esize = LMHEAD_TMA_WIDE ? 4 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)(lmh::kBK * 2 / esize), (cuuint64_t)rows,
+                              (cuuint64_t)(H / lmh::kBK)};
+  const cuuint64_t strides[2] = {(cuuint64_t)(H * 2), (cuuint64_t)(lmh::kBK * 2)};
+  const cuuint32_t box[3] = {(cuuint32_t)(lmh::kBK * 2 / esize), box_rows, box_k};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      enc(map, LMHEAD_TMA_WIDE ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+          3, const_cast<void*>(hidden), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
 // Rows of hidden one TMA box brings: the call's rows when they fit one row tile (the MMA still
@@ -224,6 +250,10 @@ const char* lmhead_status_string(int status) {
 void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) {
   g_starve_loads.store(starve_loads ? 1 : 0);
   g_wait_limit_ns.store(wait_limit_ns);
+}
+
+void lmhead_debug_set_nvfp4_conversion(int path) {
+  g_nvfp4_path.store(path == 1 || path == 2 ? path : 0);
 }
 
 int lmhead_device_status(int clear) {
@@ -329,12 +359,23 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
   if (st != LMHEAD_OK) return st;
   p.num_kb = (int32_t)(H / lmh::kBK);
-  const int reserve = 1024 + 512;
-  const int stage_bytes = (int)lmh::nvfp4_stage_bytes(p.bn);
-  int stages = (dev.smem_optin - dev.nvfp4_static_smem - reserve) / stage_bytes;
-  if (stages > 8) stages = 8;
-  if (stages < 2) return LMHEAD_ERR_SHAPE;
-  p.stages = stages;
+  // Hidden sub-tiles start on 1024-byte swizzle atoms: rows per K step rounded up to 8.
+  p.hid_rows = rows < p.bn ? (int32_t)((rows + 7) / 8 * 8) : p.bn;
+  p.max_stages = lmh::kMaxStages;
+  // Dynamic shared memory: all the opt-in room; the kernel lays its ring out in it. The window
+  // holds the reserved block, then the static variables, then the dynamic block.
+  const int dyn_bytes = dev.smem_optin - dev.nvfp4_static_smem;
+  const uint32_t stage_bytes = lmh::nvfp4_stage_bytes(p.bn, p.hid_rows);
+  const uint32_t win_base = (uint32_t)(dev.smem_reserved + dev.nvfp4_static_smem);
+  const lmh::StageLayout with_table = lmh::nvfp4_stage_layout(
+      win_base, win_base + (uint32_t)dyn_bytes, stage_bytes, true, lmh::kMaxStages);
+  const lmh::StageLayout spread = lmh::nvfp4_stage_layout(
+      win_base, win_base + (uint32_t)dyn_bytes, stage_bytes, false, lmh::kMaxStages);
+  const int path = g_nvfp4_path.load(std::memory_order_relaxed);
+  // The pair table when it leaves room for 3 stages (both conversions give the same bits).
+  const bool use_table = path == 1 ? with_table.stages >= 2
+                                   : path == 2 ? false : with_table.stages >= 3;
+  if ((use_table ? with_table.stages : spread.stages) < 2) return LMHEAD_ERR_SHAPE;
   p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
   // Block scales come by TMA when each scale row is a whole number of 16-byte units.
   p.scale_tma = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? 1 : 0;
@@ -353,15 +394,15 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   } else {
     tmap_s = tmap_q;  // unused
   }
-  p.hid_rows = hid_box_rows(rows, p.bn);
-  st = encode_rows(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H * 2, rows,
-                   lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  st = encode_hidden_ksteps(&tmap_h, hidden, rows, H, (uint32_t)p.hid_rows, lmh::kRawK);
   if (st != LMHEAD_OK) return st;
 
-  const size_t smem = (size_t)reserve + (size_t)stages * stage_bytes;
-  lmh::lmhead_w4a16_nvfp4_kernel<<<grid, lmh::kNvfp4Threads, smem, (cudaStream_t)stream>>>(
-      tmap_q, tmap_s, tmap_h, p);
+  if (use_table)
+    lmh::lmhead_w4a16_nvfp4_kernel<true><<<grid, lmh::kNvfp4Threads, (size_t)dyn_bytes,
+                                            (cudaStream_t)stream>>>(tmap_q, tmap_s, tmap_h, p);
+  else
+    lmh::lmhead_w4a16_nvfp4_kernel<false><<<grid, lmh::kNvfp4Threads, (size_t)dyn_bytes,
+                                             (cudaStream_t)stream>>>(tmap_q, tmap_s, tmap_h, p);
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 

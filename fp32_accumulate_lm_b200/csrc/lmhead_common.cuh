@@ -48,6 +48,7 @@ enum : unsigned {
 };
 
 constexpr unsigned kStatusTimeout = 6;  // == LMHEAD_ERR_TIMEOUT
+constexpr unsigned kStatusNoRoom = 2;   // == LMHEAD_ERR_SHAPE: shared memory too small
 
 // Waits that are expected to last (the epilogue waiting for a whole tile's MMAs) let the
 // hardware suspend the thread up to this long per try instead of spinning on issue slots.

@@ -14,6 +14,17 @@
 // from the subnormal range), and the epilogue restores it exactly:
 //   logits = bf16_rn( fl32( fl32( (acc * 2^7) * g ) * alpha ) ).
 //
+// Conversion, two equivalent ways (identical bits; the host picks one per call, so a row's
+// logits do not depend on which):
+//   pair table  each byte of codes (two E2M1 values) indexes a 256-entry table of bf16x2 words
+//               in shared memory, one copy per lane so a warp's 32 lookups never share a bank.
+//               The table sits on a 64 KB boundary with entries 256 bytes apart, so one prmt
+//               builds the lookup address from the code byte and the lane's base. Three
+//               instructions per two weights (prmt, lds, one bf16x2 multiply by the scale).
+//   spread      integer multiplies spread nibbles into bf16 bit positions (dequant8 below); no
+//               table, used when the table leaves room for fewer than two stages (large row
+//               tiles).
+//
 // Every hand-off covers 4 K steps (256 elements of K). The single-thread roles (TMA producer,
 // MMA issuer) share their SM sub-partitions with busy dequantiser warps, so each of their
 // instructions is slow; paying one wait and one commit per K step of 64 made them the
@@ -26,8 +37,9 @@
 //         that were just issued.
 // Roles (192 + 128 * kDequantGroups threads):
 //   warp 0      producer: fills stages.
-//   warp 1      TMEM allocator and MMA issuer: per stage waits for it and for its weight slot,
-//               16 x tcgen05.mma with A from TMEM, one commit frees each.
+//   warp 1      TMEM allocator and MMA issuer: per stage waits for its weight slot (filled only
+//               after the dequantisers saw the stage land, so the hidden rows are there too),
+//               16 x tcgen05.mma with A from TMEM, commits free the stage and the slot.
 //   warps 2-5   epilogue.
 //   warps 6-13  dequantisers: two groups of four warps (one per TMEM lane quarter); group g
 //               takes stages g, g + 2, ...; stage i goes to slot i mod slots. Each thread
@@ -54,6 +66,10 @@ constexpr uint32_t kRawCodeBytes = kBM * kRawK * kBK / 2;  // 16 KB
 constexpr uint32_t kRawScaleBytes = kBM * kRawK * 4;       // 2 KB
 constexpr uint32_t kSlotCols = kRawK * kBK / 2;            // TMEM columns of one weight slot
 
+constexpr int kMaxStages = 8;
+constexpr uint32_t kBarrierBytes = 1024;   // barrier block at the start of dynamic smem
+constexpr uint32_t kPairTableBytes = 65536;  // 256 entries x 256 bytes, on a 64 KB boundary
+
 struct Nvfp4HeadParams {
   int64_t rows, H, V;
   uint16_t* out;          // bf16 logits
@@ -61,22 +77,56 @@ struct Nvfp4HeadParams {
   float alpha;
   float gscale;
   int32_t bn;
-  int32_t hid_rows;       // rows of hidden one TMA box brings (<= bn; MMA columns past it unused)
+  int32_t hid_rows;       // hidden rows per K step in a stage: a multiple of 8, <= bn (MMA
+                          // columns past the call's rows read neighbouring data, never stored)
   TileSched sched;
   int32_t num_kb;         // K steps of 64 per tile (H / 64)
-  int32_t stages;
+  int32_t max_stages;     // cap on the shared-memory ring; the kernel fits what room allows
   int32_t slots;          // TMEM weight slots: 3 when 2 * bn + 3 * 128 <= 512, else 2
   int32_t scale_tma;      // 1: block scales by TMA (H % 256 == 0), 0: 4-byte async copies
   WaitCfg wait;
 };
 
-// Shared-memory stage (4 K steps): [hidden: 4 sub-tiles of BN x 64 bf16, 128-byte swizzle]
-// [codes: 128 rows x 128 bytes, 128-byte swizzle][scales: 128 rows x 16 bytes]
-__host__ __device__ constexpr uint32_t nvfp4_hid_sub_bytes(int bn) {
-  return (uint32_t)(bn * kBK * 2);
+// Shared-memory stage (4 K steps): [hidden: 4 sub-tiles of hid_rows x 64 bf16, 128-byte swizzle,
+// from one 3-D box, plus room for the last sub-tile's MMA to read bn rows][codes: 128 rows x
+// 128 bytes, 128-byte swizzle][scales: 128 rows x 16 bytes]. Multiples of 1024 bytes.
+__host__ __device__ constexpr uint32_t nvfp4_hid_region_bytes(int bn, int hid_rows) {
+  return (uint32_t)(((kRawK - 1) * hid_rows + bn) * kBK * 2);
 }
-__host__ __device__ constexpr uint32_t nvfp4_stage_bytes(int bn) {
-  return (uint32_t)kRawK * nvfp4_hid_sub_bytes(bn) + kRawCodeBytes + kRawScaleBytes;
+__host__ __device__ constexpr uint32_t nvfp4_stage_bytes(int bn, int hid_rows) {
+  return nvfp4_hid_region_bytes(bn, hid_rows) + kRawCodeBytes + kRawScaleBytes;
+}
+
+// Where the stages go in dynamic shared memory [base, end) (shared-window addresses): after the
+// barrier block; with the pair table, around its 64 KB-aligned block. Host and device use the
+// same arithmetic, the host on the window layout it expects, the kernel on the real one.
+struct StageLayout {
+  uint32_t lo, n_lo;  // first region: start, stages
+  uint32_t hi;        // second region start (pair table only)
+  uint32_t table;     // pair table address (pair table only)
+  int stages;
+};
+__host__ __device__ inline StageLayout nvfp4_stage_layout(uint32_t base, uint32_t end,
+                                                          uint32_t stage_bytes, bool pair_table,
+                                                          int max_stages) {
+  StageLayout L;
+  const uint32_t a0 = ((base + 1023u) & ~1023u) + kBarrierBytes;
+  L.lo = a0;
+  if (pair_table) {
+    L.table = (a0 + 0xFFFFu) & ~0xFFFFu;
+    L.hi = L.table + kPairTableBytes;
+    L.n_lo = (L.table - a0) / stage_bytes;
+    const uint32_t n_hi = end > L.hi ? (end - L.hi) / stage_bytes : 0u;
+    L.stages = (int)(L.n_lo + n_hi);
+  } else {
+    L.table = 0;
+    L.hi = 0;
+    L.n_lo = end > a0 ? (end - a0) / stage_bytes : 0u;
+    L.stages = (int)L.n_lo;
+  }
+  if (L.stages > max_stages) L.stages = max_stages;
+  if ((int)L.n_lo > L.stages) L.n_lo = (uint32_t)L.stages;
+  return L;
 }
 
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -246,6 +296,56 @@ __device__ __forceinline__ void dequant8(uint32_t x, uint32_t s2, uint32_t* w) {
   w[3] = mul_bf16x2(prmt(p26, p37, 0x7632u), s2);
 }
 
+// Pair-table entry for code byte e (element 2j in the low nibble, 2j + 1 in the high one): the
+// bf16x2 word dequant8's step 1 gives for those two nibbles, in natural order.
+__host__ __device__ constexpr uint32_t pair_entry(uint32_t e) {
+  return ((e & 7u) << 6) | ((e & 8u) << 12) | (((e >> 4) & 7u) << 22) | (((e >> 4) & 8u) << 28);
+}
+
+// dequant8 through the pair table. lane_base = table address (64 KB aligned) + 4 * lane, so its
+// bits 8..15 are zero and prmt can drop code byte k there: entry address = table + 256 * byte +
+// 4 * lane.
+__device__ __forceinline__ void dequant8_table(uint32_t x, uint32_t s2, uint32_t lane_base,
+                                               uint32_t* w) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t a = prmt(x, lane_base, 0x7604u | ((uint32_t)k << 4));
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    w[k] = mul_bf16x2(v, s2);
+  }
+}
+
+template <bool kTable>
+__device__ __forceinline__ void dequant8_any(uint32_t x, uint32_t s2, uint32_t lane_base,
+                                             uint32_t* w) {
+  if (kTable)
+    dequant8_table(x, s2, lane_base, w);
+  else
+    dequant8(x, s2, w);
+}
+
+// One K step of one weight row: 64 codes (two 16-byte words) and their four block scales (one
+// byte each in `sc`, low byte first) to 32 bf16x2 words in K order.
+template <bool kTable>
+__device__ __forceinline__ void convert_kstep(const uint4& c0, const uint4& c1, uint32_t sc,
+                                              const uint32_t* lut, uint32_t lane_base,
+                                              uint32_t (&w)[32]) {
+  const uint32_t s0 = lut[sc & 0xFFu];
+  dequant8_any<kTable>(c0.x, s0, lane_base, w + 0);
+  dequant8_any<kTable>(c0.y, s0, lane_base, w + 4);
+  const uint32_t s1 = lut[(sc >> 8) & 0xFFu];
+  dequant8_any<kTable>(c0.z, s1, lane_base, w + 8);
+  dequant8_any<kTable>(c0.w, s1, lane_base, w + 12);
+  const uint32_t s2 = lut[(sc >> 16) & 0xFFu];
+  dequant8_any<kTable>(c1.x, s2, lane_base, w + 16);
+  dequant8_any<kTable>(c1.y, s2, lane_base, w + 20);
+  const uint32_t s3 = lut[sc >> 24];
+  dequant8_any<kTable>(c1.z, s3, lane_base, w + 24);
+  dequant8_any<kTable>(c1.w, s3, lane_base, w + 28);
+}
+
+template <bool kTable>
 __global__ void __launch_bounds__(kNvfp4Threads, 1)
     lmhead_w4a16_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_q,
                               const __grid_constant__ CUtensorMap tmap_s,
@@ -253,18 +353,32 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                               const Nvfp4HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119
-  uint8_t* smem = align_up_1024(smem_raw);
   // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
   // counters and descriptors in uniform registers.
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
-  const int S = p.stages;
-  const uint32_t sub_bytes = nvfp4_hid_sub_bytes(p.bn);
-  const uint32_t stage_bytes = nvfp4_stage_bytes(p.bn);
-  const uint32_t off_q = kRawK * sub_bytes;
+  const uint32_t hsub = (uint32_t)p.hid_rows * kBK * 2;  // hidden sub-tile stride in a stage
+  const uint32_t stage_bytes = nvfp4_stage_bytes(p.bn, p.hid_rows);
+  const uint32_t off_q = nvfp4_hid_region_bytes(p.bn, p.hid_rows);
   const uint32_t off_s = off_q + kRawCodeBytes;
+  uint32_t dyn_bytes;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+  const uint32_t raw = smem_u32(smem_raw);
+  const StageLayout L = nvfp4_stage_layout(raw, raw + dyn_bytes, stage_bytes, kTable,
+                                           p.max_stages);
+  const int S = L.stages;
+  if (S < 2) {  // the host sizes calls so this cannot happen; never run a one-stage ring
+    if (threadIdx.x == 0) atomicCAS(&g_lmhead_status, 0u, kStatusNoRoom);
+    return;
+  }
+  // Stage s: shared-window address, and a generic pointer for the dequantisers' reads.
+  auto stage_addr = [&](int s) -> uint32_t {
+    return (uint32_t)s < L.n_lo ? L.lo + (uint32_t)s * stage_bytes
+                                : L.hi + ((uint32_t)s - L.n_lo) * stage_bytes;
+  };
+  auto stage_ptr = [&](int s) -> const uint8_t* { return smem_raw + (stage_addr(s) - raw); };
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (L.lo - kBarrierBytes - raw));
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + S);
   const uint32_t afull0 = smem_u32(bars + 2 * S);
@@ -306,6 +420,13 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     tmem_relinquish();
   }
   for (int c = threadIdx.x; c < 256; c += blockDim.x) scale_lut[c] = scale_bf16x2((uint32_t)c);
+  if (kTable) {
+    // 256 entries x 32 lane copies; entry e of lane l at table + 256 e + 4 l.
+    uint8_t* table = smem_raw + (L.table - raw);
+    for (int c = threadIdx.x; c < 256 * 32; c += blockDim.x)
+      *reinterpret_cast<uint32_t*>(table + (c >> 5) * 256 + (c & 31) * 4) =
+          pair_entry((uint32_t)c >> 5);
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -318,7 +439,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     // ---------------------------------------------------------------- producer
     const uint64_t pol_w = l2_policy_weights();
     const uint64_t pol_h = l2_policy_evict_last();
-    const uint32_t hid_tx = (uint32_t)p.hid_rows * kBK * 2;
+    const uint32_t hid_tx = (uint32_t)kRawK * hsub;  // one box: 4 K steps of hid_rows rows
     int gr = 0;  // stages issued so far
     int st = 0;
     uint32_t ph = 0;
@@ -334,18 +455,17 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
         if (!p.wait.starve_loads) {
           const uint32_t full = full0 + 8 * st;
-          const uint32_t sbase = smem_u32(smem + (size_t)st * stage_bytes);
+          const uint32_t sbase = stage_addr(st);
           if (lane == 0) {
-            mbar_arrive_expect_tx(full, kRawCodeBytes + (p.scale_tma ? kRawScaleBytes : 0u) +
-                                            (uint32_t)nk * hid_tx);
+            // Boxes are counted whole: K steps past H arrive zero-filled.
+            mbar_arrive_expect_tx(full,
+                                  kRawCodeBytes + (p.scale_tma ? kRawScaleBytes : 0u) + hid_tx);
             tma_load_2d(sbase + off_q, &tmap_q, full, tma_x(r * (kRawK * kBK / 2), 1),
                         (int32_t)tc.v0, pol_w);
             if (p.scale_tma)
               tma_load_2d(sbase + off_s, &tmap_s, full, tma_x(r * (kRawK * 4), 1),
                           (int32_t)tc.v0, pol_w);
-            for (int j = 0; j < nk; ++j)
-              tma_load_2d(sbase + (uint32_t)j * sub_bytes, &tmap_h, full,
-                          tma_x((r * kRawK + j) * kBK * 2, 2), (int32_t)tc.r0, pol_h);
+            tma_load_3d(sbase, &tmap_h, full, 0, (int32_t)tc.r0, r * kRawK, pol_h);
           }
           if (!p.scale_tma) {
             // 4 rows per lane, 4 K steps of 4 bytes each; rows past V and K steps past H copy
@@ -391,7 +511,6 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
     int gr = 0;
     int st = 0;
-    uint32_t ph = 0;
     int sl = 0;  // weight slot of stage gr, and its phase
     uint32_t sph = 0;
     int acc = 0;
@@ -405,8 +524,9 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
       for (int r = 0; r < n_raw; ++r, ++gr) {
-        if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag) ||
-            !wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag)) {
+        // The slot is filled only after its dequantisers waited for this stage's loads, so the
+        // hidden rows have landed too.
+        if (!wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag)) {
           fail(kRoleMma, abort_flag);
           ok = false;
           break;
@@ -414,26 +534,22 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         tc_fence_after_sync();
         {
           const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
-          const uint32_t sb = smem_u32(smem + (size_t)st * stage_bytes);
-          const uint64_t bdesc0 = sdesc_kmajor_sw128(sb);
+          const uint64_t bdesc0 = sdesc_kmajor_sw128(stage_addr(st));
           const uint32_t a0 = tmem_base + slot_col0 + (uint32_t)sl * kSlotCols;
           // descriptor start addresses are in 16-byte units
           if (nk == kRawK) {
-            mma16_bf16_ts_elect(d_tmem, a0, bdesc0, sub_bytes >> 4, idesc, r != 0);
+            mma16_bf16_ts_elect(d_tmem, a0, bdesc0, hsub >> 4, idesc, r != 0);
           } else {
             for (int j = 0; j < nk; ++j)
               mma4_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2)),
-                                 bdesc0 + (uint64_t)((j * sub_bytes) >> 4), idesc,
+                                 bdesc0 + (uint64_t)((j * hsub) >> 4), idesc,
                                  (r | j) != 0);
           }
           mma_commit_elect(empty0 + 8 * st);
           mma_commit_elect(aempty0 + 8 * sl);
         }
         __syncwarp();
-        if (++st == S) {
-          st = 0;
-          ph ^= 1u;
-        }
+        if (++st == S) st = 0;
         if (++sl == NA) {
           sl = 0;
           sph ^= 1u;
@@ -497,6 +613,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t sw = (uint32_t)(row & 7);  // 128-byte swizzle of the codes box
     const uint32_t t_slots = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot_col0;
+    const uint32_t lane_base = L.table + (uint32_t)lane * 4u;  // pair table only
     const int total_raw = my_tiles * n_raw;
     int st = group % S;             // stage and phase of stage index gr, advanced by the group
     uint32_t ph = (uint32_t)(group / S) & 1u;  // count each iteration (no divisions in the loop)
@@ -511,28 +628,31 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint8_t* sbase = smem + (size_t)st * stage_bytes;
+      const uint8_t* sbase = stage_ptr(st);
       const uint8_t* crow = sbase + off_q + row * 128;
       const uint4 sc4 = *reinterpret_cast<const uint4*>(sbase + off_s + row * 16);
       const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
-      for (int j = 0; j < nk; ++j) {
-        const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2u * j) ^ sw) << 4));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2u * j + 1u) ^ sw) << 4));
-        const uint32_t sc = scw[j];
-        uint32_t w[32];
-        const uint32_t s0 = scale_lut[sc & 0xFFu];
-        dequant8(c0.x, s0, w + 0);
-        dequant8(c0.y, s0, w + 4);
-        const uint32_t s1 = scale_lut[(sc >> 8) & 0xFFu];
-        dequant8(c0.z, s1, w + 8);
-        dequant8(c0.w, s1, w + 12);
-        const uint32_t s2 = scale_lut[(sc >> 16) & 0xFFu];
-        dequant8(c1.x, s2, w + 16);
-        dequant8(c1.y, s2, w + 20);
-        const uint32_t s3 = scale_lut[sc >> 24];
-        dequant8(c1.z, s3, w + 24);
-        dequant8(c1.w, s3, w + 28);
-        tmem_st_32x32b_x32(t_slots + (uint32_t)sl * kSlotCols + (uint32_t)j * (kBK / 2), w);
+      const uint32_t t_dst = t_slots + (uint32_t)sl * kSlotCols;
+      if (nk == kRawK) {
+        // Whole stage: all eight 16-byte code reads first, so their latency overlaps.
+        uint4 c[2 * kRawK];
+#pragma unroll
+        for (int h = 0; h < 2 * kRawK; ++h)
+          c[h] = *reinterpret_cast<const uint4*>(crow + (((uint32_t)h ^ sw) << 4));
+#pragma unroll
+        for (int j = 0; j < kRawK; ++j) {
+          uint32_t w[32];
+          convert_kstep<kTable>(c[2 * j], c[2 * j + 1], scw[j], scale_lut, lane_base, w);
+          tmem_st_32x32b_x32(t_dst + (uint32_t)j * (kBK / 2), w);
+        }
+      } else {
+        for (int j = 0; j < nk; ++j) {
+          const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2u * j) ^ sw) << 4));
+          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2u * j + 1u) ^ sw) << 4));
+          uint32_t w[32];
+          convert_kstep<kTable>(c0, c1, scw[j], scale_lut, lane_base, w);
+          tmem_st_32x32b_x32(t_dst + (uint32_t)j * (kBK / 2), w);
+        }
       }
       mbar_arrive(empty0 + 8 * st);  // this row's codes and scales are in registers
       tmem_st_wait();

@@ -122,6 +122,15 @@ int lmhead_version(void);
  */
 void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
 
+/*
+ * Test knob (host side, per process) for lmhead_logits_w4a16_nvfp4's two ways of turning codes
+ * into bf16: 1 = the shared-memory pair table whenever it leaves room for two pipeline stages,
+ * 2 = integer spreading only, anything else = automatic (the table when it leaves room for
+ * three stages). Both give identical bits; the knob exists so tests can show that. Not for
+ * production use.
+ */
+void lmhead_debug_set_nvfp4_conversion(int path);
+
 #ifdef __cplusplus
 }
 #endif

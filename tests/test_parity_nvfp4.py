@@ -18,6 +18,14 @@ from tolerance import assert_bf16_close
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[1, 2], ids=["pair_table", "spread"])
+def conversion(request):
+    """Runs a test under each of the kernel's two code-to-bf16 conversions."""
+    lm.set_nvfp4_conversion(request.param)
+    yield request.param
+    lm.set_nvfp4_conversion(0)
+
+
 def pack(codes: np.ndarray) -> np.ndarray:
     return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
 
@@ -31,7 +39,7 @@ def test_tiny_matches_oracle():
     assert_bf16_close(got, ref, absum, "nvfp4 tiny")
 
 
-def test_every_code_and_scale_decodes_exactly():
+def test_every_code_and_scale_decodes_exactly(conversion):
     """One-hot hidden rows read single weights: with g = 1 and alpha = 1 the logit is the bf16
     of e2m1 * e4m3, exact -- so this checks the dequantiser on all 16 codes (both nibble
     positions, including -0) and all 126 finite non-negative scales, plus negative scales."""
@@ -59,7 +67,7 @@ def test_every_code_and_scale_decodes_exactly():
     assert np.all((got[~nz] & 0x7FFF) == 0)
 
 
-def test_integer_valued_sums_are_exact():
+def test_integer_valued_sums_are_exact(conversion):
     rng = np.random.default_rng(12)
     rows, H, V = 23, 192, 260
     codes = rng.integers(0, 16, (V, H)).astype(np.uint8)
@@ -71,7 +79,7 @@ def test_integer_valued_sums_are_exact():
     assert np.array_equal(got, ref)
 
 
-def test_ragged_shapes_and_global_scale():
+def test_ragged_shapes_and_global_scale(conversion):
     for rows, H, V, seed in [(1, 64, 1, 1), (17, 128, 129, 2), (65, 320, 300, 3), (300, 64, 200, 4)]:
         h = synth.hidden(rows, H, seed)
         packed, scales, g = synth.nvfp4_weights(V, H, 0.02, seed)
@@ -126,3 +134,18 @@ def test_64_row_chunked_calls_equal_one_call(nvfp4_inputs):
         done += m
     check_status()
     assert torch.equal(whole.view(torch.int16), chunked.view(torch.int16))
+
+
+def test_pair_table_and_spread_give_identical_bits(nvfp4_inputs):
+    """The two conversions are the same arithmetic (the table holds exactly the spread words), so
+    every row count the table serves must match the spread path bit for bit."""
+    h, packed, scales, g, pd, sd, rows_list, alpha = nvfp4_inputs
+    try:
+        for r in (1, 8, 9, 16, 17, 33, 64):
+            lm.set_nvfp4_conversion(1)
+            a = gpu_nvfp4(h[:r], pd, sd, g, alpha)
+            lm.set_nvfp4_conversion(2)
+            b = gpu_nvfp4(h[:r], pd, sd, g, alpha)
+            assert np.array_equal(a, b), r
+    finally:
+        lm.set_nvfp4_conversion(0)
