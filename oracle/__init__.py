@@ -6,7 +6,8 @@ this package. The CUDA library never imports, links or calls it, and shares no c
 The arithmetic lives in ``lmhead_oracle.c`` (plain C, double precision, one rounding at the end);
 this module only compiles it with gcc and marshals numpy arrays through ctypes. It computes
 
-    fp32 head:  logits[r, v] = RN_fp32(alpha * sum_k hidden[r, k] * W[v, k])
+    fp32 head:  logits[r, v] = RN_fp32(alpha * (sum_k hidden[r, k] * W[v, k] + bias[v]))
+                (bf16 or fp16 inputs; bias optional)
     NVFP4 head: logits[r, v] = RN_bf16(alpha * sum_k hidden[r, k] * e2m1(q[v, k]) * e4m3(s[v, k/16]) * g)
 
 following "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)" ("Purpose";
@@ -56,6 +57,8 @@ def _load():
         i64 = ctypes.c_int64
         lib.oracle_bf16_value.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_value.restype = ctypes.c_double
+        lib.oracle_f16_value.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_value.restype = ctypes.c_double
         lib.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
         lib.oracle_e2m1_value.restype = ctypes.c_double
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -69,6 +72,9 @@ def _load():
         lib.oracle_logits_bf16_f32.argtypes = [u16p, i64, i64, u16p, i64, ctypes.c_float, f32p,
                                                f64p, ctypes.c_int]
         lib.oracle_logits_bf16_f32.restype = ctypes.c_int
+        lib.oracle_logits_f32.argtypes = [u16p, ctypes.c_int, i64, i64, u16p, i64, ctypes.c_float,
+                                          ctypes.c_void_p, f32p, f64p, ctypes.c_int]
+        lib.oracle_logits_f32.restype = ctypes.c_int
         lib.oracle_logits_w4a16_nvfp4.argtypes = [u16p, i64, i64, u8p, u8p, ctypes.c_float, i64,
                                                   ctypes.c_float, u16p, f64p, ctypes.c_int]
         lib.oracle_logits_w4a16_nvfp4.restype = ctypes.c_int
@@ -88,6 +94,10 @@ def default_threads() -> int:
 
 def bf16_value(bits: int) -> float:
     return _load().oracle_bf16_value(int(bits) & 0xFFFF)
+
+
+def f16_value(bits: int) -> float:
+    return _load().oracle_f16_value(int(bits) & 0xFFFF)
 
 
 def e2m1_value(code: int) -> float:
@@ -160,4 +170,35 @@ def logits_w4a16_nvfp4(hidden_bits: np.ndarray, packed: np.ndarray, scales: np.n
                                            threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"oracle_logits_w4a16_nvfp4 failed with {rc}")
+    return out, absum
+
+
+def logits_f32(hidden_bits: np.ndarray, w_bits: np.ndarray, alpha: float, bias_bits=None,
+               dtype: str = "bf16", threads: int | None = None):
+    """fp32 logits and the error-bound scale for bf16 or fp16 ("f16") hidden [rows, H], W [V, H]
+    and optional bias [V], all given as uint16 bit patterns."""
+    if dtype not in ("bf16", "f16"):
+        raise ValueError(f"dtype {dtype!r}")
+    h = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    if h.ndim != 2 or w.ndim != 2 or h.shape[1] != w.shape[1]:
+        raise ValueError(f"shape mismatch: hidden {h.shape}, W {w.shape}")
+    rows, H = h.shape
+    V = w.shape[0]
+    b = None
+    if bias_bits is not None:
+        b = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        if b.shape != (V,):
+            raise ValueError(f"bias shape {b.shape}, expected ({V},)")
+    out = np.zeros((rows, V), dtype=np.float32)
+    absum = np.zeros((rows, V), dtype=np.float64)
+    if rows == 0:
+        return out, absum
+    rc = _load().oracle_logits_f32(_ptr(h, ctypes.c_uint16), 1 if dtype == "f16" else 0, rows, H,
+                                   _ptr(w, ctypes.c_uint16), V, ctypes.c_float(alpha),
+                                   None if b is None else b.ctypes.data,
+                                   _ptr(out, ctypes.c_float), _ptr(absum, ctypes.c_double),
+                                   threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_logits_f32 failed with {rc}")
     return out, absum

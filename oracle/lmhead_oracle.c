@@ -7,7 +7,7 @@
  * What is computed, written out as the plain definition, in double precision:
  *
  *   S[r, v]  = sum over k = 0 .. H-1, ascending, of dec(hidden[r, k]) * dec(W[v, k])
- *   fp32 head:   logits[r, v] = RN_fp32( alpha * S[r, v] )
+ *   fp32 head:   logits[r, v] = RN_fp32( alpha * (S[r, v] + dec(bias[v])) )   (bias optional)
  *   NVFP4 head:  W[v, k] = e2m1(code[v, k]) * e4m3(scale[v, k / 16]) * g
  *                logits[r, v] = RN_bf16( alpha * S[r, v] )          (one rounding, from double)
  *
@@ -17,13 +17,19 @@
  *    with alpha = 1/mup, bf16 inputs accumulated into fp32 without an fp32 weight copy, fp32 output.
  *  - "FP32 LM head skip FP32 cast" (SGLang PR #32370 summary), sections on function/motivation and
  *    the implementation breakdown: torch.mm(hidden, W.T, out_dtype=float32), a bf16 x bf16 -> fp32
- *    product with an fp32 accumulator.
+ *    product with an fp32 accumulator; the path's predicate admits float16 as well as bfloat16
+ *    hidden states, of the same dtype as the weight.
+ *  - The first page's "Purpose" lists the embedding bias among the cases the fused multiply does
+ *    not cover; there the head is the projection with its bias, then the elementwise multiply by
+ *    1/mup, read here as alpha * (hidden @ w.t() + bias), the bias in the weight's dtype.
  *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head at its declared
  *    W4A16 precision (16-bit activations, never cast to E4M3), bf16 logits[rows, vocab], row-major
  *    layouts (row offsets done*h*2 and done*v*2 bytes), values independent of the row count.
  *
  * Readings where the pages are silent (the NVFP4 layout is not printed anywhere):
  *  - bf16 decode: the 16 bits are the top half of an IEEE binary32.
+ *  - fp16 decode: IEEE binary16 (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits;
+ *    exponent 0 is subnormal, fraction * 2^-24; exponent 31 is infinity or NaN).
  *  - E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa; exponent 0 is subnormal
  *    (value 0.5 * m). Element 2j of a row is the LOW nibble of byte j, element 2j+1 the high one.
  *  - E4M3 (the "fn" variant): bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa, no
@@ -51,6 +57,25 @@ double oracle_bf16_value(uint16_t bits) {
   float f;
   memcpy(&f, &u, sizeof f);
   return (double)f;
+}
+
+double oracle_f16_value(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int expo = (bits >> 10) & 31;
+  int frac = bits & 1023;
+  double mag;
+  if (expo == 31) {
+    mag = frac ? NAN : INFINITY;
+  } else if (expo == 0) {
+    mag = ldexp((double)frac, -24); /* subnormal: (frac / 1024) * 2^-14 */
+  } else {
+    mag = ldexp(1.0 + (double)frac / 1024.0, expo - 15);
+  }
+  return sign ? -mag : mag;
+}
+
+static double decode16(uint16_t bits, int dtype) {
+  return dtype == 1 ? oracle_f16_value(bits) : oracle_bf16_value(bits);
 }
 
 double oracle_e2m1_value(uint8_t code) {
@@ -112,16 +137,17 @@ uint16_t oracle_round_bf16(double x) {
 
 /* ---------------------------------------------------------------- the head, fp32 output */
 
-int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
-                           int64_t V, float alpha, float* logits, double* abs_sum, int threads) {
-  if (rows < 0 || H <= 0 || V <= 0) return 1;
+int oracle_logits_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                      const uint16_t* W, int64_t V, float alpha, const uint16_t* bias,
+                      float* logits, double* abs_sum, int threads) {
+  if (rows < 0 || H <= 0 || V <= 0 || (dtype != 0 && dtype != 1)) return 1;
   if (rows == 0) return 0;
   if (!hidden || !W || !logits) return 1;
   const double a = (double)alpha;
   /* hidden decoded once: hd[r * H + k] = dec(hidden[r, k]) */
   double* hd = (double*)malloc((size_t)rows * (size_t)H * sizeof(double));
   if (!hd) return 2;
-  for (int64_t i = 0; i < rows * H; ++i) hd[i] = oracle_bf16_value(hidden[i]);
+  for (int64_t i = 0; i < rows * H; ++i) hd[i] = decode16(hidden[i], dtype);
   int failed = 0;
 #pragma omp parallel num_threads(threads > 0 ? threads : 1)
   {
@@ -133,7 +159,8 @@ int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, cons
 #pragma omp for schedule(static)
     for (int64_t v = 0; v < V; ++v) {
       if (!wv) continue;
-      for (int64_t k = 0; k < H; ++k) wv[k] = oracle_bf16_value(W[v * H + k]);
+      for (int64_t k = 0; k < H; ++k) wv[k] = decode16(W[v * H + k], dtype);
+      const double b = bias ? decode16(bias[v], dtype) : 0.0;
       for (int64_t r = 0; r < rows; ++r) {
         const double* h = hd + r * H;
         double s = 0.0, sa = 0.0;
@@ -142,14 +169,19 @@ int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, cons
           s += p;
           sa += fabs(p);
         }
-        logits[r * V + v] = oracle_round_f32(a * s);
-        if (abs_sum) abs_sum[r * V + v] = fabs(a) * sa;
+        logits[r * V + v] = oracle_round_f32(a * (s + b));
+        if (abs_sum) abs_sum[r * V + v] = fabs(a) * (sa + fabs(b));
       }
     }
     free(wv);
   }
   free(hd);
   return failed ? 2 : 0;
+}
+
+int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
+                           int64_t V, float alpha, float* logits, double* abs_sum, int threads) {
+  return oracle_logits_f32(hidden, 0, rows, H, W, V, alpha, NULL, logits, abs_sum, threads);
 }
 
 /* ---------------------------------------------------------------- the NVFP4 W4A16 head */

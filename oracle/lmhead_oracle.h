@@ -12,8 +12,9 @@
 extern "C" {
 #endif
 
-/* Exact value of one bf16 / E2M1 (low 4 bits of code) / E4M3fn encoding. */
+/* Exact value of one bf16 / IEEE fp16 / E2M1 (low 4 bits of code) / E4M3fn encoding. */
 double oracle_bf16_value(uint16_t bits);
+double oracle_f16_value(uint16_t bits);
 double oracle_e2m1_value(uint8_t code);
 double oracle_e4m3_value(uint8_t code);
 
@@ -33,6 +34,16 @@ double oracle_nvfp4_weight(const uint8_t* packed, const uint8_t* scales, float g
  */
 int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
                            int64_t V, float alpha, float* logits, double* abs_sum, int threads);
+
+/*
+ * The same with the input type chosen by dtype (0 = bf16, 1 = IEEE fp16; hidden, W and bias all
+ * of it) and an optional bias [V] (NULL = none):
+ *   logits[r, v] = RN_fp32(alpha * (sum_k hidden[r, k] * W[v, k] + bias[v])),
+ * abs_sum = |alpha| * (sum_k |hidden[r, k] * W[v, k]| + |bias[v]|).
+ */
+int oracle_logits_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                      const uint16_t* W, int64_t V, float alpha, const uint16_t* bias,
+                      float* logits, double* abs_sum, int threads);
 
 /*
  * logits[r, v] = RN_bf16(alpha * sum_k hidden[r, k] * e2m1(code[v, k]) * e4m3(scale[v, k/16]) * g)

@@ -347,3 +347,95 @@ def test_synth_e4m3_table_matches_torch():
     lib = torch.from_numpy(synth._E4M3_POS_CODES.copy()).view(torch.float8_e4m3fn).double().numpy()
     assert np.array_equal(vals, lib)
     assert np.all(np.diff(vals) > 0)
+
+
+# ---------------------------------------------------------------- fp16 inputs and the bias term
+# "FP32 LM head skip FP32 cast": the fused path's predicate admits float16 as well as bfloat16
+# hidden states of the weight's dtype. The first page's "Purpose" lists the embedding bias among
+# the cases handled as projection-with-bias followed by the multiply by 1/mup:
+#     logits = RN_fp32(alpha * (hidden @ W^T + bias)).
+
+def f16_bits(x: np.ndarray) -> np.ndarray:
+    """float -> IEEE binary16 bits through numpy (round-to-nearest-even: a library routine)."""
+    return np.ascontiguousarray(x, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+def test_f16_decode_all_codes_match_numpy():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    lib_vals = codes.view(np.float16).astype(np.float64)
+    for code in range(65536):
+        got = oracle.f16_value(code)
+        want = lib_vals[code]
+        if math.isnan(want):
+            assert math.isnan(got), hex(code)
+        else:
+            assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), hex(code)
+
+
+def test_f16_head_matches_library_double_matmul():
+    rng = np.random.default_rng(21)
+    rows, H, V = 5, 96, 37
+    h = f16_bits(rng.normal(0.0, 1.0, (rows, H)))
+    w = f16_bits(rng.normal(0.0, 0.05, (V, H)))
+    hd = h.view(np.float16).astype(np.float64)
+    wd = w.view(np.float16).astype(np.float64)
+    for alpha in (1.0, 0.125, -0.7):
+        got, absum = oracle.logits_f32(h, w, alpha, dtype="f16")
+        want = (np.float64(np.float32(alpha)) * (hd @ wd.T)).astype(np.float32)
+        # products are exact in double; the two double sums differ only in order
+        assert np.allclose(got, want, rtol=0, atol=1e-6 * float(absum.max()) + 1e-30)
+        assert np.allclose(absum, abs(np.float32(alpha)) * (np.abs(hd) @ np.abs(wd).T))
+
+
+def test_f16_integer_inputs_equal_exact_integer_matmul():
+    rng = np.random.default_rng(22)
+    rows, H, V = 7, 64, 19
+    hi = rng.integers(-30, 31, (rows, H))
+    wi = rng.integers(-30, 31, (V, H))
+    got, _ = oracle.logits_f32(f16_bits(hi), f16_bits(wi), 1.0, dtype="f16")
+    assert np.array_equal(got, (hi @ wi.T).astype(np.float32))
+
+
+def test_bias_alone_is_alpha_times_bias():
+    """W = 0: logits = RN(alpha * bias[v]) for every row, in both input types."""
+    rng = np.random.default_rng(23)
+    rows, H, V = 3, 32, 50
+    bias = rng.normal(0.0, 2.0, V)
+    for dtype, enc in (("bf16", bf16_bits_of_f32), ("f16", f16_bits)):
+        bb = enc(bias)
+        bvals = (bb.view(np.float16).astype(np.float64) if dtype == "f16"
+                 else np.array([oracle.bf16_value(int(x)) for x in bb]))
+        h = enc(rng.normal(0.0, 1.0, (rows, H)))
+        w = enc(np.zeros((V, H)))
+        for alpha in (1.0, 0.25, -3.0):
+            got, absum = oracle.logits_f32(h, w, alpha, bias_bits=bb, dtype=dtype)
+            want = (np.float64(np.float32(alpha)) * bvals).astype(np.float32)
+            assert np.array_equal(got, np.broadcast_to(want, (rows, V))), (dtype, alpha)
+            assert np.allclose(absum, abs(np.float32(alpha)) * np.abs(bvals))
+
+
+def test_bias_is_added_before_alpha():
+    """One-hot rows read W[v, k]; the bias joins the sum before the multiply:
+    RN(alpha * (W[v, k] + b[v])), which differs from RN(alpha * W[v, k] + b[v]) for alpha != 1."""
+    H, V = 16, 8
+    w = np.arange(V * H, dtype=np.float64).reshape(V, H) - 40.0
+    b = np.linspace(-3.5, 3.5, V)
+    wb, bb = bf16_bits_of_f32(w), bf16_bits_of_f32(b)
+    ks = [0, 5, 15]
+    h = np.zeros((len(ks), H))
+    for i, k in enumerate(ks):
+        h[i, k] = 1.0
+    got, _ = oracle.logits_f32(bf16_bits_of_f32(h), wb, 0.5, bias_bits=bb)
+    for i, k in enumerate(ks):
+        want = (0.5 * (w[:, k] + b)).astype(np.float32)
+        assert np.array_equal(got[i], want)
+        assert not np.array_equal(got[i], (0.5 * w[:, k] + b).astype(np.float32))
+
+
+def test_bf16_entry_without_bias_is_the_plain_head():
+    rng = np.random.default_rng(24)
+    h = bf16_bits_of_f32(rng.normal(0, 1, (4, 64)))
+    w = bf16_bits_of_f32(rng.normal(0, 0.05, (33, 64)))
+    a, sa = oracle.logits_f32(h, w, 0.125)
+    b, sb = oracle.logits_bf16_f32(h, w, 0.125)
+    assert np.array_equal(a, b) and np.array_equal(sa, sb)
