@@ -47,6 +47,9 @@ WORKLOAD_TEXT = {
              "scale, bf16 hidden and logits, alpha=1/8",
     "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
                     "fp32 out, alpha=1/8",
+    "decode_f16_bias": "decode LM head with fp16 operands and an fp16 embedding bias: rows "
+                       "{1,2,4,8,16,32,64}, H=2048, V=151936, fp32 accumulate and logits, "
+                       "alpha=1/8",
 }
 
 
@@ -159,9 +162,12 @@ class Workload:
         self.rows_list, self.H, self.V, self.alpha = rows_list, H, V, alpha
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
-                "prefill_2048": synth.SEED_PREFILL}[name]
+                "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16}[name]
         rmax = max(rows_list)
-        self.hidden = synth.hidden(rmax, H, seed, device=device)
+        self.dtype = torch.float16 if name == "decode_f16_bias" else torch.bfloat16
+        self.hidden = synth.hidden(rmax, H, seed, device=device, dtype=self.dtype)
+        self.bias = (synth.bias(V, synth.SEED_BIAS, device=device, dtype=self.dtype)
+                     if name == "decode_f16_bias" else None)
         self.nvfp4 = name == "nvfp4"
         if self.nvfp4:
             self.weights = [synth.random_nvfp4_codes(V, H, seed + i, device=device) for i in (0, 1)]
@@ -169,7 +175,8 @@ class Workload:
             self.outs = {r: torch.empty((r, V), dtype=torch.bfloat16, device=device)
                          for r in rows_list}
         else:
-            self.weights = [synth.weight(V, H, std, seed + i, device=device) for i in (0, 1)]
+            self.weights = [synth.weight(V, H, std, seed + i, device=device, dtype=self.dtype)
+                            for i in (0, 1)]
             self.outs = {r: torch.empty((r, V), dtype=torch.float32, device=device)
                          for r in rows_list}
         self.hid = {r: self.hidden[:r] for r in rows_list}
@@ -183,6 +190,8 @@ class Workload:
         o = self.outs[r] if out is None else out
         if self.nvfp4:
             lm.logits_w4a16_nvfp4(h, w[0], w[1], self.g, self.alpha, out=o, stream=stream)
+        elif self.bias is not None or self.dtype != torch.bfloat16:
+            lm.logits_f32(h, w, self.alpha, bias=self.bias, out=o, stream=stream)
         else:
             lm.logits_bf16_f32(h, w, self.alpha, out=o, stream=stream)
 
@@ -190,7 +199,7 @@ class Workload:
         H, V = self.H, self.V
         if self.nvfp4:
             return V * H // 2 + V * H // 16 + 4 + r * H * 2 + r * V * 2
-        return V * H * 2 + r * H * 2 + r * V * 4
+        return V * H * 2 + r * H * 2 + r * V * 4 + (V * 2 if self.bias is not None else 0)
 
     def flops_of(self, r: int) -> int:
         return 2 * r * self.H * self.V
@@ -326,7 +335,7 @@ def run_ours(args) -> dict | None:
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if not wl.nvfp4 else "e2m1xbf16",
+        "dtype": "e2m1xbf16" if wl.nvfp4 else ("f16" if wl.dtype == torch.float16 else "bf16"),
         "data": "synthetic (seeded N(0,1) hidden, N(0,std) weights; no dataset on the pages)",
         "config": {"workload": WORKLOAD_TEXT[args.workload],
                    "l2": "weights 2x larger than L2 per call; two weight copies alternated",
@@ -391,19 +400,23 @@ def _oracle_sample(workload: str, rows: int, vocab_slice: int, wl=None):
     from fp32_accumulate_lm_b200 import synth
     rows_list, H, V, std, alpha = synth.WORKLOADS[workload]
     key = (workload, rows, vocab_slice)
+    f16 = workload == "decode_f16_bias"
     if key not in _SAMPLES:
-        h = synth.hidden(rows, H, 7)
+        import torch
+        dt = torch.float16 if f16 else torch.bfloat16
+        h = synth.hidden(rows, H, 7, dtype=dt)
         if workload == "nvfp4":
             _SAMPLES[key] = (h, synth.nvfp4_weights(vocab_slice, H, std, 7))
         else:
-            _SAMPLES[key] = (h, synth.weight(vocab_slice, H, std, 7))
+            _SAMPLES[key] = (h, (synth.weight(vocab_slice, H, std, 7, dtype=dt),
+                                 synth.bias(vocab_slice, 7, dtype=dt) if f16 else None))
     h, w = _SAMPLES[key]
     t0 = time.perf_counter()
     if workload == "nvfp4":
         packed, scales, g = w
         oracle.logits_w4a16_nvfp4(h, packed, scales, g, alpha)
     else:
-        oracle.logits_bf16_f32(h, w, alpha)
+        oracle.logits_f32(h, w[0], alpha, bias_bits=w[1], dtype="f16" if f16 else "bf16")
     return time.perf_counter() - t0, rows * vocab_slice * H
 
 
@@ -426,9 +439,12 @@ def cpu_baseline(workload: str, wl) -> dict:
             oracle.logits_w4a16_nvfp4(h, packed[:vrows], scales[:vrows], wl.g, wl.alpha)
     else:
         w = wl.weights[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        b = None if wl.bias is None else wl.bias.view(torch.int16).cpu().numpy().view(np.uint16)
+        dt = "f16" if wl.dtype == torch.float16 else "bf16"
 
         def run(h, vrows):
-            oracle.logits_bf16_f32(h, w[:vrows], wl.alpha)
+            oracle.logits_f32(h, w[:vrows], wl.alpha, bias_bits=None if b is None else b[:vrows],
+                              dtype=dt)
     probe_v = min(V, 4096)
     t0 = time.perf_counter()
     run(h_all[:1], probe_v)

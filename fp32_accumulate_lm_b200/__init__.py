@@ -18,8 +18,9 @@ import os
 import threading
 
 __all__ = [
-    "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_w4a16_nvfp4",
-    "lmhead_logits_bf16_f32", "lmhead_logits_w4a16_nvfp4", "status_string", "device_status",
+    "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32",
+    "logits_w4a16_nvfp4", "lmhead_logits_bf16_f32", "lmhead_logits_f32",
+    "lmhead_logits_w4a16_nvfp4", "status_string", "device_status", "DTYPE_BF16", "DTYPE_F16",
     "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS",
 ]
 
@@ -29,6 +30,8 @@ STATUS = {
 }
 LMHEAD_OK = 0
 LMHEAD_ERR_TIMEOUT = 6
+DTYPE_BF16 = 0  # lmhead_dtype
+DTYPE_F16 = 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liblmhead.so")
@@ -59,6 +62,8 @@ def load_library():
         vp, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
         lib.lmhead_logits_bf16_f32.argtypes = [vp, i64, i64, vp, i64, f32, vp, vp]
         lib.lmhead_logits_bf16_f32.restype = i32
+        lib.lmhead_logits_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp]
+        lib.lmhead_logits_f32.restype = i32
         lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
         lib.lmhead_logits_w4a16_nvfp4.restype = i32
         lib.lmhead_status_string.argtypes = [i32]
@@ -81,6 +86,12 @@ def lmhead_logits_bf16_f32(hidden_ptr: int, rows: int, H: int, w_ptr: int, V: in
                            logits_ptr: int, stream: int = 0) -> int:
     return load_library().lmhead_logits_bf16_f32(hidden_ptr, rows, H, w_ptr, V, alpha,
                                                   logits_ptr, stream)
+
+
+def lmhead_logits_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: int, V: int,
+                      alpha: float, bias_ptr: int, logits_ptr: int, stream: int = 0) -> int:
+    return load_library().lmhead_logits_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
+                                             bias_ptr or None, logits_ptr, stream)
 
 
 def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
@@ -150,6 +161,33 @@ def logits_bf16_f32(hidden, W, alpha: float = 1.0, out=None, stream=None):
                                 out.data_ptr(), _stream_handle(stream))
     if st != LMHEAD_OK:
         raise LmheadError(st, "lmhead_logits_bf16_f32")
+    return out
+
+
+def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None):
+    """fp32 logits[rows, V] = alpha * (hidden @ W^T + bias) for bf16 or fp16 CUDA tensors hidden
+    [rows, H], W [V, H] and optional bias [V], all of one dtype. Runs asynchronously on
+    ``stream`` (default: torch's current stream)."""
+    import torch
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}.get(hidden.dtype)
+    _check(dt is not None and W.dtype == hidden.dtype, "bf16 or fp16 operands of one dtype required")
+    _check(hidden.dim() == 2 and W.dim() == 2 and hidden.shape[1] == W.shape[1], "shape mismatch")
+    _check(hidden.is_cuda and W.is_cuda, "CUDA tensors required")
+    _check(hidden.is_contiguous() and W.is_contiguous(), "contiguous tensors required")
+    rows, H = hidden.shape
+    V = W.shape[0]
+    if bias is not None:
+        _check(bias.dtype == hidden.dtype and bias.is_cuda and bias.is_contiguous()
+               and tuple(bias.shape) == (V,), "bias must be a contiguous [V] tensor of the dtype")
+    if out is None:
+        out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
+    _check(out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (rows, V),
+           "out must be a contiguous fp32 [rows, V] tensor")
+    st = lmhead_logits_f32(hidden.data_ptr(), dt, rows, H, W.data_ptr(), V, float(alpha),
+                           0 if bias is None else bias.data_ptr(), out.data_ptr(),
+                           _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logits_f32")
     return out
 
 

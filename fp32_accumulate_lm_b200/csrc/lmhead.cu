@@ -270,14 +270,26 @@ int lmhead_device_status(int clear) {
 
 int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const void* W, int64_t V,
                            float alpha, float* logits, lmhead_stream_t stream) {
+  return lmhead_logits_f32(hidden, LMHEAD_DTYPE_BF16, rows, H, W, V, alpha, nullptr, logits,
+                           stream);
+}
+
+int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                      int64_t V, float alpha, const void* bias, float* logits,
+                      lmhead_stream_t stream) {
+  if (dtype != LMHEAD_DTYPE_BF16 && dtype != LMHEAD_DTYPE_F16) return LMHEAD_ERR_SHAPE;
   if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
   if (H % 8 != 0) return LMHEAD_ERR_ALIGN;
   if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
   if (rows == 0) return LMHEAD_OK;
   if (hidden == nullptr || W == nullptr || logits == nullptr) return LMHEAD_ERR_NULL;
-  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(logits, 4)) return LMHEAD_ERR_ALIGN;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(logits, 4) ||
+      (bias != nullptr && !aligned(bias, 2))) {
+    return LMHEAD_ERR_ALIGN;
+  }
   if (overlaps(logits, rows * V * 4, hidden, rows * H * 2) ||
-      overlaps(logits, rows * V * 4, W, V * H * 2)) {
+      overlaps(logits, rows * V * 4, W, V * H * 2) ||
+      (bias != nullptr && overlaps(logits, rows * V * 4, bias, V * 2))) {
     return LMHEAD_ERR_ALIAS;
   }
   DeviceInfo dev;
@@ -289,7 +301,9 @@ int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const vo
   p.H = H;
   p.V = V;
   p.out = logits;
+  p.bias = reinterpret_cast<const uint16_t*>(bias);
   p.alpha = alpha;
+  p.fp16 = dtype == LMHEAD_DTYPE_F16 ? 1 : 0;
   p.bn = pick_bn(rows);
   int grid = 0;
   st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
@@ -306,11 +320,13 @@ int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const vo
   p.wait = wait_cfg();
 
   CUtensorMap tmap_w, tmap_h;
-  st = encode_rows(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, H * 2, V, lmh::kBK * 2,
+  const CUtensorMapDataType tdt =
+      p.fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  st = encode_rows(&tmap_w, tdt, 2, W, H * 2, V, lmh::kBK * 2,
                    lmh::kBM, CU_TENSOR_MAP_SWIZZLE_128B, kWeightPromo);
   if (st != LMHEAD_OK) return st;
   p.hid_rows = hid_box_rows(rows, p.bn);
-  st = encode_rows(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H * 2, rows,
+  st = encode_rows(&tmap_h, tdt, 2, hidden, H * 2, rows,
                    lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (st != LMHEAD_OK) return st;

@@ -1,4 +1,9 @@
-// fp32-accumulate LM head, bf16 operands: logits[r, v] = fl32(alpha * sum_k h[r, k] * W[v, k]).
+// fp32-accumulate LM head, bf16 or fp16 operands:
+//   logits[r, v] = fl32(alpha * sum_k h[r, k] * W[v, k])                       (no bias)
+//   logits[r, v] = fl32(alpha * fl32(sum_k h[r, k] * W[v, k] + bias[v]))      (with bias)
+// ("[Model] Honor fp32 head_dtype in Inkling muP logits", "Purpose": the projection with its
+// embedding bias, then the multiply by 1/mup; "FP32 LM head skip FP32 cast": fp16 or bf16
+// hidden states of the weight's dtype, fp32 accumulation and output).
 //
 // One persistent, warp-specialised tcgen05 kernel serves every row count (decode, speculative
 // verify and prefill alike), so a row's reduction order never depends on how many rows a call
@@ -15,7 +20,8 @@
 //   warp 1     TMEM allocator and MMA issuer: 4 * NSUB tcgen05.mma (K = 16 each) per stage into
 //              one of two TMEM accumulators; tcgen05.commit frees the stage (empty[s]) and, after
 //              the last K step, hands the accumulator to the epilogue (tmem_full[a]).
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, one IEEE fp32 multiply by alpha, store.
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, the bias (one IEEE fp32 add) if any, one
+//              IEEE fp32 multiply by alpha, store.
 // Tile ownership: see TileSched.
 #pragma once
 
@@ -26,7 +32,9 @@ namespace lmh {
 struct Bf16HeadParams {
   int64_t rows, H, V;
   float* out;
+  const uint16_t* bias;  // [V] in the operand type, or null
   float alpha;
+  int32_t fp16;          // operands (and bias) are IEEE fp16, else bf16
   int32_t bn;        // rows per tile: multiple of 16 in [16, 256]
   int32_t hid_rows;  // rows of hidden one TMA box brings (<= bn; MMA columns past it unused)
   TileSched sched;
@@ -145,7 +153,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
+    const uint32_t idesc = idesc_f16kind_f32(kBM, p.bn, p.fp16 == 0);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -210,6 +218,12 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
       const int64_t r0 = tc.r0;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.bn);
       const bool v_ok = v_local < tc.vrows;
+      // This lane's vocab entry's bias, decoded exactly to fp32 (null: none, and no add).
+      float b = 0.0f;
+      if (p.bias != nullptr && v_ok) {
+        const uint16_t bits = p.bias[v];
+        b = p.fp16 ? __half2float(__ushort_as_half(bits)) : __uint_as_float((uint32_t)bits << 16);
+      }
       for (int c = 0; c < p.bn; c += 16) {
         if (r0 + c >= p.rows) break;  // warp-uniform
         uint32_t r[16];
@@ -217,10 +231,19 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         tmem_ld_wait();
         if (v_ok) {
           float* dst = p.out + (r0 + c) * p.V + v;
+          if (p.bias == nullptr) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (r0 + c + j < p.rows)
-              __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
+            for (int j = 0; j < 16; ++j) {
+              if (r0 + c + j < p.rows)
+                __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (r0 + c + j < p.rows)
+                __stcs(dst + (int64_t)j * p.V,
+                       __fmul_rn(p.alpha, __fadd_rn(__uint_as_float(r[j]), b)));
+            }
           }
         }
       }

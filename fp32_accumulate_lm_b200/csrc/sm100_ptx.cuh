@@ -234,10 +234,14 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
   return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// kind::f16 instruction descriptor: bf16 x bf16 -> f32, both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+// kind::f16 instruction descriptor, f32 accumulator, both operands K-major: A and B both bf16
+// (format 1) or both fp16 (format 0) -- one MMA never mixes the two.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int m, int n, bool bf16) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(m >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
+  return idesc_f16kind_f32(m, n, true);
 }
 
 }  // namespace lmh

@@ -30,6 +30,9 @@ SEED_SPEC = 1002
 SEED_PREFILL = 1003
 SEED_NVFP4 = 1004
 SEED_PREFILL_SAMPLE = 2003
+SEED_F16 = 1005
+SEED_BIAS = 1006
+BIAS_STD = 0.5  # embedding bias ~ N(0, 0.5), a few logit units like a trained head's bias
 
 WORKLOADS = {
     # name: (rows list, H, V, weight std, alpha)
@@ -38,35 +41,54 @@ WORKLOADS = {
     "spec_verify": ([128, 97, 32], 4096, 128256, 0.015, 1.0 / 16),
     "prefill": ([8192], 4096, 151936, 0.02, 1.0 / 8),
     "nvfp4": ([1, 16, 64, 65, 256], 2048, 151936, 0.02, 1.0 / 8),
+    # the decode shape with fp16 operands and an fp16 embedding bias
+    "decode_f16_bias": ([1, 2, 4, 8, 16, 32, 64], 2048, 151936, 0.02, 1.0 / 8),
     # profiling case: the prefill kernel and tile shape on 2048 rows (a few GB on the device)
     "prefill_2048": ([2048], 4096, 151936, 0.02, 1.0 / 8),
 }
 
 
-def _normal_bf16(shape, std: float, seed: int, device=None) -> torch.Tensor:
+def _normal(shape, std: float, seed: int, device=None, dtype=torch.bfloat16) -> torch.Tensor:
     dev = torch.device(device) if device is not None else torch.device("cpu")
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
     x = torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32)
     if std != 1.0:
         x.mul_(std)
-    return x.to(torch.bfloat16)
+    return x.to(dtype)
+
+
+def _normal_bf16(shape, std: float, seed: int, device=None) -> torch.Tensor:
+    return _normal(shape, std, seed, device, torch.bfloat16)
 
 
 def _as_bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def hidden(rows: int, H: int, seed: int, device=None):
-    """hidden[rows, H] ~ N(0,1) in bf16. numpy uint16 bits, or a bf16 tensor on ``device``."""
-    t = _normal_bf16((rows, H), 1.0, seed, device)
+def hidden(rows: int, H: int, seed: int, device=None, dtype=torch.bfloat16):
+    """hidden[rows, H] ~ N(0,1) in bf16 (or ``dtype``, e.g. torch.float16). numpy uint16 bits,
+    or a tensor on ``device``."""
+    t = _normal((rows, H), 1.0, seed, device, dtype)
     return t if device is not None else _as_bits(t)
 
 
-def weight(V: int, H: int, std: float, seed: int, device=None):
-    """W[V, H] ~ N(0, std) in bf16. numpy uint16 bits, or a bf16 tensor on ``device``."""
-    t = _normal_bf16((V, H), std, seed + 500_000, device)
+def weight(V: int, H: int, std: float, seed: int, device=None, dtype=torch.bfloat16):
+    """W[V, H] ~ N(0, std) in bf16 (or ``dtype``). numpy uint16 bits, or a tensor on ``device``."""
+    t = _normal((V, H), std, seed + 500_000, device, dtype)
     return t if device is not None else _as_bits(t)
+
+
+def bias(V: int, seed: int, device=None, dtype=torch.bfloat16, std: float = BIAS_STD):
+    """Embedding bias[V] ~ N(0, std) in ``dtype``. numpy uint16 bits, or a tensor on ``device``."""
+    t = _normal((V,), std, seed + 900_000, device, dtype)
+    return t if device is not None else _as_bits(t)
+
+
+def bits_to_torch(bits: np.ndarray, dtype, device="cpu") -> torch.Tensor:
+    """uint16 bit patterns -> bf16 or fp16 tensor (a reinterpretation, no rounding)."""
+    a = np.ascontiguousarray(bits, dtype=np.uint16)
+    return torch.from_numpy(a.view(np.int16)).view(dtype).to(device)
 
 
 def bits_to_torch_bf16(bits: np.ndarray, device="cpu") -> torch.Tensor:

@@ -4,7 +4,7 @@
  *   logits[rows, V] = alpha * (hidden[rows, H] @ W[V, H]^T)
  *
  * Entry 1 takes bf16 hidden and W, accumulates in fp32 and writes fp32 logits; no fp32 copy of
- * either operand is ever made. Entry 2 is the W4A16 NVFP4 head: E2M1 weights with per-16 E4M3
+ * either operand is ever made. Its general form also takes fp16 operands and an embedding bias. Entry 2 is the W4A16 NVFP4 head: E2M1 weights with per-16 E4M3
  * block scales and one fp32 per-tensor scale, bf16 activations that are never quantised, bf16
  * logits.
  *
@@ -75,6 +75,30 @@ typedef enum {
  */
 int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const void* W, int64_t V,
                            float alpha, float* logits, lmhead_stream_t stream);
+
+/* Operand types of lmhead_logits_f32. */
+typedef enum { LMHEAD_DTYPE_BF16 = 0, LMHEAD_DTYPE_F16 = 1 } lmhead_dtype;
+
+/*
+ * Entry 1 in general form: fp32 logits from bf16 or IEEE fp16 operands, with an optional
+ * embedding bias.
+ *   no bias:   logits[r, v] = fl32(alpha * acc[r, v])                (exactly entry 1)
+ *   bias:      logits[r, v] = fl32(alpha * fl32(acc[r, v] + bias[v]))
+ *   acc[r, v]  = sum_k hidden[r, k] * W[v, k] in fp32 (every product exact).
+ * "FP32 LM head skip FP32 cast" takes the fused fp32-accumulate path for fp16 as well as bf16
+ * hidden states of the weight's dtype; the first page ("Purpose") applies 1/mup after the
+ * projection with its embedding bias, so the bias joins the sum before alpha. The add and the
+ * multiply are single IEEE round-to-nearest fp32 operations (no FMA contraction).
+ *
+ *   hidden  dtype [rows, H], 16-byte aligned         rows >= 0
+ *   W       dtype [V, H],    16-byte aligned         H > 0, H % 8 == 0
+ *   bias    dtype [V], 2-byte aligned, or NULL       read only, must not overlap logits
+ *   logits  fp32 [rows, V], 4-byte aligned           V > 0
+ * dtype is an lmhead_dtype (anything else: LMHEAD_ERR_SHAPE). Returns an lmhead_status.
+ */
+int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                      int64_t V, float alpha, const void* bias, float* logits,
+                      lmhead_stream_t stream);
 
 /*
  * Entry 2: bf16 logits from the W4A16 NVFP4 head.

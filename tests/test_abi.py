@@ -84,6 +84,22 @@ def test_bf16_null_align_alias(lib):
     assert lm.lmhead_logits_bf16_f32(A16, 4, 64, B16, 128, 1.0, A16 - 16, 0) == 7
 
 
+def test_general_entry_argument_errors(lib):
+    """lmhead_logits_f32: operand type, bias alignment and bias/logits overlap are checked on the
+    host before anything is launched; without a bias it takes the bf16 entry's checks."""
+    f = lm.lmhead_logits_f32
+    for dt in (lm.DTYPE_BF16, lm.DTYPE_F16):
+        assert f(A16, dt, -1, 64, B16, 128, 1.0, 0, C16, 0) == 2
+        assert f(A16, dt, 4, 60, B16, 128, 1.0, 0, C16, 0) == 3
+        assert f(0, dt, 4, 64, B16, 128, 1.0, 0, C16, 0) == 1
+        assert f(A16, dt, 4, 64, B16, 128, 1.0, 0x7000001, C16, 0) == 3     # odd bias address
+        assert f(A16, dt, 4, 64, B16, 128, 1.0, C16 + 64, C16, 0) == 7      # bias inside logits
+        assert f(A16, dt, 4, 64, B16, 128, 1.0, 0, B16 + 64, 0) == 7
+    for bad in (2, -1, 7):
+        assert f(A16, bad, 4, 64, B16, 128, 1.0, 0, C16, 0) == 2
+    assert f(0, lm.DTYPE_F16, 0, 64, 0, 128, 1.0, 0, 0, 0) == 0             # rows == 0: no-op
+
+
 def test_rows_zero_launches_nothing(lib):
     # rows == 0 is a no-op even with NULL pointers (no CUDA call is made)
     assert lm.lmhead_logits_bf16_f32(0, 0, 64, 0, 128, 1.0, 0, 0) == 0
