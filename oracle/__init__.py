@@ -78,6 +78,12 @@ def _load():
         lib.oracle_logits_w4a16_nvfp4.argtypes = [u16p, i64, i64, u8p, u8p, ctypes.c_float, i64,
                                                   ctypes.c_float, u16p, f64p, ctypes.c_int]
         lib.oracle_logits_w4a16_nvfp4.restype = ctypes.c_int
+        lib.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, u8p, u8p, f32p]
+        lib.oracle_nvfp4_quantize.restype = ctypes.c_int
+        lib.oracle_rn_e4m3.argtypes = [ctypes.c_float]
+        lib.oracle_rn_e4m3.restype = ctypes.c_uint8
+        lib.oracle_rn_e2m1.argtypes = [ctypes.c_float]
+        lib.oracle_rn_e2m1.restype = ctypes.c_uint8
         _lib = lib
         return lib
 
@@ -202,3 +208,28 @@ def logits_f32(hidden_bits: np.ndarray, w_bits: np.ndarray, alpha: float, bias_b
     if rc != 0:
         raise RuntimeError(f"oracle_logits_f32 failed with {rc}")
     return out, absum
+
+
+# ---------------------------------------------------------------- the NVFP4 quantiser
+
+def rn_e4m3(t: float) -> int:
+    return int(_load().oracle_rn_e4m3(ctypes.c_float(t)))
+
+
+def rn_e2m1(x: float) -> int:
+    return int(_load().oracle_rn_e2m1(ctypes.c_float(x)))
+
+
+def nvfp4_quantize(w_bits: np.ndarray):
+    """(packed [V, H/2] u8, scales [V, H/16] u8, g float32) for bf16 W [V, H] given as uint16 bits
+    (H % 16 == 0), by the binary32 reading in lmhead_oracle.c."""
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    V, H = w.shape
+    packed = np.zeros((V, H // 2), dtype=np.uint8)
+    scales = np.zeros((V, H // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    rc = _load().oracle_nvfp4_quantize(_ptr(w, ctypes.c_uint16), V, H, _ptr(packed, ctypes.c_uint8),
+                                       _ptr(scales, ctypes.c_uint8), _ptr(g, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle_nvfp4_quantize failed with {rc}")
+    return packed, scales, np.float32(g[0])

@@ -38,6 +38,15 @@
  *    [16j, 16j+16). g is the per-tensor decode multiplier (w = q * s * g).
  *  - Rounding is IEEE round-to-nearest-even, done once from double.
  *
+ * NVFP4 quantiser (oracle_nvfp4_quantize). lm_head_nvfp4_rows.rs and mtp_head/new_bf16_moe.rs
+ * ("quantize_to_nvfp4(w, n, k, gpu, absmax_k, nvfp4_k, stream)": an absmax kernel, then an encode
+ * kernel) name it but print no rules. Reading, with every step one IEEE binary32 operation so that
+ * a GPU implementation can take the same decisions bit for bit:
+ *   amax = max |w| over the tensor;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
+ *   per 16-element block: t = bmax / (6 * g);  s = RN_e4m3(t), saturating at 448
+ *   per element: d = e4m3(s) * g;  x = w / d (0 when d = 0);  q = RN_e2m1(x), saturating at 6,
+ *   sign kept only when the magnitude is not zero. RN = nearest, ties to the even code.
+ *
  * Why double is exact enough: a bf16 x bf16 product has at most 16 significant bits and an
  * e2m1 * e4m3 * g * bf16 product at most 2+4+24+8 = 38, so every product is exact in double;
  * the double sum's error is below H * 2^-53 * sum|p|, far inside any fp32 tolerance.
@@ -182,6 +191,74 @@ int oracle_logits_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H
 int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
                            int64_t V, float alpha, float* logits, double* abs_sum, int threads) {
   return oracle_logits_f32(hidden, 0, rows, H, W, V, alpha, NULL, logits, abs_sum, threads);
+}
+
+/* ---------------------------------------------------------------- the NVFP4 quantiser */
+
+/* Nearest entry of an ascending table of exact values (ties to the even index); x >= 0 finite
+ * or +inf. Differences are taken in double: x and the table entries are floats, so a tie (x
+ * exactly halfway, itself a short float) is detected exactly. */
+static int nearest_even_index(float x, const double* vals, int n) {
+  if (!(x > vals[0])) return 0;
+  if (x >= vals[n - 1]) return n - 1;
+  int hi = 1;
+  while (vals[hi] < (double)x) ++hi;
+  const int lo = hi - 1;
+  const double dlo = (double)x - vals[lo];
+  const double dhi = vals[hi] - (double)x;
+  if (dhi < dlo) return hi;
+  if (dlo < dhi) return lo;
+  return (hi % 2 == 0) ? hi : lo;
+}
+
+uint8_t oracle_rn_e4m3(float t) {
+  static double vals[127];
+  static int ready = 0;
+  if (!ready) {
+    for (int c = 0; c < 127; ++c) vals[c] = oracle_e4m3_value((uint8_t)c);
+    ready = 1;
+  }
+  return (uint8_t)nearest_even_index(t, vals, 127);
+}
+
+uint8_t oracle_rn_e2m1(float x) {
+  static const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const int m = nearest_even_index(fabsf(x), mags, 8);
+  return (uint8_t)((x < 0.0f && m != 0) ? (m | 8) : m);
+}
+
+int oracle_nvfp4_quantize(const uint16_t* w, int64_t V, int64_t H, uint8_t* packed,
+                          uint8_t* scales, float* g_out) {
+  if (V <= 0 || H <= 0 || H % 16 != 0 || !w || !packed || !scales || !g_out) return 1;
+  float amax = 0.0f;
+  for (int64_t i = 0; i < V * H; ++i) {
+    const float a = fabsf((float)oracle_bf16_value(w[i]));
+    if (a > amax) amax = a;
+  }
+  const float g = amax > 0.0f ? amax / 2688.0f : 1.0f;
+  const float six_g = 6.0f * g;
+  for (int64_t v = 0; v < V; ++v) {
+    for (int64_t j = 0; j < H / 16; ++j) {
+      const uint16_t* blk = w + v * H + j * 16;
+      float bmax = 0.0f;
+      for (int i = 0; i < 16; ++i) {
+        const float a = fabsf((float)oracle_bf16_value(blk[i]));
+        if (a > bmax) bmax = a;
+      }
+      const float t = bmax / six_g;
+      const uint8_t s = oracle_rn_e4m3(t);
+      scales[v * (H / 16) + j] = s;
+      const float d = (float)oracle_e4m3_value(s) * g;
+      for (int i = 0; i < 16; i += 2) {
+        const float x0 = d > 0.0f ? (float)oracle_bf16_value(blk[i]) / d : 0.0f;
+        const float x1 = d > 0.0f ? (float)oracle_bf16_value(blk[i + 1]) / d : 0.0f;
+        packed[v * (H / 2) + j * 8 + i / 2] =
+            (uint8_t)(oracle_rn_e2m1(x0) | (oracle_rn_e2m1(x1) << 4));
+      }
+    }
+  }
+  *g_out = g;
+  return 0;
 }
 
 /* ---------------------------------------------------------------- the NVFP4 W4A16 head */

@@ -54,6 +54,18 @@ int oracle_logits_w4a16_nvfp4(const uint16_t* hidden, int64_t rows, int64_t H,
                               const uint8_t* packed, const uint8_t* scales, float g, int64_t V,
                               float alpha, uint16_t* logits, double* abs_sum, int threads);
 
+/*
+ * NVFP4 quantiser (this library's reading; every decision step one IEEE binary32 operation):
+ * amax = max|w|, g = amax / 2688 (1 when amax = 0); per 16-element block s = RN_e4m3(bmax / (6g))
+ * saturating; per element q = RN_e2m1(w / (e4m3(s) * g)) saturating, sign only on non-zero
+ * magnitudes. w is bf16 [V, H] bits, H % 16 == 0; outputs packed [V, H/2], scales [V, H/16], g.
+ */
+int oracle_nvfp4_quantize(const uint16_t* w, int64_t V, int64_t H, uint8_t* packed,
+                          uint8_t* scales, float* g_out);
+/* Nearest E4M3 code (non-negative, saturating at 448) / E2M1 code, ties to the even code. */
+uint8_t oracle_rn_e4m3(float t);
+uint8_t oracle_rn_e2m1(float x);
+
 #ifdef __cplusplus
 }
 #endif

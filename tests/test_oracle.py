@@ -439,3 +439,138 @@ def test_bf16_entry_without_bias_is_the_plain_head():
     a, sa = oracle.logits_f32(h, w, 0.125)
     b, sb = oracle.logits_bf16_f32(h, w, 0.125)
     assert np.array_equal(a, b) and np.array_equal(sa, sb)
+
+
+# ---------------------------------------------------------------- the NVFP4 quantiser
+# lm_head_nvfp4_rows.rs / mtp_head/new_bf16_moe.rs name quantize_to_nvfp4 (absmax, then encode)
+# without printing its rules; the oracle's reading takes every decision in IEEE binary32 (see
+# lmhead_oracle.c). These pins re-derive each decision independently: exact rationals for the
+# nearest-even encoders, torch's float8_e4m3fn conversion, and numpy float32 for the arithmetic.
+from fractions import Fraction
+
+E2M1_MAGS = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3),
+             Fraction(4), Fraction(6)]
+
+
+def e4m3_fraction(c: int) -> Fraction:
+    e, m = (c >> 3) & 15, c & 7
+    return Fraction(m, 8) * Fraction(1, 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+
+
+E4M3_VALS = [e4m3_fraction(c) for c in range(127)]
+
+
+def brute_nearest_even(x: Fraction, vals) -> int:
+    """Index of the nearest value (ties to the even index), saturating at both ends."""
+    best = min(range(len(vals)), key=lambda i: (abs(vals[i] - x), i % 2))
+    return best
+
+
+def float32_points(rng, lo, hi, n):
+    """Random float32 values in [lo, hi] plus every table midpoint and its float32 neighbours."""
+    return np.float32(rng.uniform(lo, hi, n))
+
+
+def test_rn_e4m3_matches_bruteforce_and_torch():
+    rng = np.random.default_rng(71)
+    pts = list(float32_points(rng, 0.0, 460.0, 3000)) + list(np.float32(2.0 ** rng.uniform(-12, 9, 3000)))
+    for a, b in zip(E4M3_VALS[:-1], E4M3_VALS[1:]):   # midpoints (exact in float32) and neighbours
+        mid = np.float32(float((a + b) / 2))
+        pts += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9))]
+    pts += [np.float32(0.0), np.float32(448.0), np.float32(500.0), np.float32(1e30)]
+    for t in pts:
+        got = oracle.rn_e4m3(float(t))
+        want = brute_nearest_even(Fraction(float(t)), E4M3_VALS)
+        assert got == want, (float(t), got, want)
+        if float(t) <= 448.0:
+            via_torch = torch.tensor([float(t)], dtype=torch.float32).to(torch.float8_e4m3fn)
+            assert int(via_torch.view(torch.uint8)[0]) == got, float(t)
+
+
+def test_rn_e2m1_matches_bruteforce():
+    rng = np.random.default_rng(72)
+    pts = list(np.float32(rng.uniform(-7.0, 7.0, 4000)))
+    for a, b in zip(E2M1_MAGS[:-1], E2M1_MAGS[1:]):
+        mid = np.float32(float((a + b) / 2))
+        for x in (mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(9))):
+            pts += [x, -x]
+    pts += [np.float32(0.0), np.float32(-0.0), np.float32(6.0), np.float32(-100.0), np.float32(np.inf)]
+    for x in pts:
+        got = oracle.rn_e2m1(float(x))
+        m = brute_nearest_even(Fraction(abs(float(x))) if np.isfinite(x) else Fraction(10 ** 9), E2M1_MAGS)
+        want = (m | 8) if (float(x) < 0 and m != 0) else m
+        assert got == want, (float(x), got, want)
+
+
+def numpy_quantize_f32(w_bits: np.ndarray):
+    """The reading re-derived with numpy float32 arithmetic and exact nearest-even searches."""
+    wf = synth.bf16_bits_to_f32(w_bits)
+    V, H = wf.shape
+    amax = np.float32(np.max(np.abs(wf)))
+    g = np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
+    six_g = np.float32(np.float32(6.0) * g)
+    scales = np.zeros((V, H // 16), np.uint8)
+    codes = np.zeros((V, H), np.uint8)
+    for v in range(V):
+        for j in range(H // 16):
+            blk = wf[v, 16 * j:16 * j + 16]
+            t = np.float32(np.float32(np.max(np.abs(blk))) / six_g)
+            s = brute_nearest_even(Fraction(float(t)), E4M3_VALS)
+            scales[v, j] = s
+            d = np.float32(np.float32(float(E4M3_VALS[s])) * g)
+            for i in range(16):
+                x = np.float32(blk[i] / d) if d > 0 else np.float32(0.0)
+                m = brute_nearest_even(Fraction(abs(float(x))) if np.isfinite(x) else Fraction(10 ** 9),
+                                       E2M1_MAGS)
+                codes[v, 16 * j + i] = (m | 8) if (x < 0 and m != 0) else m
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, scales, g
+
+
+def test_quantiser_matches_numpy_float32_rederivation():
+    rng = np.random.default_rng(73)
+    # a spread of block magnitudes, so scales cover subnormal to large E4M3 codes
+    w = rng.normal(0, 1, (6, 64)) * (10.0 ** rng.uniform(-4, 2, (6, 4))).repeat(16, axis=1)
+    wb = bf16_bits_of_f32(w)
+    p, s, g = oracle.nvfp4_quantize(wb)
+    p2, s2, g2 = numpy_quantize_f32(wb)
+    assert g == g2
+    assert np.array_equal(s, s2)
+    assert np.array_equal(p, p2)
+
+
+def test_quantiser_closed_forms():
+    # amax = 2688 gives g = 1; a block whose max is 6 gets scale 1.0 (0x38) and codes that are
+    # the E2M1 values themselves
+    H = 32
+    w = np.zeros((2, H))
+    w[0, 0] = 2688.0                                     # block 0 of row 0: t = 448 -> 0x7E
+    w[1, :8] = [6.0, 3.0, -1.5, 0.5, -0.0, 2.0, -4.0, 1.0]
+    w[1, 16:20] = [-6.0, 0.25, 0.75, 5.0]                # ties: 0.25 -> 0, 0.75 -> 1.0, 5 -> 4
+    p, s, g = oracle.nvfp4_quantize(bf16_bits_of_f32(w))
+    assert g == np.float32(1.0)
+    assert s[0, 0] == 0x7E and s[0, 1] == 0 and s[1, 0] == 0x38 and s[1, 1] == 0x38
+    codes = np.stack([p & 0x0F, p >> 4], axis=2).reshape(2, H)
+    assert list(codes[1, :8]) == [7, 5, 11, 1, 0, 4, 14, 2]
+    assert list(codes[1, 16:20]) == [15, 0, 2, 6]
+    assert codes[0, 0] == 7 and not codes[0, 1:].any()
+
+
+def test_quantiser_all_zero_weights():
+    p, s, g = oracle.nvfp4_quantize(np.zeros((3, 48), np.uint16))
+    assert g == np.float32(1.0) and not p.any() and not s.any()
+
+
+def test_quantiser_round_trip_error_is_within_half_a_code():
+    """Dequantising gives each weight back to within half the E2M1 spacing at its magnitude
+    (times s * g), except where the scale saturates or underflows."""
+    wb = synth.weight(64, 256, 0.02, 74)
+    p, s, g = oracle.nvfp4_quantize(wb)
+    wf = synth.bf16_bits_to_f32(wb).astype(np.float64)
+    for v in range(0, 64, 7):
+        for k in range(0, 256, 5):
+            deq = oracle.nvfp4_weight(p, s, float(g), v, k)
+            unit = oracle.e4m3_value(int(s[v, k // 16])) * float(g)
+            x = abs(wf[v, k]) / unit if unit > 0 else 0.0
+            step = 0.5 if x < 2 else (1.0 if x < 4 else 2.0)
+            assert abs(deq - wf[v, k]) <= 0.5 * step * unit * (1 + 1e-6) + 1e-30, (v, k)
