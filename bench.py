@@ -47,6 +47,8 @@ WORKLOAD_TEXT = {
              "scale, bf16 hidden and logits, alpha=1/8",
     "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
                     "fp32 out, alpha=1/8",
+    "nvfp4_quantize": "NVFP4 quantiser (absmax pass, then encode pass) of a bf16 W[151936, 2048] "
+                      "into E2M1 codes, E4M3 block scales and an fp32 global scale",
     "decode_f16_bias": "decode LM head with fp16 operands and an fp16 embedding bias: rows "
                        "{1,2,4,8,16,32,64}, H=2048, V=151936, fp32 accumulate and logits, "
                        "alpha=1/8",
@@ -162,8 +164,26 @@ class Workload:
         self.rows_list, self.H, self.V, self.alpha = rows_list, H, V, alpha
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
-                "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16}[name]
+                "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16,
+                "nvfp4_quantize": synth.SEED_NVFP4}[name]
         rmax = max(rows_list)
+        self.quantize = name == "nvfp4_quantize"
+        if self.quantize:
+            # one call quantises all V rows of a bf16 W; two copies alternate (each > L2)
+            import fp32_accumulate_lm_b200 as lm
+            self.dtype = torch.bfloat16
+            self.bias = None
+            self.nvfp4 = False
+            self.weights = [synth.weight(V, H, std, seed + i, device=device) for i in (0, 1)]
+            self.hidden = self.weights[0]
+            self.hid = {V: self.weights[0]}
+            self.outs = {V: torch.empty((V, H // 2), dtype=torch.uint8, device=device)}
+            self.q_scales = torch.empty((V, H // 16), dtype=torch.uint8, device=device)
+            self.q_g = torch.empty((1,), dtype=torch.float32, device=device)
+            self.ws = torch.empty((lm.nvfp4_quantize_workspace_bytes(),), dtype=torch.uint8,
+                                  device=device)
+            self.calls = 0
+            return
         self.dtype = torch.float16 if name == "decode_f16_bias" else torch.bfloat16
         self.hidden = synth.hidden(rmax, H, seed, device=device, dtype=self.dtype)
         self.bias = (synth.bias(V, synth.SEED_BIAS, device=device, dtype=self.dtype)
@@ -184,6 +204,13 @@ class Workload:
 
     def call(self, r: int, hidden=None, out=None, stream=None):
         import fp32_accumulate_lm_b200 as lm
+        if self.quantize:
+            W = self.weights[self.calls & 1] if hidden is None else hidden
+            self.calls += 1
+            lm.nvfp4_quantize(W, workspace=self.ws,
+                              out=(self.outs[r] if out is None else out, self.q_scales, self.q_g),
+                              stream=stream)
+            return
         w = self.weights[self.calls & 1]
         self.calls += 1
         h = self.hid[r] if hidden is None else hidden
@@ -197,12 +224,14 @@ class Workload:
 
     def bytes_of(self, r: int) -> int:
         H, V = self.H, self.V
+        if self.quantize:  # two passes over W (absmax, then encode), codes, scales and g out
+            return 2 * V * H * 2 + V * H // 2 + V * H // 16 + 4
         if self.nvfp4:
             return V * H // 2 + V * H // 16 + 4 + r * H * 2 + r * V * 2
         return V * H * 2 + r * H * 2 + r * V * 4 + (V * 2 if self.bias is not None else 0)
 
     def flops_of(self, r: int) -> int:
-        return 2 * r * self.H * self.V
+        return 0 if self.quantize else 2 * r * self.H * self.V
 
 
 def dist_setup(n_gpus: int, backend: str = "nccl"):
@@ -321,7 +350,8 @@ def run_ours(args) -> dict | None:
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": f"HBM copy ({peaks['source']})"}
-    roof["kernel"] = "lmhead_w4a16_nvfp4_kernel" if wl.nvfp4 else "lmhead_bf16_f32_kernel"
+    roof["kernel"] = ("nvfp4_encode_kernel + nvfp4_absmax_kernel" if wl.quantize else
+                      "lmhead_w4a16_nvfp4_kernel" if wl.nvfp4 else "lmhead_bf16_f32_kernel")
     roof["traffic"] = recorded_traffic(roof["kernel"], args.workload)
     roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
     roof["source_hash"] = kernel_source_hash()
@@ -335,7 +365,8 @@ def run_ours(args) -> dict | None:
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1xbf16" if wl.nvfp4 else ("f16" if wl.dtype == torch.float16 else "bf16"),
+        "dtype": ("f32" if wl.quantize else "e2m1xbf16" if wl.nvfp4 else
+                  "f16" if wl.dtype == torch.float16 else "bf16"),
         "data": "synthetic (seeded N(0,1) hidden, N(0,std) weights; no dataset on the pages)",
         "config": {"workload": WORKLOAD_TEXT[args.workload],
                    "l2": "weights 2x larger than L2 per call; two weight copies alternated",
@@ -343,7 +374,7 @@ def run_ours(args) -> dict | None:
                    "calls_per_step": calls_per_step, "per_rows": detail},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": n_ev,
+        "gpu_launches": n_ev * (2 if wl.quantize else 1),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -429,6 +460,14 @@ def cpu_baseline(workload: str, wl) -> dict:
     import torch
     cores = oracle.default_threads()
     H, V = wl.H, wl.V
+    if wl.quantize:  # the oracle quantiser is single-threaded: time a slice of W's rows
+        w = wl.weights[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        n = 4096
+        t0 = time.perf_counter()
+        oracle.nvfp4_quantize(w[:n])
+        secs = time.perf_counter() - t0
+        return {"value": round(1e6 * secs * V / n, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"{n} of W's {V} rows x H={H} ({secs:.1f} s), scaled by rows"}
     rows_in_step = sum(wl.rows_list)
     h_all = wl.hidden.view(torch.int16).cpu().numpy().view(np.uint16)
     if wl.nvfp4:
@@ -459,6 +498,37 @@ def cpu_baseline(workload: str, wl) -> dict:
                       f"({secs:.1f} s), scaled by rows to the step, per call"}
 
 
+def _reference_quantize(args, H: int, V: int) -> dict:
+    """The oracle quantiser as the reference arm: each step quantises a slice of W's rows, scaled
+    by rows to one call."""
+    import oracle
+    from fp32_accumulate_lm_b200 import synth
+    n = 2048
+    w = synth.weight(n, H, 0.02, 7)
+    for _ in range(args.warmup):
+        oracle.nvfp4_quantize(w)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.nvfp4_quantize(w)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    us = 1e6 * total / args.steps * V / n
+    sample = f"per step: {n} of W's {V} rows x H={H}, scaled by rows to one call"
+    return {
+        "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "parallelism": "host core"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args) -> dict | None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -467,6 +537,8 @@ def run_reference(args) -> dict | None:
     from fp32_accumulate_lm_b200 import synth
     rows_list, H, V, std, alpha = synth.WORKLOADS[args.workload]
     cores = oracle.default_threads()
+    if args.workload == "nvfp4_quantize":
+        return _reference_quantize(args, H, V)
     mean_macs_per_call = sum(r * H * V for r in rows_list) / len(rows_list)
     # bounded per-step sample sized so warm-up + steps stay near a minute of CPU time
     vslice = 256

@@ -20,7 +20,8 @@ import threading
 __all__ = [
     "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32",
     "logits_w4a16_nvfp4", "lmhead_logits_bf16_f32", "lmhead_logits_f32",
-    "lmhead_logits_w4a16_nvfp4", "status_string", "device_status", "DTYPE_BF16", "DTYPE_F16",
+    "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "nvfp4_quantize",
+    "nvfp4_quantize_workspace_bytes", "status_string", "device_status", "DTYPE_BF16", "DTYPE_F16",
     "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS",
 ]
 
@@ -66,6 +67,10 @@ def load_library():
         lib.lmhead_logits_f32.restype = i32
         lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
         lib.lmhead_logits_w4a16_nvfp4.restype = i32
+        lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
+        lib.lmhead_nvfp4_quantize_workspace_bytes.restype = ctypes.c_size_t
+        lib.lmhead_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.lmhead_nvfp4_quantize.restype = i32
         lib.lmhead_status_string.argtypes = [i32]
         lib.lmhead_status_string.restype = ctypes.c_char_p
         lib.lmhead_device_status.argtypes = [i32]
@@ -99,6 +104,47 @@ def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: in
                               logits_ptr: int, stream: int = 0) -> int:
     return load_library().lmhead_logits_w4a16_nvfp4(hidden_ptr, rows, H, packed_ptr, scales_ptr,
                                                      w_global_scale, V, alpha, logits_ptr, stream)
+
+
+def nvfp4_quantize_workspace_bytes() -> int:
+    return int(load_library().lmhead_nvfp4_quantize_workspace_bytes())
+
+
+def lmhead_nvfp4_quantize(w_ptr: int, V: int, H: int, packed_ptr: int, scales_ptr: int,
+                          g_ptr: int, workspace_ptr: int, workspace_bytes: int,
+                          stream: int = 0) -> int:
+    return load_library().lmhead_nvfp4_quantize(w_ptr, V, H, packed_ptr, scales_ptr, g_ptr,
+                                                workspace_ptr, workspace_bytes, stream)
+
+
+def nvfp4_quantize(W, workspace=None, out=None, stream=None):
+    """Quantise a bf16 CUDA tensor W [V, H] (H % 16 == 0) for the NVFP4 head. Returns (packed uint8
+    [V, H/2], scales uint8 [V, H/16], g: fp32 CUDA tensor of one element), all on W's device;
+    runs asynchronously on ``stream``. ``workspace`` (a CUDA tensor of at least
+    nvfp4_quantize_workspace_bytes() bytes) is allocated here when not given, and so are the
+    outputs unless ``out`` = (packed, scales, g) supplies them."""
+    import torch
+    _check(W.dtype == torch.bfloat16 and W.dim() == 2 and W.is_cuda and W.is_contiguous(),
+           "a contiguous bf16 CUDA matrix is required")
+    V, H = W.shape
+    if out is None:
+        packed = torch.empty((V, H // 2), dtype=torch.uint8, device=W.device)
+        scales = torch.empty((V, H // 16), dtype=torch.uint8, device=W.device)
+        g = torch.empty((1,), dtype=torch.float32, device=W.device)
+    else:
+        packed, scales, g = out
+        _check(packed.dtype == torch.uint8 and tuple(packed.shape) == (V, H // 2) and
+               scales.dtype == torch.uint8 and tuple(scales.shape) == (V, H // 16) and
+               g.dtype == torch.float32 and g.numel() == 1, "out = (packed, scales, g) mismatch")
+    need = nvfp4_quantize_workspace_bytes()
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=W.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lmhead_nvfp4_quantize(W.data_ptr(), V, H, packed.data_ptr(), scales.data_ptr(),
+                               g.data_ptr(), workspace.data_ptr(), nbytes, _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_nvfp4_quantize")
+    return packed, scales, g
 
 
 def status_string(status: int) -> str:

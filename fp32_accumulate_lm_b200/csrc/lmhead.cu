@@ -16,6 +16,7 @@
 #include "lmhead.h"
 #include "lmhead_bf16.cuh"
 #include "lmhead_nvfp4.cuh"
+#include "lmhead_quant.cuh"
 
 namespace {
 
@@ -254,6 +255,55 @@ void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) 
 
 void lmhead_debug_set_nvfp4_conversion(int path) {
   g_nvfp4_path.store(path == 1 || path == 2 ? path : 0);
+}
+
+size_t lmhead_nvfp4_quantize_workspace_bytes(void) {
+  return (size_t)lmh::kQuantMaxPartials * sizeof(uint32_t);
+}
+
+int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
+                          uint8_t* w_scales, float* w_global_scale, void* workspace,
+                          size_t workspace_bytes, lmhead_stream_t stream) {
+  if (V <= 0 || H <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 16 != 0) return LMHEAD_ERR_ALIGN;
+  if (V > kInt32Max || H > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (w == nullptr || w_packed == nullptr || w_scales == nullptr || w_global_scale == nullptr ||
+      workspace == nullptr) {
+    return LMHEAD_ERR_NULL;
+  }
+  if (!aligned(w, 16) || !aligned(w_packed, 8) || !aligned(w_global_scale, 4) ||
+      !aligned(workspace, 4)) {
+    return LMHEAD_ERR_ALIGN;
+  }
+  const int64_t n = V * H;
+  const struct { const void* p; int64_t bytes; } regions[5] = {
+      {w, n * 2}, {w_packed, n / 2}, {w_scales, n / 16}, {w_global_scale, 4},
+      {workspace, (int64_t)workspace_bytes}};
+  for (int i = 0; i < 5; ++i)
+    for (int j = i + 1; j < 5; ++j)
+      if (overlaps(regions[i].p, regions[i].bytes, regions[j].p, regions[j].bytes))
+        return LMHEAD_ERR_ALIAS;
+  DeviceInfo dev;
+  const int st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+  // Pass 1 grid: a few CTAs per SM, one partial word each, never past the workspace.
+  const int64_t n_chunks = n / 8;
+  int64_t grid = (int64_t)dev.num_sms * 4;
+  const int64_t by_work = (n_chunks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
+  if (grid > by_work) grid = by_work;
+  if (grid > lmh::kQuantMaxPartials) grid = lmh::kQuantMaxPartials;
+  if (workspace_bytes < (size_t)grid * sizeof(uint32_t)) return LMHEAD_ERR_SHAPE;
+  const int64_t n_blocks = n / 16;
+  int64_t grid2 = (int64_t)dev.num_sms * 4;
+  const int64_t by_blocks = (n_blocks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
+  if (grid2 > by_blocks) grid2 = by_blocks;
+  uint32_t* partial = reinterpret_cast<uint32_t*>(workspace);
+  lmh::nvfp4_absmax_kernel<<<(unsigned)grid, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(w), n_chunks, partial);
+  lmh::nvfp4_encode_kernel<<<(unsigned)grid2, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(w), n_blocks, partial, (int)grid,
+      reinterpret_cast<uint2*>(w_packed), w_scales, w_global_scale);
+  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
 int lmhead_device_status(int clear) {

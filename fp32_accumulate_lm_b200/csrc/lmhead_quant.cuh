@@ -1,0 +1,120 @@
+// NVFP4 quantiser for the W4A16 head's weights: an absmax pass, then an encode pass, as the
+// two kernels lm_head_nvfp4_rows.rs / mtp_head/new_bf16_moe.rs name ("quantize_to_nvfp4(w, n, k,
+// gpu, absmax_k, nvfp4_k, stream)"). The pages print no rules; this library's reading takes every
+// decision as one IEEE binary32 operation, so a CPU re-implementation can match it bit for bit:
+//   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
+//   per 16-element block:  s = RN_e4m3(bmax / (6 * g)), saturating at 448
+//   per element:           q = RN_e2m1(w / (e4m3(s) * g)), saturating at 6; the sign is kept
+//                          only on a non-zero magnitude
+// RN is round to nearest, ties to the even code (the conversions' .rn mode).
+//
+// Both passes stream W once (HBM-bound); the encode pass's divisions are IEEE (div.rn).
+#pragma once
+
+#include "lmhead_common.cuh"
+
+namespace lmh {
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantMaxPartials = 1024;  // absmax partials: one 32-bit word per CTA of pass 1
+
+// Largest |bf16| of a 16-byte chunk as its magnitude bits (0x0000..0x7F80 for finite values and
+// infinity, ordered like the values).
+__device__ __forceinline__ uint32_t chunk_absmax_bits(const uint4& c) {
+  const uint32_t m = __vmaxu2(__vmaxu2(c.x & 0x7FFF7FFFu, c.y & 0x7FFF7FFFu),
+                              __vmaxu2(c.z & 0x7FFF7FFFu, c.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
+  v = __reduce_max_sync(0xffffffffu, v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0u;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  const uint32_t r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// Pass 1: partial[blockIdx.x] = largest |w| (magnitude bits) over this CTA's grid-stride share.
+__global__ void __launch_bounds__(kQuantThreads)
+    nvfp4_absmax_kernel(const uint4* __restrict__ w, int64_t n_chunks, uint32_t* partial) {
+  __shared__ uint32_t red[32];
+  uint32_t m = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_chunks; i += stride)
+    m = max(m, chunk_absmax_bits(__ldcs(w + i)));
+  m = block_max_u32(m, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+}
+
+// Nearest E4M3 code of t >= 0 (saturating at 448): the conversion packs two values; both lanes
+// get t, so either byte is the answer.
+__device__ __forceinline__ uint32_t rn_e4m3_code(float t) {
+  uint16_t two;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(two) : "f"(t));
+  return two & 0xFFu;
+}
+
+// Exact value of an E4M3 code (through the e4m3 -> f16 conversion, which is exact).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h2;
+  const uint16_t both = (uint16_t)(code | (code << 8));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(both));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Nearest E2M1 code of x (saturating at +-6), with no negative zero.
+__device__ __forceinline__ uint32_t rn_e2m1_code(float x) {
+  uint16_t two;
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %1;\n\tcvt.u16.u8 %0, q;\n\t}"
+      : "=h"(two)
+      : "f"(x));
+  const uint32_t c = two & 0x0Fu;
+  return (c & 7u) ? c : 0u;
+}
+
+// Pass 2: every CTA reduces the partials to amax (the same value everywhere), then each thread
+// encodes 16-element blocks: 32 bytes of W in, 8 bytes of codes and one scale byte out.
+__global__ void __launch_bounds__(kQuantThreads)
+    nvfp4_encode_kernel(const uint4* __restrict__ w, int64_t n_blocks,
+                        const uint32_t* __restrict__ partial, int n_partial, uint2* packed,
+                        uint8_t* scales, float* g_out) {
+  __shared__ uint32_t red[32];
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < n_partial; i += blockDim.x) m = max(m, partial[i]);
+  m = block_max_u32(m, red);
+  const float amax = __uint_as_float(m << 16);
+  const float g = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+  const float six_g = __fmul_rn(6.0f, g);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks; b += stride) {
+    const uint4 c0 = __ldcs(w + 2 * b);
+    const uint4 c1 = __ldcs(w + 2 * b + 1);
+    const float bmax =
+        __uint_as_float(max(chunk_absmax_bits(c0), chunk_absmax_bits(c1)) << 16);
+    const uint32_t s = rn_e4m3_code(__fdiv_rn(bmax, six_g));
+    const float d = __fmul_rn(e4m3_value(s), g);
+    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
+      const float w0 = __uint_as_float(words[i] << 16);
+      const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
+      const uint32_t q0 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w0, d)) : 0u;
+      const uint32_t q1 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w1, d)) : 0u;
+      out[i >> 2] |= (q0 | (q1 << 4)) << (8 * (i & 3));
+    }
+    packed[b] = make_uint2(out[0], out[1]);
+    scales[b] = (uint8_t)s;
+  }
+}
+
+}  // namespace lmh

@@ -27,7 +27,7 @@
  *  - Matrices are row-major and contiguous: hidden [rows, H], W [V, H] (used transposed), logits
  *    [rows, V].
  *  - A call validates its arguments synchronously on the host and launches nothing on error; it
- *    then enqueues ONE kernel on `stream` and returns without waiting. Faults surface at the
+ *    then enqueues its kernel (two for the quantiser) on `stream` and returns without waiting. Faults surface at the
  *    caller's next synchronisation. There is no fallback path of any kind.
  *  - rows == 0 is valid and launches nothing.
  *  - Determinism: the same inputs give the same bits on every run (no atomics, no split-K). Each
@@ -40,6 +40,7 @@
 #ifndef LMHEAD_H
 #define LMHEAD_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -121,6 +122,33 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
 int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,
                               const uint8_t* w_scales, float w_global_scale, int64_t V,
                               float alpha, void* logits, lmhead_stream_t stream);
+
+/*
+ * NVFP4 quantiser: bf16 W -> the three inputs of lmhead_logits_w4a16_nvfp4. The pages name a
+ * two-kernel quantiser, an absmax pass then an encode pass (lm_head_nvfp4_rows.rs and
+ * mtp_head/new_bf16_moe.rs, quantize_to_nvfp4(w, n, k, gpu, absmax_k, nvfp4_k, stream)), but print
+ * no rules. This library's rules take every decision as one IEEE binary32 operation:
+ *   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
+ *   w_scales[v, j]  = RN_e4m3(max_{k in block j} |w[v, k]| / (6 * g)), saturating at 448
+ *   code[v, k]      = RN_e2m1(w[v, k] / (e4m3(w_scales[v, k/16]) * g)), saturating at +-6,
+ *                     with no negative zero; RN = nearest, ties to the even code
+ * Packing as lmhead_logits_w4a16_nvfp4 reads it (element 2j in the low nibble of byte j).
+ *
+ *   w               bf16 [V, H], 16-byte aligned, finite    H > 0, H % 16 == 0, V > 0
+ *   w_packed        u8 [V, H/2], 8-byte aligned (output)
+ *   w_scales        u8 [V, H/16] (output)
+ *   w_global_scale  one fp32 in DEVICE memory, 4-byte aligned (output: g)
+ *   workspace       device scratch of at least lmhead_nvfp4_quantize_workspace_bytes() bytes,
+ *                   4-byte aligned, owned by the caller; it carries the absmax pass's per-block
+ *                   maxima to the encode pass and may be reused once the call's work is done
+ * No region may overlap another. Two kernels are enqueued on `stream`: the absmax pass reads W
+ * once, the encode pass reads it again and writes the outputs. Returns an lmhead_status
+ * (LMHEAD_ERR_SHAPE also when the workspace is too small).
+ */
+size_t lmhead_nvfp4_quantize_workspace_bytes(void);
+int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
+                          uint8_t* w_scales, float* w_global_scale, void* workspace,
+                          size_t workspace_bytes, lmhead_stream_t stream);
 
 /* A static English description of a status code. Never NULL. */
 const char* lmhead_status_string(int status);

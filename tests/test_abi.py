@@ -100,6 +100,22 @@ def test_general_entry_argument_errors(lib):
     assert f(0, lm.DTYPE_F16, 0, 64, 0, 128, 1.0, 0, 0, 0) == 0             # rows == 0: no-op
 
 
+def test_quantiser_argument_errors(lib):
+    f = lm.lmhead_nvfp4_quantize
+    WS = 0x50000000
+    need = lm.nvfp4_quantize_workspace_bytes()
+    assert need >= 4 and need % 4 == 0
+    assert f(A16, 0, 64, B16, C16, 0x60000000, WS, need, 0) == 2
+    assert f(A16, 4, 40, B16, C16, 0x60000000, WS, need, 0) == 3        # H % 16 != 0
+    assert f(0, 4, 64, B16, C16, 0x60000000, WS, need, 0) == 1
+    assert f(A16, 4, 64, B16, C16, 0x60000000, 0, need, 0) == 1         # no workspace
+    assert f(A16 + 8, 4, 64, B16, C16, 0x60000000, WS, need, 0) == 3
+    assert f(A16, 4, 64, B16 + 4, C16, 0x60000000, WS, need, 0) == 3    # packed not 8-aligned
+    assert f(A16, 4, 64, B16, C16, 0x60000002, WS, need, 0) == 3
+    assert f(A16, 4, 64, A16 + 16, C16, 0x60000000, WS, need, 0) == 7   # packed over W
+    assert f(A16, 4, 64, B16, C16, B16 + 8, WS, need, 0) == 7           # g inside packed
+
+
 def test_rows_zero_launches_nothing(lib):
     # rows == 0 is a no-op even with NULL pointers (no CUDA call is made)
     assert lm.lmhead_logits_bf16_f32(0, 0, 64, 0, 128, 1.0, 0, 0) == 0

@@ -1,0 +1,104 @@
+"""GPU parity of the NVFP4 quantiser (lmhead_nvfp4_quantize) against the CPU oracle, bit for bit.
+
+lm_head_nvfp4_rows.rs and mtp_head/new_bf16_moe.rs name a two-kernel quantiser (absmax, then
+encode); the rules are this library's reading, every decision one IEEE binary32 operation, so the
+codes, scales and g must equal the oracle's exactly. The quantised head then runs through the
+NVFP4 entry and is checked against the oracle head.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp32_accumulate_lm_b200 as lm
+from fp32_accumulate_lm_b200 import synth
+from gpu_helpers import check_status, dev_bf16, gpu_nvfp4
+from tolerance import assert_bf16_close
+
+pytestmark = pytest.mark.gpu
+
+
+def bf16_bits(x):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def gpu_quantize(w_bits):
+    p, s, g = lm.nvfp4_quantize(dev_bf16(w_bits))
+    check_status()
+    return p.cpu().numpy(), s.cpu().numpy(), np.float32(g.item())
+
+
+def assert_same_as_oracle(w_bits, what):
+    p, s, g = gpu_quantize(w_bits)
+    p0, s0, g0 = oracle.nvfp4_quantize(w_bits)
+    assert g == g0, (what, g, g0)
+    assert np.array_equal(s, s0), (what, int((s != s0).sum()))
+    assert np.array_equal(p, p0), (what, int((p != p0).sum()))
+    return p, s, g
+
+
+@pytest.mark.parametrize("V,H,seed", [(1, 16, 1), (3, 48, 2), (257, 2048, 3), (1024, 4096, 4)])
+def test_seeded_weights_match_oracle(V, H, seed):
+    assert_same_as_oracle(synth.weight(V, H, 0.02, seed), f"{V}x{H}")
+
+
+def test_block_magnitudes_across_the_e4m3_range():
+    """Blocks scaled from 1e-6 to 1e3 relative to each other: scales from subnormal E4M3 codes
+    to saturation, and codes that saturate at 6 where the block scale saturates."""
+    rng = np.random.default_rng(81)
+    V, H = 64, 512
+    w = rng.normal(0, 1, (V, H)) * (10.0 ** rng.uniform(-6, 3, (V, H // 16))).repeat(16, axis=1)
+    assert_same_as_oracle(bf16_bits(w), "spread")
+
+
+def test_ties_signed_zeros_and_exact_values():
+    """amax = 2688 makes g = 1; values on E2M1 midpoints exercise ties to the even code, -0 and
+    tiny negatives must come out as code 0."""
+    H = 64
+    w = np.zeros((4, H))
+    w[0, 0] = 2688.0
+    w[1, :16] = [6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -0.25, -0.75, -2.5, -5, -0.0, -1e-3, 3, -6]
+    w[2, :16] = [0.5] * 16
+    w[3, 16:32] = np.linspace(-6, 6, 16)
+    p, s, g = assert_same_as_oracle(bf16_bits(w), "ties")
+    assert g == np.float32(1.0)
+    codes = np.stack([p & 0x0F, p >> 4], axis=2).reshape(4, H)
+    assert list(codes[1, :16]) == [7, 0, 2, 2, 4, 4, 6, 6, 0, 10, 12, 14, 0, 0, 5, 15]
+
+
+def test_all_zero_and_single_spike():
+    z = np.zeros((5, 32), np.uint16)
+    p, s, g = assert_same_as_oracle(z, "zero")
+    assert g == np.float32(1.0) and not p.any() and not s.any()
+    w = np.zeros((3, 64))
+    w[2, 63] = -3.0e38                     # near the top of bf16's range
+    w[0, 1] = 1e-38                        # below every block scale after g is set by the spike
+    assert_same_as_oracle(bf16_bits(w), "spike")
+
+
+def test_quantised_head_runs_through_the_nvfp4_entry():
+    """quantise on the GPU, then the W4A16 head on the GPU against the oracle head on the same
+    codes."""
+    rows, H, V = 17, 1024, 3000
+    wb = synth.weight(V, H, 0.02, 85)
+    h = synth.hidden(rows, H, 86)
+    pd, sd, gd = lm.nvfp4_quantize(dev_bf16(wb))
+    g = float(gd.item())
+    got = gpu_nvfp4(h, pd, sd, g, 0.125)
+    ref, absum = oracle.logits_w4a16_nvfp4(h, pd.cpu().numpy(), sd.cpu().numpy(), g, 0.125)
+    assert_bf16_close(got, ref, absum, "quantised head")
+
+
+def test_workspace_is_reused_and_rejected_when_too_small():
+    wb = synth.weight(300, 256, 0.02, 87)
+    W = dev_bf16(wb)
+    ws = torch.zeros(lm.nvfp4_quantize_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    first = lm.nvfp4_quantize(W, workspace=ws)
+    second = lm.nvfp4_quantize(W, workspace=ws)
+    check_status()
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)
+    tiny = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(lm.LmheadError):
+        lm.nvfp4_quantize(W, workspace=tiny)
