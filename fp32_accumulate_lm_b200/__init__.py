@@ -20,7 +20,8 @@ import threading
 __all__ = [
     "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32",
     "logits_w4a16_nvfp4", "lmhead_logits_bf16_f32", "lmhead_logits_f32",
-    "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "nvfp4_quantize",
+    "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "lmhead_nvfp4_quantize_noalloc",
+    "nvfp4_quantize",
     "nvfp4_quantize_workspace_bytes", "status_string", "device_status", "DTYPE_BF16", "DTYPE_F16",
     "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS",
 ]
@@ -71,6 +72,8 @@ def load_library():
         lib.lmhead_nvfp4_quantize_workspace_bytes.restype = ctypes.c_size_t
         lib.lmhead_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
         lib.lmhead_nvfp4_quantize.restype = i32
+        lib.lmhead_nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        lib.lmhead_nvfp4_quantize_noalloc.restype = i32
         lib.lmhead_status_string.argtypes = [i32]
         lib.lmhead_status_string.restype = ctypes.c_char_p
         lib.lmhead_device_status.argtypes = [i32]
@@ -115,6 +118,14 @@ def lmhead_nvfp4_quantize(w_ptr: int, V: int, H: int, packed_ptr: int, scales_pt
                           stream: int = 0) -> int:
     return load_library().lmhead_nvfp4_quantize(w_ptr, V, H, packed_ptr, scales_ptr, g_ptr,
                                                 workspace_ptr, workspace_bytes, stream)
+
+
+def lmhead_nvfp4_quantize_noalloc(w_ptr: int, V: int, H: int, packed_ptr: int, scales_ptr: int,
+                                  g_ptr: int, stream: int = 0) -> int:
+    """The quantiser for callers that cannot allocate device memory: the library's own 4 KB
+    per-GPU scratch replaces the workspace (see include/lmhead.h)."""
+    return load_library().lmhead_nvfp4_quantize_noalloc(w_ptr, V, H, packed_ptr, scales_ptr,
+                                                        g_ptr, stream)
 
 
 def nvfp4_quantize(W, workspace=None, out=None, stream=None):

@@ -228,6 +228,31 @@ int pick_nsub(int32_t bn, int smem_budget) {
   return 1;
 }
 
+// ---- library-held scratch for lmhead_nvfp4_quantize_noalloc
+// The absmax pass's per-CTA maxima, for callers that cannot hand the quantiser a workspace.
+// 4 KB per GPU, held by every GPU that loads the library until the process exits.
+static __device__ __align__(256) uint32_t g_quant_scratch[lmh::kQuantMaxPartials];
+
+std::mutex g_scratch_mu;
+uint32_t* g_scratch_ptr[kMaxDevices] = {};
+
+// The scratch array's device address on the current device. Host code may not use the array's
+// name as a device address (it names a host-side stand-in), so the address is looked up once per
+// device, with that device current, and cached.
+int quant_scratch(uint32_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMHEAD_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_quant_scratch) != cudaSuccess || ptr == nullptr)
+      return LMHEAD_ERR_LAUNCH;
+    g_scratch_ptr[dev] = static_cast<uint32_t*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return LMHEAD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -304,6 +329,24 @@ int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed
       reinterpret_cast<const uint4*>(w), n_blocks, partial, (int)grid,
       reinterpret_cast<uint2*>(w_packed), w_scales, w_global_scale);
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+int lmhead_nvfp4_quantize_noalloc(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
+                                  uint8_t* w_scales, float* w_global_scale,
+                                  lmhead_stream_t stream) {
+  // Validate first, as every entry does, so an invalid call touches no device state.
+  if (V <= 0 || H <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 16 != 0) return LMHEAD_ERR_ALIGN;
+  if (w == nullptr || w_packed == nullptr || w_scales == nullptr || w_global_scale == nullptr)
+    return LMHEAD_ERR_NULL;
+  uint32_t* scratch = nullptr;
+  const int st = quant_scratch(&scratch);
+  if (st != LMHEAD_OK) return st;
+  // The quantiser needs one word per CTA of its absmax pass; it sizes that grid to at most
+  // kQuantMaxPartials, so the 4 KB array always suffices, and the workspace entry rejects a
+  // call that would need more.
+  return lmhead_nvfp4_quantize(w, V, H, w_packed, w_scales, w_global_scale, scratch,
+                               sizeof(g_quant_scratch), stream);
 }
 
 int lmhead_device_status(int clear) {

@@ -150,6 +150,27 @@ int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed
                           uint8_t* w_scales, float* w_global_scale, void* workspace,
                           size_t workspace_bytes, lmhead_stream_t stream);
 
+/*
+ * lmhead_nvfp4_quantize without a workspace argument, for callers that cannot obtain device
+ * memory of their own: code that is handed its weight and output buffers by another component
+ * (a model loader or a serving engine's memory pool) and is not allowed to call cudaMalloc, which
+ * can synchronise the whole device and bypasses the pool that owns the GPU's memory. The paper
+ * has no counterpart to this entry point; it exists for those callers.
+ *
+ * Same arguments, rules and results as lmhead_nvfp4_quantize. The absmax pass's scratch is a 4 KB
+ * array that the library keeps on every GPU it is loaded on, until the process exits; the call
+ * allocates nothing. Its first call on a device looks up that array's device address (a host-side
+ * setup step, once per device, done while that device is current), so make that first call
+ * before any stream capture. All calls on a device share the one array: calls whose work overlaps
+ * on the GPU (on different streams without ordering between them) race and give undefined
+ * results, so order them. The array needs no clearing; each call's absmax pass writes every word
+ * its encode pass reads. A call that would need more than the 4 KB is rejected with
+ * LMHEAD_ERR_SHAPE (the quantiser's grid is sized to stay within it). Returns an lmhead_status.
+ */
+int lmhead_nvfp4_quantize_noalloc(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
+                                  uint8_t* w_scales, float* w_global_scale,
+                                  lmhead_stream_t stream);
+
 /* A static English description of a status code. Never NULL. */
 const char* lmhead_status_string(int status);
 
