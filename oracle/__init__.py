@@ -78,6 +78,11 @@ def _load():
         lib.oracle_logits_w4a16_nvfp4.argtypes = [u16p, i64, i64, u8p, u8p, ctypes.c_float, i64,
                                                   ctypes.c_float, u16p, f64p, ctypes.c_int]
         lib.oracle_logits_w4a16_nvfp4.restype = ctypes.c_int
+        lib.oracle_logprobs_f32.argtypes = [u16p, ctypes.c_int, i64, i64, u16p, i64,
+                                            ctypes.c_float, ctypes.c_void_p,
+                                            ctypes.POINTER(ctypes.c_int32), f32p, f32p,
+                                            ctypes.c_int]
+        lib.oracle_logprobs_f32.restype = ctypes.c_int
         lib.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, u8p, u8p, f32p]
         lib.oracle_nvfp4_quantize.restype = ctypes.c_int
         lib.oracle_rn_e4m3.argtypes = [ctypes.c_float]
@@ -233,3 +238,31 @@ def nvfp4_quantize(w_bits: np.ndarray):
     if rc != 0:
         raise RuntimeError(f"oracle_nvfp4_quantize failed with {rc}")
     return packed, scales, np.float32(g[0])
+
+
+# ---------------------------------------------------------------- log-probabilities
+
+def logprobs_f32(hidden_bits: np.ndarray, w_bits: np.ndarray, alpha: float, targets: np.ndarray,
+                 bias_bits=None, dtype: str = "bf16", threads: int | None = None):
+    """(logprobs [rows], lse [rows]) as float32: the log-softmax of the fp32 logits of
+    logits_f32 at each row's target token (NaN for a target outside [0, V))."""
+    h = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    t = np.ascontiguousarray(targets, dtype=np.int32)
+    rows, H = h.shape
+    V = w.shape[0]
+    if w.shape[1] != H or t.shape != (rows,):
+        raise ValueError("shape mismatch")
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    lp = np.zeros(rows, dtype=np.float32)
+    lse = np.zeros(rows, dtype=np.float32)
+    if rows == 0:
+        return lp, lse
+    rc = _load().oracle_logprobs_f32(_ptr(h, ctypes.c_uint16), 1 if dtype == "f16" else 0, rows, H,
+                                     _ptr(w, ctypes.c_uint16), V, ctypes.c_float(alpha),
+                                     None if b is None else b.ctypes.data,
+                                     _ptr(t, ctypes.c_int32), _ptr(lp, ctypes.c_float),
+                                     _ptr(lse, ctypes.c_float), threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_logprobs_f32 failed with {rc}")
+    return lp, lse

@@ -38,6 +38,14 @@
  *    [16j, 16j+16). g is the per-tensor decode multiplier (w = q * s * g).
  *  - Rounding is IEEE round-to-nearest-even, done once from double.
  *
+ * Log-probabilities of given tokens (oracle_logprobs_f32). The first page's "Purpose" wants fp32
+ * logits for RL training-inference consistency and for speculative decoding, where the logits
+ * drive rejection sampling; what those consume is the log-softmax. Reading: with z[r, v] the fp32
+ * logits above (bias and alpha applied, rounded to fp32),
+ *   lse[r] = log sum_v exp(z[r, v]),   logprob[r] = z[r, target[r]] - lse[r]
+ * computed in double from the fp32 z (max-shifted), each rounded once to fp32; a target outside
+ * [0, V) gives NaN.
+ *
  * NVFP4 quantiser (oracle_nvfp4_quantize). lm_head_nvfp4_rows.rs and mtp_head/new_bf16_moe.rs
  * ("quantize_to_nvfp4(w, n, k, gpu, absmax_k, nvfp4_k, stream)": an absmax kernel, then an encode
  * kernel) name it but print no rules. Reading, with every step one IEEE binary32 operation so that
@@ -191,6 +199,37 @@ int oracle_logits_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H
 int oracle_logits_bf16_f32(const uint16_t* hidden, int64_t rows, int64_t H, const uint16_t* W,
                            int64_t V, float alpha, float* logits, double* abs_sum, int threads) {
   return oracle_logits_f32(hidden, 0, rows, H, W, V, alpha, NULL, logits, abs_sum, threads);
+}
+
+/* ---------------------------------------------------------------- log-probabilities */
+
+int oracle_logprobs_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                        const uint16_t* W, int64_t V, float alpha, const uint16_t* bias,
+                        const int32_t* targets, float* logprobs, float* lse, int threads) {
+  if (rows < 0 || H <= 0 || V <= 0) return 1;
+  if (rows == 0) return 0;
+  if (!targets || !logprobs) return 1;
+  float* z = (float*)malloc((size_t)rows * (size_t)V * sizeof(float));
+  if (!z) return 2;
+  int rc = oracle_logits_f32(hidden, dtype, rows, H, W, V, alpha, bias, z, NULL, threads);
+  if (rc != 0) {
+    free(z);
+    return rc;
+  }
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* zr = z + r * V;
+    double m = -INFINITY;
+    for (int64_t v = 0; v < V; ++v)
+      if ((double)zr[v] > m) m = (double)zr[v];
+    double sum = 0.0;
+    for (int64_t v = 0; v < V; ++v) sum += exp((double)zr[v] - m);
+    const double l = m + log(sum);
+    if (lse) lse[r] = oracle_round_f32(l);
+    const int32_t t = targets[r];
+    logprobs[r] = (t >= 0 && t < V) ? oracle_round_f32((double)zr[t] - l) : (float)NAN;
+  }
+  free(z);
+  return 0;
 }
 
 /* ---------------------------------------------------------------- the NVFP4 quantiser */

@@ -55,6 +55,15 @@ int oracle_logits_w4a16_nvfp4(const uint16_t* hidden, int64_t rows, int64_t H,
                               float alpha, uint16_t* logits, double* abs_sum, int threads);
 
 /*
+ * Log-probabilities of given tokens: with z the fp32 logits of oracle_logits_f32 (same arguments),
+ * lse[r] = log sum_v exp(z[r, v]) and logprobs[r] = z[r, targets[r]] - lse[r], computed in double
+ * from the fp32 z and rounded once; NaN for a target outside [0, V). lse may be NULL.
+ */
+int oracle_logprobs_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                        const uint16_t* W, int64_t V, float alpha, const uint16_t* bias,
+                        const int32_t* targets, float* logprobs, float* lse, int threads);
+
+/*
  * NVFP4 quantiser (this library's reading; every decision step one IEEE binary32 operation):
  * amax = max|w|, g = amax / 2688 (1 when amax = 0); per 16-element block s = RN_e4m3(bmax / (6g))
  * saturating; per element q = RN_e2m1(w / (e4m3(s) * g)) saturating, sign only on non-zero

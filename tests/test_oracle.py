@@ -574,3 +574,55 @@ def test_quantiser_round_trip_error_is_within_half_a_code():
             x = abs(wf[v, k]) / unit if unit > 0 else 0.0
             step = 0.5 if x < 2 else (1.0 if x < 4 else 2.0)
             assert abs(deq - wf[v, k]) <= 0.5 * step * unit * (1 + 1e-6) + 1e-30, (v, k)
+
+
+# ---------------------------------------------------------------- log-probabilities of tokens
+# The first page's "Purpose": fp32 logits for RL training-inference consistency and for the
+# rejection sampling of speculative decoding, which consume the log-softmax. Reading:
+#     logprob[r] = z[r, t_r] - log sum_v exp(z[r, v]),  z = the fp32 logits.
+
+def test_logprobs_uniform_logits_give_minus_log_v():
+    rows, H, V = 3, 32, 1000
+    h = bf16_bits_of_f32(np.random.default_rng(101).normal(0, 1, (rows, H)))
+    w = np.zeros((V, H), np.uint16)
+    t = np.array([0, 499, 999], np.int32)
+    lp, lse = oracle.logprobs_f32(h, w, 0.5, t)
+    assert np.allclose(lse, np.float32(math.log(V)), rtol=0, atol=1e-6)
+    assert np.allclose(lp, np.float32(-math.log(V)), rtol=0, atol=1e-6)
+
+
+def test_logprobs_two_level_closed_form():
+    """Bias-only logits: one token at a, the other V - 1 at b."""
+    rows, H, V, a, b = 2, 16, 64, 3.0, -1.0
+    h = bf16_bits_of_f32(np.ones((rows, H)))
+    w = np.zeros((V, H), np.uint16)
+    bias = np.full(V, b)
+    bias[7] = a
+    t = np.array([7, 8], np.int32)
+    lp, lse = oracle.logprobs_f32(h, w, 1.0, t, bias_bits=bf16_bits_of_f32(bias))
+    want_lse = math.log(math.exp(a) + (V - 1) * math.exp(b))
+    assert abs(lse[0] - want_lse) < 1e-6 and abs(lse[1] - want_lse) < 1e-6
+    assert abs(lp[0] - (a - want_lse)) < 1e-6 and abs(lp[1] - (b - want_lse)) < 1e-6
+
+
+def test_logprobs_match_scipy_logsumexp_of_the_oracle_logits():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(102)
+    rows, H, V = 6, 128, 3001
+    h = bf16_bits_of_f32(rng.normal(0, 1, (rows, H)))
+    w = bf16_bits_of_f32(rng.normal(0, 0.2, (V, H)))
+    b = bf16_bits_of_f32(rng.normal(0, 1.0, V))
+    t = rng.integers(0, V, rows).astype(np.int32)
+    for dtype in ("bf16",):
+        z, _ = oracle.logits_f32(h, w, 0.125, bias_bits=b, dtype=dtype)
+        lp, lse = oracle.logprobs_f32(h, w, 0.125, t, bias_bits=b, dtype=dtype)
+        want_lse = logsumexp(z.astype(np.float64), axis=1)
+        assert np.allclose(lse, want_lse, rtol=2e-7, atol=0)
+        assert np.allclose(lp, z[np.arange(rows), t] - want_lse, rtol=0, atol=1e-6)
+
+
+def test_logprobs_out_of_range_target_is_nan():
+    h = bf16_bits_of_f32(np.ones((2, 16)))
+    w = bf16_bits_of_f32(np.ones((10, 16)))
+    lp, _ = oracle.logprobs_f32(h, w, 1.0, np.array([-1, 10], np.int32))
+    assert np.isnan(lp).all()
