@@ -47,6 +47,9 @@ WORKLOAD_TEXT = {
              "scale, bf16 hidden and logits, alpha=1/8",
     "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
                     "fp32 out, alpha=1/8",
+    "prefill_logprobs": "prefill LM head computing log-probabilities of one target token per row "
+                        "(log-softmax in the epilogue, no logits written): rows=8192, H=4096, "
+                        "V=151936, bf16 in, fp32 out, alpha=1/8",
     "nvfp4_quantize": "NVFP4 quantiser (absmax pass, then encode pass) of a bf16 W[151936, 2048] "
                       "into E2M1 codes, E4M3 block scales and an fp32 global scale",
     "decode_f16_bias": "decode LM head with fp16 operands and an fp16 embedding bias: rows "
@@ -165,7 +168,7 @@ class Workload:
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
                 "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16,
-                "nvfp4_quantize": synth.SEED_NVFP4}[name]
+                "nvfp4_quantize": synth.SEED_NVFP4, "prefill_logprobs": synth.SEED_PREFILL}[name]
         rmax = max(rows_list)
         self.quantize = name == "nvfp4_quantize"
         if self.quantize:
@@ -174,6 +177,7 @@ class Workload:
             self.dtype = torch.bfloat16
             self.bias = None
             self.nvfp4 = False
+            self.logprobs = False
             self.weights = [synth.weight(V, H, std, seed + i, device=device) for i in (0, 1)]
             self.hidden = self.weights[0]
             self.hid = {V: self.weights[0]}
@@ -200,6 +204,17 @@ class Workload:
             self.outs = {r: torch.empty((r, V), dtype=torch.float32, device=device)
                          for r in rows_list}
         self.hid = {r: self.hidden[:r] for r in rows_list}
+        self.general = self.bias is not None or self.dtype != torch.bfloat16  # lmhead_logits_f32
+        self.logprobs = name == "prefill_logprobs"
+        if self.logprobs:
+            import fp32_accumulate_lm_b200 as lm
+            gen = torch.Generator(device="cpu")
+            gen.manual_seed(seed + 700_000)
+            self.targets = torch.randint(0, V, (rmax,), generator=gen, dtype=torch.int32).to(device)
+            self.outs = {r: torch.empty((r,), dtype=torch.float32, device=device) for r in rows_list}
+            self.lse = {r: torch.empty((r,), dtype=torch.float32, device=device) for r in rows_list}
+            self.ws = torch.empty((lm.logprobs_workspace_bytes(rmax, V),), dtype=torch.uint8,
+                                  device=device)
         self.calls = 0
 
     def call(self, r: int, hidden=None, out=None, stream=None):
@@ -217,7 +232,10 @@ class Workload:
         o = self.outs[r] if out is None else out
         if self.nvfp4:
             lm.logits_w4a16_nvfp4(h, w[0], w[1], self.g, self.alpha, out=o, stream=stream)
-        elif self.bias is not None or self.dtype != torch.bfloat16:
+        elif self.logprobs:
+            lm.logprobs_f32(h, w, self.targets[:r], self.alpha, workspace=self.ws,
+                            out=(o, self.lse[r]), stream=stream)
+        elif self.general:
             lm.logits_f32(h, w, self.alpha, bias=self.bias, out=o, stream=stream)
         else:
             lm.logits_bf16_f32(h, w, self.alpha, out=o, stream=stream)
@@ -228,6 +246,9 @@ class Workload:
             return 2 * V * H * 2 + V * H // 2 + V * H // 16 + 4
         if self.nvfp4:
             return V * H // 2 + V * H // 16 + 4 + r * H * 2 + r * V * 2
+        if self.logprobs:  # W, hidden, targets in; the chunk pairs out and back; lp, lse out
+            n_chunks = 4 * ((V + 127) // 128)
+            return V * H * 2 + r * H * 2 + r * 4 + 2 * r * n_chunks * 8 + r * 8
         return V * H * 2 + r * H * 2 + r * V * 4 + (V * 2 if self.bias is not None else 0)
 
     def flops_of(self, r: int) -> int:
@@ -338,7 +359,7 @@ def run_ours(args) -> dict | None:
         tot_bytes += b
         tot_flops += fl
         tot_ms += mean_ms
-    tensor_bound = args.workload.startswith("prefill")
+    tensor_bound = args.workload.startswith("prefill")  # prefill, its profiling case, log-probs
     if tensor_bound:
         achieved = tot_flops / (tot_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -374,7 +395,7 @@ def run_ours(args) -> dict | None:
                    "calls_per_step": calls_per_step, "per_rows": detail},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": n_ev * (2 if wl.quantize else 1),
+        "gpu_launches": n_ev * (2 if (wl.quantize or wl.logprobs) else 1),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -481,9 +502,15 @@ def cpu_baseline(workload: str, wl) -> dict:
         b = None if wl.bias is None else wl.bias.view(torch.int16).cpu().numpy().view(np.uint16)
         dt = "f16" if wl.dtype == torch.float16 else "bf16"
 
+        tg = wl.targets.cpu().numpy() if wl.logprobs else None
+
         def run(h, vrows):
-            oracle.logits_f32(h, w[:vrows], wl.alpha, bias_bits=None if b is None else b[:vrows],
-                              dtype=dt)
+            if wl.logprobs:
+                oracle.logprobs_f32(h, w[:vrows], wl.alpha, np.minimum(tg[:h.shape[0]], vrows - 1),
+                                    dtype=dt)
+            else:
+                oracle.logits_f32(h, w[:vrows], wl.alpha,
+                                  bias_bits=None if b is None else b[:vrows], dtype=dt)
     probe_v = min(V, 4096)
     t0 = time.perf_counter()
     run(h_all[:1], probe_v)

@@ -18,7 +18,8 @@ import os
 import threading
 
 __all__ = [
-    "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32",
+    "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32", "logprobs_f32",
+    "lmhead_logprobs_f32", "logprobs_workspace_bytes",
     "logits_w4a16_nvfp4", "lmhead_logits_bf16_f32", "lmhead_logits_f32",
     "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "lmhead_nvfp4_quantize_noalloc",
     "nvfp4_quantize",
@@ -66,6 +67,11 @@ def load_library():
         lib.lmhead_logits_bf16_f32.restype = i32
         lib.lmhead_logits_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp]
         lib.lmhead_logits_f32.restype = i32
+        lib.lmhead_logprobs_workspace_bytes.argtypes = [i64, i64]
+        lib.lmhead_logprobs_workspace_bytes.restype = ctypes.c_size_t
+        lib.lmhead_logprobs_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp, vp, vp,
+                                            ctypes.c_size_t, vp]
+        lib.lmhead_logprobs_f32.restype = i32
         lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
         lib.lmhead_logits_w4a16_nvfp4.restype = i32
         lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
@@ -100,6 +106,20 @@ def lmhead_logits_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: int
                       alpha: float, bias_ptr: int, logits_ptr: int, stream: int = 0) -> int:
     return load_library().lmhead_logits_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
                                              bias_ptr or None, logits_ptr, stream)
+
+
+def logprobs_workspace_bytes(rows: int, V: int) -> int:
+    return int(load_library().lmhead_logprobs_workspace_bytes(rows, V))
+
+
+def lmhead_logprobs_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: int, V: int,
+                        alpha: float, bias_ptr: int, targets_ptr: int, logprobs_ptr: int,
+                        lse_ptr: int, workspace_ptr: int, workspace_bytes: int,
+                        stream: int = 0) -> int:
+    return load_library().lmhead_logprobs_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
+                                               bias_ptr or None, targets_ptr, logprobs_ptr,
+                                               lse_ptr or None, workspace_ptr, workspace_bytes,
+                                               stream)
 
 
 def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
@@ -246,6 +266,43 @@ def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None):
     if st != LMHEAD_OK:
         raise LmheadError(st, "lmhead_logits_f32")
     return out
+
+
+def logprobs_f32(hidden, W, targets, alpha: float = 1.0, bias=None, workspace=None, out=None,
+                 stream=None):
+    """(logprobs [rows], lse [rows]) fp32: the log-softmax of the fp32 logits alpha * (hidden @
+    W^T + bias) at each row's target token (int32 CUDA tensor [rows]), without writing logits.
+    The workspace (logprobs_workspace_bytes(rows, V) bytes) and outputs are allocated here unless
+    given (``out`` = (logprobs, lse))."""
+    import torch
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}.get(hidden.dtype)
+    _check(dt is not None and W.dtype == hidden.dtype, "bf16 or fp16 operands of one dtype required")
+    _check(hidden.dim() == 2 and W.dim() == 2 and hidden.shape[1] == W.shape[1], "shape mismatch")
+    _check(hidden.is_cuda and W.is_cuda and hidden.is_contiguous() and W.is_contiguous(),
+           "contiguous CUDA tensors required")
+    rows, H = hidden.shape
+    V = W.shape[0]
+    _check(targets.dtype == torch.int32 and targets.is_cuda and targets.is_contiguous()
+           and tuple(targets.shape) == (rows,), "targets must be a contiguous int32 [rows] tensor")
+    if bias is not None:
+        _check(bias.dtype == hidden.dtype and bias.is_cuda and bias.is_contiguous()
+               and tuple(bias.shape) == (V,), "bias must be a contiguous [V] tensor of the dtype")
+    if out is None:
+        lp = torch.empty((rows,), dtype=torch.float32, device=hidden.device)
+        lse = torch.empty((rows,), dtype=torch.float32, device=hidden.device)
+    else:
+        lp, lse = out
+    need = logprobs_workspace_bytes(rows, V)
+    if workspace is None:
+        workspace = torch.empty((max(need, 8),), dtype=torch.uint8, device=hidden.device)
+    st = lmhead_logprobs_f32(hidden.data_ptr(), dt, rows, H, W.data_ptr(), V, float(alpha),
+                             0 if bias is None else bias.data_ptr(), targets.data_ptr(),
+                             lp.data_ptr(), 0 if lse is None else lse.data_ptr(),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logprobs_f32")
+    return lp, lse
 
 
 def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha: float = 1.0,

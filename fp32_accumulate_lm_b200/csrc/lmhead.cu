@@ -367,24 +367,22 @@ int lmhead_logits_bf16_f32(const void* hidden, int64_t rows, int64_t H, const vo
                            stream);
 }
 
-int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
-                      int64_t V, float alpha, const void* bias, float* logits,
-                      lmhead_stream_t stream) {
-  if (dtype != LMHEAD_DTYPE_BF16 && dtype != LMHEAD_DTYPE_F16) return LMHEAD_ERR_SHAPE;
-  if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
-  if (H % 8 != 0) return LMHEAD_ERR_ALIGN;
-  if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
-  if (rows == 0) return LMHEAD_OK;
-  if (hidden == nullptr || W == nullptr || logits == nullptr) return LMHEAD_ERR_NULL;
-  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(logits, 4) ||
-      (bias != nullptr && !aligned(bias, 2))) {
-    return LMHEAD_ERR_ALIGN;
-  }
-  if (overlaps(logits, rows * V * 4, hidden, rows * H * 2) ||
-      overlaps(logits, rows * V * 4, W, V * H * 2) ||
-      (bias != nullptr && overlaps(logits, rows * V * 4, bias, V * 2))) {
-    return LMHEAD_ERR_ALIAS;
-  }
+}  // extern "C"
+
+namespace {
+
+// Everything after validation for the fp32 head: logits to `logits`, or, when lp is given,
+// log-probabilities of its targets (no logits written).
+struct LogprobArgs {
+  const int32_t* targets;
+  float* logprobs;
+  float* lse;
+  void* workspace;
+};
+
+int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W, int64_t V,
+                 float alpha, const void* bias, float* logits, const LogprobArgs* lp,
+                 lmhead_stream_t stream) {
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != LMHEAD_OK) return st;
@@ -394,6 +392,11 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
   p.H = H;
   p.V = V;
   p.out = logits;
+  p.logprob = lp != nullptr ? 1 : 0;
+  p.n_chunks = (int32_t)(4 * ((V + lmh::kBM - 1) / lmh::kBM));
+  p.partials = lp != nullptr ? reinterpret_cast<float2*>(lp->workspace) : nullptr;
+  p.targets = lp != nullptr ? lp->targets : nullptr;
+  p.target_z = lp != nullptr ? lp->logprobs : nullptr;
   p.bias = reinterpret_cast<const uint16_t*>(bias);
   p.alpha = alpha;
   p.fp16 = dtype == LMHEAD_DTYPE_F16 ? 1 : 0;
@@ -429,7 +432,78 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
                 : nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2>
                             : lmh::lmhead_bf16_f32_kernel<1>;
   kernel<<<grid, lmh::kHeadThreads, smem, (cudaStream_t)stream>>>(tmap_w, tmap_h, p);
+  if (lp != nullptr) {
+    const int64_t blocks = (rows + lmh::kCombineRows - 1) / lmh::kCombineRows;
+    lmh::lmhead_logprob_combine_kernel<<<(unsigned)blocks, 1024, 0, (cudaStream_t)stream>>>(
+        p.partials, p.n_chunks, rows, V, lp->targets, lp->logprobs, lp->lse);
+  }
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+}
+
+
+int check_f32_head_args(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                        int64_t V, const void* bias) {
+  if (dtype != LMHEAD_DTYPE_BF16 && dtype != LMHEAD_DTYPE_F16) return LMHEAD_ERR_SHAPE;
+  if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 8 != 0) return LMHEAD_ERR_ALIGN;
+  if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (hidden == nullptr || W == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || (bias != nullptr && !aligned(bias, 2)))
+    return LMHEAD_ERR_ALIGN;
+  return LMHEAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                      int64_t V, float alpha, const void* bias, float* logits,
+                      lmhead_stream_t stream) {
+  const int st = check_f32_head_args(hidden, dtype, rows, H, W, V, bias);
+  if (st != LMHEAD_OK || rows == 0) return st;
+  if (logits == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(logits, 4)) return LMHEAD_ERR_ALIGN;
+  if (overlaps(logits, rows * V * 4, hidden, rows * H * 2) ||
+      overlaps(logits, rows * V * 4, W, V * H * 2) ||
+      (bias != nullptr && overlaps(logits, rows * V * 4, bias, V * 2))) {
+    return LMHEAD_ERR_ALIAS;
+  }
+  return run_f32_head(hidden, dtype, rows, H, W, V, alpha, bias, logits, nullptr, stream);
+}
+
+size_t lmhead_logprobs_workspace_bytes(int64_t rows, int64_t V) {
+  if (rows <= 0 || V <= 0) return 0;
+  return (size_t)rows * (size_t)(4 * ((V + lmh::kBM - 1) / lmh::kBM)) * 8u;
+}
+
+int lmhead_logprobs_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                        int64_t V, float alpha, const void* bias, const int32_t* targets,
+                        float* logprobs, float* lse, void* workspace, size_t workspace_bytes,
+                        lmhead_stream_t stream) {
+  const int st = check_f32_head_args(hidden, dtype, rows, H, W, V, bias);
+  if (st != LMHEAD_OK || rows == 0) return st;
+  if (targets == nullptr || logprobs == nullptr || workspace == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(targets, 4) || !aligned(logprobs, 4) || (lse != nullptr && !aligned(lse, 4)) ||
+      !aligned(workspace, 8)) {
+    return LMHEAD_ERR_ALIGN;
+  }
+  if (workspace_bytes < lmhead_logprobs_workspace_bytes(rows, V)) return LMHEAD_ERR_SHAPE;
+  const struct { const void* p; int64_t bytes; } in[4] = {
+      {hidden, rows * H * 2}, {W, V * H * 2}, {bias, bias ? V * 2 : 0}, {targets, rows * 4}};
+  const struct { const void* p; int64_t bytes; } out[3] = {
+      {logprobs, rows * 4}, {lse, lse ? rows * 4 : 0}, {workspace, (int64_t)workspace_bytes}};
+  for (const auto& o : out) {
+    if (o.p == nullptr) continue;
+    for (const auto& i : in)
+      if (i.p != nullptr && overlaps(o.p, o.bytes, i.p, i.bytes)) return LMHEAD_ERR_ALIAS;
+    for (const auto& o2 : out)
+      if (&o2 != &o && o2.p != nullptr && overlaps(o.p, o.bytes, o2.p, o2.bytes))
+        return LMHEAD_ERR_ALIAS;
+  }
+  const LogprobArgs lp{targets, logprobs, lse, workspace};
+  return run_f32_head(hidden, dtype, rows, H, W, V, alpha, bias, nullptr, &lp, stream);
 }
 
 int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,

@@ -21,7 +21,10 @@
 //              one of two TMEM accumulators; tcgen05.commit frees the stage (empty[s]) and, after
 //              the last K step, hands the accumulator to the epilogue (tmem_full[a]).
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, the bias (one IEEE fp32 add) if any, one
-//              IEEE fp32 multiply by alpha, store.
+//              IEEE fp32 multiply by alpha, store. In log-prob mode the logits are not stored:
+//              each warp reduces its 32 vocab entries to (max, sum of exp(z - max)) per row
+//              and writes that pair to the workspace, and the lane holding a row's target token
+//              writes that logit; a combine kernel (lmhead_logprob_combine_kernel) finishes.
 // Tile ownership: see TileSched.
 #pragma once
 
@@ -42,8 +45,62 @@ struct Bf16HeadParams {
   int32_t stages;
   uint32_t tmem_cols;
   uint32_t stage_bytes;
+  // log-prob mode (logprob != 0): no logits are written; see the epilogue
+  int32_t logprob;
+  int32_t n_chunks;         // 32-entry vocab chunks per row: 4 * ceil(V / 128)
+  float2* partials;         // [n_chunks, rows] (max, sum of exp(z - max)) per chunk and row
+  const int32_t* targets;   // [rows] token ids
+  float* target_z;          // [rows] the target's logit (written by the chunk that holds it)
   WaitCfg wait;
 };
+
+// (m, s) pairs standing for the partial sums s * exp(m): the pair of their union, with no branch
+// (lanes of a warp take different sides). Symmetric in its two arguments bit for bit; a pair
+// with s = 0 (no entries) contributes nothing.
+__device__ __forceinline__ void merge_max_sum(float m1, float s1, float m2, float s2, float& m,
+                                              float& s) {
+  const bool first = m1 >= m2;
+  const float big = first ? s1 : s2;
+  const float small = first ? s2 : s1;
+  m = first ? m1 : m2;
+  const float e = __expf(__fsub_rn(first ? m2 : m1, m));
+  s = small > 0.0f ? __fadd_rn(big, __fmul_rn(small, e)) : big;
+}
+
+// Log-sum-exp of each row from its chunk pairs, then logprob = z[target] - lse. A block of 32
+// warps serves 32 rows: lane i is row i; warp w folds chunk segment w in order (coalesced reads
+// of the chunk-major pairs), then warp 0 folds the 32 segment pairs of its row in order. The
+// result depends only on the row's logits and V.
+constexpr int kCombineRows = 32;
+__global__ void __launch_bounds__(1024)
+    lmhead_logprob_combine_kernel(const float2* __restrict__ partials, int32_t n_chunks,
+                                  int64_t rows, int64_t V, const int32_t* __restrict__ targets,
+                                  float* logprobs, float* lse_out) {
+  __shared__ float2 seg[32][kCombineRows + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * kCombineRows + lane;
+  const int per_seg = (n_chunks + 31) / 32;
+  const int c0 = warp * per_seg;
+  const int c1 = min(n_chunks, c0 + per_seg);
+  float m = -INFINITY, s = 0.0f;
+  if (row < rows) {
+    for (int c = c0; c < c1; ++c) {
+      const float2 q = partials[(int64_t)c * rows + row];
+      merge_max_sum(m, s, q.x, q.y, m, s);
+    }
+  }
+  seg[warp][lane] = make_float2(m, s);
+  __syncthreads();
+  if (warp == 0 && row < rows) {
+    m = -INFINITY;
+    s = 0.0f;
+    for (int w = 0; w < 32; ++w) merge_max_sum(m, s, seg[w][lane].x, seg[w][lane].y, m, s);
+    const float l = __fadd_rn(m, logf(s));
+    if (lse_out != nullptr) lse_out[row] = l;
+    const int32_t t = targets[row];
+    logprobs[row] = (t >= 0 && t < V) ? __fsub_rn(logprobs[row], l) : __int_as_float(0x7fc00000);
+  }
+}
 
 template <int NSUB>
 __global__ void __launch_bounds__(kHeadThreads, 1)
@@ -229,6 +286,70 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c, r);
         tmem_ld_wait();
+        if (p.logprob) {
+          // This warp's 32 vocab entries of rows r0 + c + j: the same fp32 logits the store
+          // path writes, reduced per row to (max, sum of exp(z - max)) in two butterfly phases
+          // over the lanes, so lanes 2i and 2i + 1 both hold row i's pair.
+          const int32_t chunk = (int32_t)(tc.v0 / kBM) * 4 + quarter;
+          const int64_t rl = r0 + c + lane;
+          const int32_t tgt = (lane < 16 && rl < p.rows) ? p.targets[rl] : -1;
+          // Which of these 16 rows has its target among this warp's 32 entries (usually none).
+          const int64_t wv0 = tc.v0 + quarter * 32;
+          const uint32_t hits = __ballot_sync(0xffffffffu, tgt >= wv0 && tgt < wv0 + 32);
+          float zz[16], pm[16], ps[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a = __uint_as_float(r[j]);
+            const float z = !v_ok ? -INFINITY
+                            : p.bias == nullptr ? __fmul_rn(p.alpha, a)
+                                                : __fmul_rn(p.alpha, __fadd_rn(a, b));
+            if (hits & (1u << j)) {  // warp-uniform
+              const int32_t tj = __shfl_sync(0xffffffffu, tgt, j);
+              if (v_ok && v == (int64_t)tj) p.target_z[r0 + c + j] = z;
+            }
+            zz[j] = z;
+            pm[j] = z;
+          }
+          // Phase 1, the maxima: butterfly over the lanes, each step keeping half the rows; lanes
+          // 2i and 2i + 1 end with row i's max, which every lane then fetches.
+#pragma unroll
+          for (int w = 8, off = 16; w >= 1; w >>= 1, off >>= 1) {
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int j = 0; j < w; ++j) {
+              const float keep = upper ? pm[j + w] : pm[j];
+              const float send = upper ? pm[j] : pm[j + w];
+              pm[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+            }
+          }
+          pm[0] = fmaxf(pm[0], __shfl_xor_sync(0xffffffffu, pm[0], 1));
+          // Phase 2, the sums of exp(z - max), the same butterfly with adds.
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float mj = __shfl_sync(0xffffffffu, pm[0], 2 * j);
+            ps[j] = v_ok ? __expf(__fsub_rn(zz[j], mj)) : 0.0f;
+          }
+#pragma unroll
+          for (int w = 8, off = 16; w >= 1; w >>= 1, off >>= 1) {
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int j = 0; j < w; ++j) {
+              const float keep = upper ? ps[j + w] : ps[j];
+              const float send = upper ? ps[j] : ps[j + w];
+              const float got = __shfl_xor_sync(0xffffffffu, send, off);
+              // the lower lane's half first, so partners add in the same order
+              ps[j] = upper ? __fadd_rn(got, keep) : __fadd_rn(keep, got);
+            }
+          }
+          {
+            const float got = __shfl_xor_sync(0xffffffffu, ps[0], 1);
+            ps[0] = (lane & 1) ? __fadd_rn(got, ps[0]) : __fadd_rn(ps[0], got);
+          }
+          const int64_t row = r0 + c + ((lane >> 1) & 15);
+          if ((lane & 1) == 0 && row < p.rows)
+            p.partials[(int64_t)chunk * p.rows + row] = make_float2(pm[0], ps[0]);
+          continue;
+        }
         if (v_ok) {
           float* dst = p.out + (r0 + c) * p.V + v;
           if (p.bias == nullptr) {

@@ -41,6 +41,8 @@ WORKLOADS = {
     "spec_verify": ([128, 97, 32], 4096, 128256, 0.015, 1.0 / 16),
     "prefill": ([8192], 4096, 151936, 0.02, 1.0 / 8),
     "nvfp4": ([1, 16, 64, 65, 256], 2048, 151936, 0.02, 1.0 / 8),
+    # the prefill shape computing log-probabilities of one target token per row (no logits out)
+    "prefill_logprobs": ([8192], 4096, 151936, 0.02, 1.0 / 8),
     # the NVFP4 quantiser on the NVFP4 head's weight shape (rows = the V rows quantised per call)
     "nvfp4_quantize": ([151936], 2048, 151936, 0.02, 1.0),
     # the decode shape with fp16 operands and an fp16 embedding bias

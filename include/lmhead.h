@@ -102,6 +102,36 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
                       lmhead_stream_t stream);
 
 /*
+ * Log-probabilities of given tokens, without writing logits. With z[r, v] the fp32 logits that
+ * lmhead_logits_f32 would write for the same arguments (same bits),
+ *   lse[r]       = log sum_v exp(z[r, v])
+ *   logprobs[r]  = z[r, targets[r]] - lse[r]      (NaN when targets[r] is outside [0, V))
+ * The first page ("Purpose") wants fp32 logits for RL training-inference consistency and for
+ * speculative decoding, whose rejection sampling consumes exactly these; at prefill sizes this
+ * avoids writing rows * V * 4 bytes of logits (5 GB at 8192 x 151936).
+ * The head's epilogue reduces every 32-entry vocab chunk of a row to (max, sum of exp(z - max))
+ * in fp32 and stores that pair in `workspace` (chunk-major); a second kernel folds a row's pairs
+ * in a fixed order. So a row's results do not depend on the row count, and they are
+ * reproducible.
+ * Accuracy: lse and logprobs are fp32 sums of expf terms; against the exact values over the same
+ * fp32 logits they are good to a few units in 1e-6 relative.
+ *
+ *   hidden, W, bias, dtype, alpha: as lmhead_logits_f32
+ *   targets    int32 [rows], 4-byte aligned
+ *   logprobs   fp32 [rows], 4-byte aligned (output)
+ *   lse        fp32 [rows], 4-byte aligned (output), or NULL
+ *   workspace  at least lmhead_logprobs_workspace_bytes(rows, V) bytes, 8-byte aligned, owned by
+ *              the caller (rows * 4 * ceil(V / 128) * 8 bytes)
+ * Outputs and workspace must not overlap each other or the inputs. Two kernels are enqueued.
+ * Returns an lmhead_status (LMHEAD_ERR_SHAPE also when the workspace is too small).
+ */
+size_t lmhead_logprobs_workspace_bytes(int64_t rows, int64_t V);
+int lmhead_logprobs_f32(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W,
+                        int64_t V, float alpha, const void* bias, const int32_t* targets,
+                        float* logprobs, float* lse, void* workspace, size_t workspace_bytes,
+                        lmhead_stream_t stream);
+
+/*
  * Entry 2: bf16 logits from the W4A16 NVFP4 head.
  *   W[v, k]      = e2m1(code[v, k]) * e4m3(w_scales[v, k / 16])      (exact in bf16)
  *   logits[r, v] = bf16_rn( fl32( fl32(acc[r, v] * w_global_scale) * alpha ) ),

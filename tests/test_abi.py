@@ -116,6 +116,24 @@ def test_quantiser_argument_errors(lib):
     assert f(A16, 4, 64, B16, C16, B16 + 8, WS, need, 0) == 7           # g inside packed
 
 
+def test_logprobs_argument_errors(lib):
+    f = lm.lmhead_logprobs_f32
+    T, LP, LSE, WS = 0x60000000, 0x61000000, 0x62000000, 0x63000000
+    need = lm.logprobs_workspace_bytes(4, 300)
+    assert need == 4 * 4 * 3 * 8                       # rows x 4 chunks per 128 vocab x 8 bytes
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, LP, LSE, WS, need, 0) != 2   # valid shape passes
+    assert f(A16, 5, 4, 64, B16, 300, 1.0, 0, T, LP, LSE, WS, need, 0) == 2   # bad dtype
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, 0, LP, LSE, WS, need, 0) == 1   # no targets
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, 0, LSE, WS, need, 0) == 1    # no logprobs
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, LP, LSE, 0, need, 0) == 1    # no workspace
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, LP, LSE, WS, need - 8, 0) == 2  # too small
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T + 2, LP, LSE, WS, need, 0) == 3
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, LP, LSE, WS + 4, need, 0) == 3
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, LP, LP + 8, WS, need, 0) == 7  # lse over logprobs
+    assert f(A16, 0, 4, 64, B16, 300, 1.0, 0, T, B16 + 16, LSE, WS, need, 0) == 7  # over W
+    assert f(A16, 0, 0, 64, B16, 300, 1.0, 0, 0, 0, 0, 0, 0, 0) == 0            # rows == 0
+
+
 def test_rows_zero_launches_nothing(lib):
     # rows == 0 is a no-op even with NULL pointers (no CUDA call is made)
     assert lm.lmhead_logits_bf16_f32(0, 0, 64, 0, 128, 1.0, 0, 0) == 0
