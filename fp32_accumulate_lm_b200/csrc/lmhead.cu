@@ -313,13 +313,13 @@ int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed
   if (st != LMHEAD_OK) return st;
   // Pass 1 grid: a few CTAs per SM, one partial word each, never past the workspace.
   const int64_t n_chunks = n / 8;
-  int64_t grid = (int64_t)dev.num_sms * 4;
+  int64_t grid = (int64_t)dev.num_sms * 6;
   const int64_t by_work = (n_chunks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
   if (grid > by_work) grid = by_work;
   if (grid > lmh::kQuantMaxPartials) grid = lmh::kQuantMaxPartials;
   if (workspace_bytes < (size_t)grid * sizeof(uint32_t)) return LMHEAD_ERR_SHAPE;
   const int64_t n_blocks = n / 16;
-  int64_t grid2 = (int64_t)dev.num_sms * 4;
+  int64_t grid2 = (int64_t)dev.num_sms * 8;
   const int64_t by_blocks = (n_blocks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
   if (grid2 > by_blocks) grid2 = by_blocks;
   uint32_t* partial = reinterpret_cast<uint32_t*>(workspace);

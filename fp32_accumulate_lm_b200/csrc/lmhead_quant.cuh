@@ -48,8 +48,16 @@ __global__ void __launch_bounds__(kQuantThreads)
   __shared__ uint32_t red[32];
   uint32_t m = 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_chunks; i += stride)
-    m = max(m, chunk_absmax_bits(__ldcs(w + i)));
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // Four independent 16-byte loads in flight per thread: enough bytes in flight per SM to cover
+  // the DRAM latency at the HBM rate.
+  for (; i + 3 * stride < n_chunks; i += 4 * stride) {
+    const uint4 a = __ldcs(w + i), b = __ldcs(w + i + stride), c = __ldcs(w + i + 2 * stride),
+                d = __ldcs(w + i + 3 * stride);
+    m = max(max(m, chunk_absmax_bits(a)), max(chunk_absmax_bits(b),
+                                              max(chunk_absmax_bits(c), chunk_absmax_bits(d))));
+  }
+  for (; i < n_chunks; i += stride) m = max(m, chunk_absmax_bits(__ldcs(w + i)));
   m = block_max_u32(m, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = m;
 }
@@ -80,6 +88,26 @@ __device__ __forceinline__ uint32_t rn_e2m1_code(float x) {
   return (c & 7u) ? c : 0u;
 }
 
+// One 16-element block: 32 bytes of W (c0, c1) to 8 bytes of codes and one scale byte.
+__device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, float g,
+                                             float six_g, uint2* packed, uint8_t* scale) {
+  const float bmax = __uint_as_float(max(chunk_absmax_bits(c0), chunk_absmax_bits(c1)) << 16);
+  const uint32_t s = rn_e4m3_code(__fdiv_rn(bmax, six_g));
+  const float d = __fmul_rn(e4m3_value(s), g);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
+    const float w0 = __uint_as_float(words[i] << 16);
+    const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
+    const uint32_t q0 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w0, d)) : 0u;
+    const uint32_t q1 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w1, d)) : 0u;
+    out[i >> 2] |= (q0 | (q1 << 4)) << (8 * (i & 3));
+  }
+  *packed = make_uint2(out[0], out[1]);
+  *scale = (uint8_t)s;
+}
+
 // Pass 2: every CTA reduces the partials to amax (the same value everywhere), then each thread
 // encodes 16-element blocks: 32 bytes of W in, 8 bytes of codes and one scale byte out.
 __global__ void __launch_bounds__(kQuantThreads)
@@ -95,25 +123,18 @@ __global__ void __launch_bounds__(kQuantThreads)
   const float six_g = __fmul_rn(6.0f, g);
   if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks; b += stride) {
+  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // Two blocks per iteration, their four loads issued together.
+  for (; b + stride < n_blocks; b += 2 * stride) {
+    const uint4 a0 = __ldcs(w + 2 * b), a1 = __ldcs(w + 2 * b + 1);
+    const uint4 b0 = __ldcs(w + 2 * (b + stride)), b1 = __ldcs(w + 2 * (b + stride) + 1);
+    encode_block(a0, a1, g, six_g, packed + b, scales + b);
+    encode_block(b0, b1, g, six_g, packed + b + stride, scales + b + stride);
+  }
+  for (; b < n_blocks; b += stride) {
     const uint4 c0 = __ldcs(w + 2 * b);
     const uint4 c1 = __ldcs(w + 2 * b + 1);
-    const float bmax =
-        __uint_as_float(max(chunk_absmax_bits(c0), chunk_absmax_bits(c1)) << 16);
-    const uint32_t s = rn_e4m3_code(__fdiv_rn(bmax, six_g));
-    const float d = __fmul_rn(e4m3_value(s), g);
-    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    uint32_t out[2] = {0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
-      const float w0 = __uint_as_float(words[i] << 16);
-      const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
-      const uint32_t q0 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w0, d)) : 0u;
-      const uint32_t q1 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w1, d)) : 0u;
-      out[i >> 2] |= (q0 | (q1 << 4)) << (8 * (i & 3));
-    }
-    packed[b] = make_uint2(out[0], out[1]);
-    scales[b] = (uint8_t)s;
+    encode_block(c0, c1, g, six_g, packed + b, scales + b);
   }
 }
 
