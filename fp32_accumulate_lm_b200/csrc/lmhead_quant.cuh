@@ -78,14 +78,18 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-// Nearest E2M1 code of x (saturating at +-6), with no negative zero.
-__device__ __forceinline__ uint32_t rn_e2m1_code(float x) {
+// Nearest E2M1 codes of two values (saturating at +-6) as one byte: lo in the low nibble, hi in
+// the high one (the conversion puts its first operand in the upper half), with no negative
+// zero.
+__device__ __forceinline__ uint32_t rn_e2m1_pair(float lo, float hi) {
   uint16_t two;
-  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %1;\n\tcvt.u16.u8 %0, q;\n\t}"
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u16.u8 %0, q;\n\t}"
       : "=h"(two)
-      : "f"(x));
-  const uint32_t c = two & 0x0Fu;
-  return (c & 7u) ? c : 0u;
+      : "f"(hi), "f"(lo));
+  uint32_t b = two & 0xFFu;
+  if ((b & 0x07u) == 0u) b &= ~0x08u;
+  if ((b & 0x70u) == 0u) b &= ~0x80u;
+  return b;
 }
 
 // One 16-element block: 32 bytes of W (c0, c1) to 8 bytes of codes and one scale byte.
@@ -100,9 +104,8 @@ __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, f
   for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
     const float w0 = __uint_as_float(words[i] << 16);
     const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
-    const uint32_t q0 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w0, d)) : 0u;
-    const uint32_t q1 = d > 0.0f ? rn_e2m1_code(__fdiv_rn(w1, d)) : 0u;
-    out[i >> 2] |= (q0 | (q1 << 4)) << (8 * (i & 3));
+    const uint32_t q = d > 0.0f ? rn_e2m1_pair(__fdiv_rn(w0, d), __fdiv_rn(w1, d)) : 0u;
+    out[i >> 2] |= q << (8 * (i & 3));
   }
   *packed = make_uint2(out[0], out[1]);
   *scale = (uint8_t)s;
