@@ -206,13 +206,19 @@ uint32_t tmem_cols_for(int32_t bn) {
 constexpr int kInt32Max = 0x7fffffff;
 
 // Tile ownership (see TileSched) and grid size: one persistent CTA per SM at most.
-int make_sched(int64_t rows, int64_t V, int32_t bn, int num_sms, lmh::TileSched* s, int* grid) {
+int make_sched(int64_t rows, int64_t V, int64_t H, int32_t bn, int num_sms, lmh::TileSched* s,
+               int* grid) {
   s->bn = bn;
   s->n_rtiles = (int32_t)((rows + bn - 1) / bn);
   const int64_t n_vtiles = (V + lmh::kBM - 1) / lmh::kBM;
   const int64_t tiles = (int64_t)s->n_rtiles * n_vtiles;
   if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
   s->num_tiles = (int32_t)tiles;
+  s->n_vtiles = (int32_t)n_vtiles;
+  // Row tiles per group: their hidden rows within 16 MB (an eighth of L2).
+  const int64_t tile_hidden_bytes = (int64_t)bn * H * 2;
+  const int64_t rg = (16ll << 20) / (tile_hidden_bytes > 0 ? tile_hidden_bytes : 1);
+  s->rgroup = (int32_t)(rg < 1 ? 1 : (rg > s->n_rtiles ? s->n_rtiles : rg));
   *grid = s->num_tiles < num_sms ? s->num_tiles : num_sms;
   return LMHEAD_OK;
 }
@@ -402,7 +408,7 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   p.fp16 = dtype == LMHEAD_DTYPE_F16 ? 1 : 0;
   p.bn = pick_bn(rows);
   int grid = 0;
-  st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
+  st = make_sched(rows, V, H, p.bn, dev.num_sms, &p.sched, &grid);
   if (st != LMHEAD_OK) return st;
   const int reserve = 1024 + 512;  // alignment slack + barriers
   const int nsub = pick_nsub(p.bn, dev.smem_optin - reserve);
@@ -539,7 +545,7 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.gscale = w_global_scale;
   p.bn = pick_bn(rows) < lmh::kBnMax ? pick_bn(rows) : lmh::kBnMax;
   int grid = 0;
-  st = make_sched(rows, V, p.bn, dev.num_sms, &p.sched, &grid);
+  st = make_sched(rows, V, H, p.bn, dev.num_sms, &p.sched, &grid);
   if (st != LMHEAD_OK) return st;
   p.num_kb = (int32_t)(H / lmh::kBK);
   // Hidden sub-tiles start on 1024-byte swizzle atoms: rows per K step rounded up to 8.

@@ -88,16 +88,23 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-// Which output tiles a CTA owns. Tile t = (v-tile, row-tile) = (t / n_rtiles, t % n_rtiles):
-// 128 vocab rows by bn hidden rows; CTA i of G takes t = i, i + G, i + 2G, ... At any moment the
-// G CTAs work on neighbouring v-tiles, which keeps the weight stream on few DRAM pages and, with
-// many row tiles, lets CTAs share each weight tile through L2. (Balanced per-CTA strips of W and
-// splitting the last partial wave into 16-row pieces were both measured slower on B200.)
-// Every tile runs the same MMA chain over K, so the schedule changes no output bit.
+// Which output tiles a CTA owns. A tile is 128 vocab rows by bn hidden rows. Row tiles come in
+// groups of `rgroup` (whose hidden rows fit comfortably in L2); tiles run group by group, and
+// within a group v-major: t -> (v-tile, row-tile) = (local / rg, group * rgroup + local % rg),
+// rg = the group's row tiles. CTA i of G takes t = i, i + G, i + 2G, ... At any moment the G CTAs
+// work on neighbouring v-tiles of one group: the weight stream stays on few DRAM pages, CTAs
+// share each weight tile through L2, and the group's hidden rows stay in L2 instead of being
+// re-read for every v-tile (at 8192 x 4096 hidden rows, 64 MB, they did not survive the weight
+// and logits streams). With rgroup >= the row tiles there is one group: plain v-major order.
+// (Balanced per-CTA strips of W and splitting the last partial wave into 16-row pieces were both
+// measured slower on B200.) Every tile runs the same MMA chain over K, so the schedule changes no
+// output bit.
 struct TileSched {
   int32_t n_rtiles;
   int32_t num_tiles;
   int32_t bn;
+  int32_t n_vtiles;
+  int32_t rgroup;
 };
 
 struct TileCoord {
@@ -115,8 +122,13 @@ __device__ __forceinline__ int sched_count(const TileSched& s) {
 __device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, int i) {
   TileCoord c;
   const int t = (int)blockIdx.x + i * (int)gridDim.x;
-  const int vt = t / s.n_rtiles;
-  const int rt = t - vt * s.n_rtiles;
+  const int per_group = s.n_vtiles * s.rgroup;
+  const int g = t / per_group;
+  const int local = t - g * per_group;
+  const int left_rt = s.n_rtiles - g * s.rgroup;
+  const int rg = left_rt < s.rgroup ? left_rt : s.rgroup;
+  const int vt = local / rg;
+  const int rt = g * s.rgroup + (local - vt * rg);
   c.v0 = (int64_t)vt * kBM;
   const int64_t left = V - c.v0;
   c.vrows = (int32_t)(left < kBM ? left : kBM);
