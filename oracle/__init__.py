@@ -83,6 +83,13 @@ def _load():
                                             ctypes.POINTER(ctypes.c_int32), f32p, f32p,
                                             ctypes.c_int]
         lib.oracle_logprobs_f32.restype = ctypes.c_int
+        lib.oracle_logprob_shard_stats.argtypes = [u16p, ctypes.c_int, i64, i64, u16p, i64, i64,
+                                                   ctypes.c_float, ctypes.c_void_p,
+                                                   ctypes.POINTER(ctypes.c_int32), f64p,
+                                                   ctypes.c_int]
+        lib.oracle_logprob_shard_stats.restype = ctypes.c_int
+        lib.oracle_logprob_merge_shards.argtypes = [f64p, i64, i64, f32p, f32p]
+        lib.oracle_logprob_merge_shards.restype = ctypes.c_int
         lib.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, u8p, u8p, f32p]
         lib.oracle_nvfp4_quantize.restype = ctypes.c_int
         lib.oracle_rn_e4m3.argtypes = [ctypes.c_float]
@@ -265,4 +272,45 @@ def logprobs_f32(hidden_bits: np.ndarray, w_bits: np.ndarray, alpha: float, targ
                                      _ptr(lse, ctypes.c_float), threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"oracle_logprobs_f32 failed with {rc}")
+    return lp, lse
+
+
+def logprob_shard_stats(hidden_bits: np.ndarray, w_shard_bits: np.ndarray, v_begin: int,
+                        alpha: float, targets: np.ndarray, bias_bits=None, dtype: str = "bf16",
+                        threads: int | None = None) -> np.ndarray:
+    """float64 [rows, 3]: (max, sum of exp(z - max), target logit or NaN) over the fp32 logits of
+    the vocab slice W[v_begin : v_begin + V_shard] (targets are global ids)."""
+    h = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_shard_bits, dtype=np.uint16)
+    t = np.ascontiguousarray(targets, dtype=np.int32)
+    rows, H = h.shape
+    if w.shape[1] != H or t.shape != (rows,):
+        raise ValueError("shape mismatch")
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    stats = np.zeros((rows, 3), dtype=np.float64)
+    if rows == 0:
+        return stats
+    rc = _load().oracle_logprob_shard_stats(
+        _ptr(h, ctypes.c_uint16), 1 if dtype == "f16" else 0, rows, H, _ptr(w, ctypes.c_uint16),
+        w.shape[0], int(v_begin), ctypes.c_float(alpha), None if b is None else b.ctypes.data,
+        _ptr(t, ctypes.c_int32), _ptr(stats, ctypes.c_double), threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle_logprob_shard_stats failed with {rc}")
+    return stats
+
+
+def logprob_merge_shards(stats: np.ndarray):
+    """(logprobs [rows], lse [rows]) float32 from float64 shard stats [shards, rows, 3]."""
+    st = np.ascontiguousarray(stats, dtype=np.float64)
+    if st.ndim != 3 or st.shape[2] != 3:
+        raise ValueError(f"stats shape {st.shape}")
+    rows = st.shape[1]
+    lp = np.zeros(rows, dtype=np.float32)
+    lse = np.zeros(rows, dtype=np.float32)
+    if rows == 0:
+        return lp, lse
+    rc = _load().oracle_logprob_merge_shards(_ptr(st, ctypes.c_double), st.shape[0], rows,
+                                             _ptr(lp, ctypes.c_float), _ptr(lse, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle_logprob_merge_shards failed with {rc}")
     return lp, lse

@@ -232,6 +232,65 @@ int oracle_logprobs_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t
   return 0;
 }
 
+/* Vocab-parallel split. "FP32 LM head skip FP32 cast" (key source excerpt, _compute_lm_head)
+ * takes the head as a VocabParallelEmbedding, whose rows of W are spread over GPUs; the
+ * log-softmax above then needs a max and a sum over every slice. The definition is unchanged:
+ * the union of the slices' terms, merged here in double. */
+int oracle_logprob_shard_stats(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                               const uint16_t* W_shard, int64_t V_shard, int64_t v_begin,
+                               float alpha, const uint16_t* bias_shard, const int32_t* targets,
+                               double* stats, int threads) {
+  if (rows < 0 || H <= 0 || V_shard <= 0 || v_begin < 0) return 1;
+  if (rows == 0) return 0;
+  if (!targets || !stats) return 1;
+  float* z = (float*)malloc((size_t)rows * (size_t)V_shard * sizeof(float));
+  if (!z) return 2;
+  int rc = oracle_logits_f32(hidden, dtype, rows, H, W_shard, V_shard, alpha, bias_shard, z, NULL,
+                             threads);
+  if (rc != 0) {
+    free(z);
+    return rc;
+  }
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* zr = z + r * V_shard;
+    double m = -INFINITY;
+    for (int64_t v = 0; v < V_shard; ++v)
+      if ((double)zr[v] > m) m = (double)zr[v];
+    double sum = 0.0;
+    for (int64_t v = 0; v < V_shard; ++v) sum += exp((double)zr[v] - m);
+    const int64_t t = (int64_t)targets[r] - v_begin;
+    stats[3 * r] = m;
+    stats[3 * r + 1] = sum;
+    stats[3 * r + 2] = (t >= 0 && t < V_shard) ? (double)zr[t] : NAN;
+  }
+  free(z);
+  return 0;
+}
+
+int oracle_logprob_merge_shards(const double* stats, int64_t shards, int64_t rows,
+                                float* logprobs, float* lse) {
+  if (shards <= 0 || rows < 0) return 1;
+  if (rows == 0) return 0;
+  if (!stats || !logprobs) return 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    double big = -INFINITY;
+    for (int64_t g = 0; g < shards; ++g) {
+      const double m = stats[3 * (g * rows + r)];
+      if (m > big) big = m;
+    }
+    double sum = 0.0, zt = NAN;
+    for (int64_t g = 0; g < shards; ++g) {
+      const double* q = stats + 3 * (g * rows + r);
+      sum += q[1] * exp(q[0] - big);
+      if (isnan(zt) && !isnan(q[2])) zt = q[2];
+    }
+    const double l = big + log(sum);
+    if (lse) lse[r] = oracle_round_f32(l);
+    logprobs[r] = isnan(zt) ? (float)NAN : oracle_round_f32(zt - l);
+  }
+  return 0;
+}
+
 /* ---------------------------------------------------------------- the NVFP4 quantiser */
 
 /* Nearest entry of an ascending table of exact values (ties to the even index); x >= 0 finite

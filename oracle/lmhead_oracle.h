@@ -64,6 +64,22 @@ int oracle_logprobs_f32(const uint16_t* hidden, int dtype, int64_t rows, int64_t
                         const int32_t* targets, float* logprobs, float* lse, int threads);
 
 /*
+ * Vocab-parallel log-probabilities, the same quantities split over slices of W's rows. For the
+ * slice W_shard = W[v_begin, v_begin + V_shard), with z its fp32 logits (oracle_logits_f32):
+ *   stats[3r] = max_v z[r, v],  stats[3r+1] = sum_v exp(z[r, v] - stats[3r])  (double),
+ *   stats[3r+2] = z[r, targets[r]] when the slice holds the target (global id), else NaN.
+ * oracle_logprob_merge_shards takes [shards][rows][3] such stats and returns, rounded once,
+ *   lse[r] = M + log(sum_g s_g exp(m_g - M)),  M = max_g m_g,   logprobs[r] = z_t - lse[r]
+ * with z_t from the shard that holds the target (NaN when none does). lse may be NULL.
+ */
+int oracle_logprob_shard_stats(const uint16_t* hidden, int dtype, int64_t rows, int64_t H,
+                               const uint16_t* W_shard, int64_t V_shard, int64_t v_begin,
+                               float alpha, const uint16_t* bias_shard, const int32_t* targets,
+                               double* stats, int threads);
+int oracle_logprob_merge_shards(const double* stats, int64_t shards, int64_t rows,
+                                float* logprobs, float* lse);
+
+/*
  * NVFP4 quantiser (this library's reading; every decision step one IEEE binary32 operation):
  * amax = max|w|, g = amax / 2688 (1 when amax = 0); per 16-element block s = RN_e4m3(bmax / (6g))
  * saturating; per element q = RN_e2m1(w / (e4m3(s) * g)) saturating, sign only on non-zero

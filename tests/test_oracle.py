@@ -626,3 +626,61 @@ def test_logprobs_out_of_range_target_is_nan():
     w = bf16_bits_of_f32(np.ones((10, 16)))
     lp, _ = oracle.logprobs_f32(h, w, 1.0, np.array([-1, 10], np.int32))
     assert np.isnan(lp).all()
+
+
+# ---------------------------------------------------------------- vocab-parallel log-probabilities
+# "FP32 LM head skip FP32 cast" (key source excerpt, _compute_lm_head) takes the head as a
+# VocabParallelEmbedding: W's rows split over GPUs. The log-softmax is still over the whole row;
+# a slice contributes (max, sum of exp(z - max), target logit if held).
+
+def _split(V, g):
+    base, extra = divmod(V, g)
+    starts = [r * base + min(r, extra) for r in range(g)]
+    return [(b, base + (1 if r < extra else 0)) for r, b in enumerate(starts)]
+
+
+def test_shard_merge_matches_scipy_logsumexp_of_the_whole_row():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(103)
+    rows, H, V = 5, 96, 2003
+    h = bf16_bits_of_f32(rng.normal(0, 1, (rows, H)))
+    w = bf16_bits_of_f32(rng.normal(0, 0.3, (V, H)))
+    t = np.array([0, 667, 668, 2002, 1001], np.int32)
+    z, _ = oracle.logits_f32(h, w, 0.25)
+    want_lse = logsumexp(z.astype(np.float64), axis=1)
+    for g in (1, 2, 3, 7):
+        stats = np.stack([oracle.logprob_shard_stats(h, w[b:b + n], b, 0.25, t)
+                          for b, n in _split(V, g)])
+        lp, lse = oracle.logprob_merge_shards(stats)
+        assert np.allclose(lse, want_lse, rtol=2e-7, atol=0), g
+        assert np.allclose(lp, z[np.arange(rows), t] - want_lse, rtol=0, atol=1e-6), g
+
+
+def test_shard_stats_are_max_sum_and_held_target():
+    rng = np.random.default_rng(104)
+    rows, H, V, b0, n = 4, 64, 300, 100, 120
+    h = bf16_bits_of_f32(rng.normal(0, 1, (rows, H)))
+    w = bf16_bits_of_f32(rng.normal(0, 0.3, (V, H)))
+    t = np.array([99, 100, 219, 220], np.int32)      # just outside, first, last, just outside
+    z, _ = oracle.logits_f32(h, w[b0:b0 + n], 2.0)
+    st = oracle.logprob_shard_stats(h, w[b0:b0 + n], b0, 2.0, t)
+    zmax = z.astype(np.float64).max(axis=1)
+    assert np.array_equal(st[:, 0], zmax)
+    assert np.allclose(st[:, 1], np.exp(z.astype(np.float64) - zmax[:, None]).sum(axis=1),
+                       rtol=1e-15, atol=0)
+    assert np.isnan(st[0, 2]) and np.isnan(st[3, 2])
+    assert st[1, 2] == z[1, 0] and st[2, 2] == z[2, n - 1]
+
+
+def test_shard_merge_uniform_logits_and_missing_target():
+    """W = 0: every logit is 0, so lse = log V whatever the split; a target no shard holds is
+    NaN."""
+    rows, H, V = 2, 16, 1000
+    h = bf16_bits_of_f32(np.random.default_rng(105).normal(0, 1, (rows, H)))
+    w = np.zeros((V, H), np.uint16)
+    t = np.array([999, 1000], np.int32)
+    stats = np.stack([oracle.logprob_shard_stats(h, w[b:b + n], b, 1.0, t)
+                      for b, n in _split(V, 3)])
+    lp, lse = oracle.logprob_merge_shards(stats)
+    assert np.allclose(lse, np.float32(math.log(V)), rtol=0, atol=1e-6)
+    assert abs(lp[0] + math.log(V)) < 1e-6 and np.isnan(lp[1])
