@@ -78,36 +78,74 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-// Nearest E2M1 codes of two values (saturating at +-6) as one byte: lo in the low nibble, hi in
-// the high one (the conversion puts its first operand in the upper half), with no negative
-// zero.
-__device__ __forceinline__ uint32_t rn_e2m1_pair(float lo, float hi) {
+// E2M1 codes of two values (saturating at +-6, round to nearest, ties to the even code) as one
+// byte: lo in the low nibble, hi in the high one (the conversion puts its first operand in the
+// upper half). A zero magnitude may carry a sign bit here; drop_negative_zeros clears it.
+__device__ __forceinline__ uint32_t e2m1_pair_code(float lo, float hi) {
   uint16_t two;
   asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u16.u8 %0, q;\n\t}"
       : "=h"(two)
       : "f"(hi), "f"(lo));
-  uint32_t b = two & 0xFFu;
-  if ((b & 0x07u) == 0u) b &= ~0x08u;
-  if ((b & 0x70u) == 0u) b &= ~0x80u;
-  return b;
+  return two & 0xFFu;
 }
 
+// Eight E2M1 codes in a word: clear the sign bit of every nibble whose magnitude is zero. Adding
+// 7 to a 3-bit magnitude carries into the nibble's bit 3 exactly when the magnitude is non-zero,
+// and never out of the nibble.
+__device__ __forceinline__ uint32_t drop_negative_zeros(uint32_t q) {
+  const uint32_t mag = q & 0x77777777u;
+  return mag | (q & ((mag + 0x77777777u) & 0x88888888u));
+}
+
+// Relative guard band of the quotient shortcut in encode_block.
+constexpr float kQuotientBand = 0x1p-16f;
+
 // One 16-element block: 32 bytes of W (c0, c1) to 8 bytes of codes and one scale byte.
+//
+// Each code is that of the correctly rounded quotient x = fl(w / d). Instead of dividing every
+// element, the block takes one correctly rounded reciprocal r = fl(1 / d) and converts the two
+// products w * fl(r (1 - b)) and w * fl(r (1 + b)), b = 2^-16. Their magnitudes bracket |x|
+// strictly: each is within 3 * 2^-24 relative of w / d times (1 -+ b), and x within 2^-24 of it
+// wherever a code boundary can lie (|x| >= 1/4, all normal numbers). The code is monotone in the
+// magnitude, so when both products give the same code, x has that code as well. Only a pair with
+// a quotient within about 2^-16 of a boundary (0.25, 0.75, ..., 5) is divided exactly. d outside
+// [2^-120, 2^120], where r could leave the normal range, is always divided exactly.
 __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, float g,
                                              float six_g, uint2* packed, uint8_t* scale) {
   const float bmax = __uint_as_float(max(chunk_absmax_bits(c0), chunk_absmax_bits(c1)) << 16);
   const uint32_t s = rn_e4m3_code(__fdiv_rn(bmax, six_g));
   const float d = __fmul_rn(e4m3_value(s), g);
+  const bool shortcut = d >= 0x1p-120f && d <= 0x1p120f;
+  const float r = __frcp_rn(d);
+  const float r_lo = __fmul_rn(r, 1.0f - kQuotientBand);
+  const float r_hi = __fmul_rn(r, 1.0f + kQuotientBand);
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  uint32_t out[2] = {0u, 0u};
+  uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
     const float w0 = __uint_as_float(words[i] << 16);
     const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
-    const uint32_t q = d > 0.0f ? rn_e2m1_pair(__fdiv_rn(w0, d), __fdiv_rn(w1, d)) : 0u;
-    out[i >> 2] |= q << (8 * (i & 3));
+    lo[i >> 2] |= e2m1_pair_code(__fmul_rn(w0, r_lo), __fmul_rn(w1, r_lo)) << (8 * (i & 3));
+    hi[i >> 2] |= e2m1_pair_code(__fmul_rn(w0, r_hi), __fmul_rn(w1, r_hi)) << (8 * (i & 3));
   }
-  *packed = make_uint2(out[0], out[1]);
+  if (!shortcut || lo[0] != hi[0] || lo[1] != hi[1]) {
+    // Some quotient of the block sits near a code boundary (or r is unusable): divide those
+    // pairs exactly.
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int sh = 8 * (i & 3);
+      const uint32_t a = (lo[i >> 2] >> sh) & 0xFFu;
+      if (shortcut && a == ((hi[i >> 2] >> sh) & 0xFFu)) continue;
+      const float w0 = __uint_as_float(words[i] << 16);
+      const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
+      const uint32_t q = e2m1_pair_code(__fdiv_rn(w0, d), __fdiv_rn(w1, d));
+      lo[i >> 2] = (lo[i >> 2] & ~(0xFFu << sh)) | (q << sh);
+    }
+  }
+  // d = 0 only when the block's scale code is 0 (a block far below amax): every code is 0.
+  const bool zero = !(d > 0.0f);
+  *packed = make_uint2(zero ? 0u : drop_negative_zeros(lo[0]),
+                       zero ? 0u : drop_negative_zeros(lo[1]));
   *scale = (uint8_t)s;
 }
 

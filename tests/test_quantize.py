@@ -102,3 +102,64 @@ def test_workspace_is_reused_and_rejected_when_too_small():
     tiny = torch.zeros(4, dtype=torch.uint8, device="cuda")
     with pytest.raises(lm.LmheadError):
         lm.nvfp4_quantize(W, workspace=tiny)
+
+
+def _near_boundary_weights(seed: int, amax: float):
+    """Blocks whose elements divide by their block's d = e4m3(s) * g to within a few bf16 steps
+    of the E2M1 code boundaries (0.25, 0.75, ..., 5). numpy float32 and torch's E4M3 conversion
+    only aim the values; the expected codes are the oracle's."""
+    rng = np.random.default_rng(seed)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    V, H = 256, 256
+    w = np.zeros((V, H), np.float32)
+    w[0, 0] = amax
+    g = np.float32(np.float32(bf16_round(amax)) / np.float32(2688.0))
+    six_g = np.float32(np.float32(6.0) * g)
+    for v in range(V):
+        for j in range(H // 16):
+            if v == 0 and j == 0:
+                continue
+            bmax = bf16_round(float(six_g) * 2.0 ** rng.uniform(-6, np.log2(amax / float(six_g))))
+            t = np.float32(np.float32(bmax) / six_g)
+            s = float(torch.tensor([t]).to(torch.float8_e4m3fn).to(torch.float32)[0])
+            d = np.float32(np.float32(s) * g)
+            m = rng.choice(mids, 15)
+            base = bf16_round_array(m * float(d))
+            step = rng.integers(-2, 3, 15)
+            vals = bf16_step(base, step) * rng.choice([-1.0, 1.0], 15)
+            w[v, 16 * j] = bmax
+            w[v, 16 * j + 1:16 * j + 16] = np.clip(vals, -bmax, bmax)
+    return w
+
+
+def bf16_round(x: float) -> float:
+    return float(torch.tensor([x], dtype=torch.float32).to(torch.bfloat16).to(torch.float32)[0])
+
+
+def bf16_round_array(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def bf16_step(x: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """x (bf16 values, positive) moved by k bf16 steps."""
+    bits = (x.astype(np.float32).view(np.uint32) >> 16).astype(np.int64) + k
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("seed,amax", [(88, 7.3), (89, 0.0123), (90, 411.0)])
+def test_quotients_near_code_boundaries(seed, amax):
+    """The encode pass decides most codes from one reciprocal per block and divides exactly only
+    near a code boundary; quotients aimed at the boundaries must still give the oracle's codes,
+    and enough of them land inside the exact-division band to exercise it."""
+    w = _near_boundary_weights(seed, amax)
+    bits = bf16_bits(w)
+    p, s, g = assert_same_as_oracle(bits, f"near-boundary {amax}")
+    # how many quotients fell within 2^-16 of a boundary (numpy float32 = IEEE binary32)
+    wf = (bits.astype(np.uint32) << 16).view(np.float32)
+    e4m3 = torch.from_numpy(s.view(np.uint8).copy()).view(torch.float8_e4m3fn).to(torch.float32)
+    d = (e4m3.numpy() * g).astype(np.float32).repeat(16, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = np.abs(wf / d)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rel = np.min(np.abs(x[..., None] / mids - 1.0), axis=-1)
+    assert int((rel < 2.0 ** -16).sum()) >= 20
