@@ -1,7 +1,6 @@
 """Benchmark of the LM-head library on B200: one JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|spec_verify|prefill|nvfp4]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 Workloads (seeded synthetic inputs from fp32_accumulate_lm_b200.synth; the pages use no dataset):
   decode       (default) rows in {1,2,4,8,16,32,64}, H = 2048, V = 151936, bf16 -> fp32,
@@ -9,13 +8,21 @@ Workloads (seeded synthetic inputs from fp32_accumulate_lm_b200.synth; the pages
   spec_verify  rows in {128, 97, 32}, H = 4096, V = 128256, alpha = 1/16 (3 calls per step).
   prefill      rows = 8192, H = 4096, V = 151936, alpha = 1/8 (1 call per step).
   nvfp4        W4A16 NVFP4 head, rows in {1, 16, 64, 65, 256}, H = 2048, V = 151936, bf16 out.
+  decode_f16_bias   the decode shape with fp16 operands and an fp16 embedding bias.
+  prefill_logprobs  the prefill shape, log-probabilities of one target per row, no logits out.
+  vocab_parallel_logprobs  the same with W's rows split over the GPUs (see below).
+  nvfp4_quantize    the NVFP4 quantiser of a bf16 W [151936, 2048].
+  prefill_2048      the prefill kernel on 2048 rows (a small case for profiling).
 Metric: microseconds per LM-head call (lower is better) and the fraction of the roofline the
 kernel reaches. Every call reads a weight matrix larger than L2 (126 MB); two copies of it are
 alternated so no call starts with its weights cached by the previous one.
 
 Multi-GPU: the head does not shard across the replicas (one process per GPU runs the same
 workload on its own GPU, no collective in the data path); timing is the max over ranks and
-`value` is the job's time per call: max elapsed / (calls per rank * N).
+`value` is the job's time per call: max elapsed / (calls per rank * N). The exception is
+vocab_parallel_logprobs (the prefill log-probabilities with W's rows split over the N GPUs, one
+all-gather of 12 bytes per row and GPU per call): there the N ranks make each call together, so
+`value` = max elapsed / calls, and the scaling is strong.
 
 --impl reference times the CPU oracle (the reference arm of this build) on a bounded sample of
 the same workload, scaled to the same metric; only rank 0 runs it.
@@ -50,6 +57,10 @@ WORKLOAD_TEXT = {
     "prefill_logprobs": "prefill LM head computing log-probabilities of one target token per row "
                         "(log-softmax in the epilogue, no logits written): rows=8192, H=4096, "
                         "V=151936, bf16 in, fp32 out, alpha=1/8",
+    "vocab_parallel_logprobs": "vocab-parallel prefill log-probabilities: W[151936, 4096] split "
+                               "in contiguous row slices over the GPUs; per GPU the slice's "
+                               "(max, sum, target logit) for rows=8192, an all-gather of 12 B "
+                               "per row, the merge; bf16 in, fp32 out, alpha=1/8",
     "nvfp4_quantize": "NVFP4 quantiser (absmax pass, then encode pass) of a bf16 W[151936, 2048] "
                       "into E2M1 codes, E4M3 block scales and an fp32 global scale",
     "decode_f16_bias": "decode LM head with fp16 operands and an fp16 embedding bias: rows "
@@ -159,7 +170,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs and outputs of one workload, and one step = its list of calls."""
 
-    def __init__(self, name: str, device):
+    def __init__(self, name: str, device, world: int = 1, rank: int = 0):
         import torch
         from fp32_accumulate_lm_b200 import synth
         self.name = name
@@ -168,9 +179,12 @@ class Workload:
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
                 "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16,
-                "nvfp4_quantize": synth.SEED_NVFP4, "prefill_logprobs": synth.SEED_PREFILL}[name]
+                "nvfp4_quantize": synth.SEED_NVFP4, "prefill_logprobs": synth.SEED_PREFILL,
+                "vocab_parallel_logprobs": synth.SEED_PREFILL}[name]
         rmax = max(rows_list)
         self.quantize = name == "nvfp4_quantize"
+        self.vocab_parallel = name == "vocab_parallel_logprobs"
+        self.world = world
         if self.quantize:
             # one call quantises all V rows of a bf16 W; two copies alternate (each > L2)
             import fp32_accumulate_lm_b200 as lm
@@ -178,6 +192,7 @@ class Workload:
             self.bias = None
             self.nvfp4 = False
             self.logprobs = False
+            self.vocab_parallel = False
             self.weights = [synth.weight(V, H, std, seed + i, device=device) for i in (0, 1)]
             self.hidden = self.weights[0]
             self.hid = {V: self.weights[0]}
@@ -198,6 +213,16 @@ class Workload:
             self.g = 1.0 / 4096
             self.outs = {r: torch.empty((r, V), dtype=torch.bfloat16, device=device)
                          for r in rows_list}
+        elif self.vocab_parallel:
+            # this rank's contiguous slice of each of the two weight copies
+            import fp32_accumulate_lm_b200 as lm
+            self.v_begin, self.V_shard = lm.vocab_shard(V, world, rank)
+            self.weights = []
+            for i in (0, 1):
+                full = synth.weight(V, H, std, seed + i, device=device, dtype=self.dtype)
+                self.weights.append(full if world == 1 else
+                                    full[self.v_begin:self.v_begin + self.V_shard].clone())
+                del full
         else:
             self.weights = [synth.weight(V, H, std, seed + i, device=device, dtype=self.dtype)
                             for i in (0, 1)]
@@ -205,7 +230,7 @@ class Workload:
                          for r in rows_list}
         self.hid = {r: self.hidden[:r] for r in rows_list}
         self.general = self.bias is not None or self.dtype != torch.bfloat16  # lmhead_logits_f32
-        self.logprobs = name == "prefill_logprobs"
+        self.logprobs = name in ("prefill_logprobs", "vocab_parallel_logprobs")
         if self.logprobs:
             import fp32_accumulate_lm_b200 as lm
             gen = torch.Generator(device="cpu")
@@ -213,8 +238,12 @@ class Workload:
             self.targets = torch.randint(0, V, (rmax,), generator=gen, dtype=torch.int32).to(device)
             self.outs = {r: torch.empty((r,), dtype=torch.float32, device=device) for r in rows_list}
             self.lse = {r: torch.empty((r,), dtype=torch.float32, device=device) for r in rows_list}
-            self.ws = torch.empty((lm.logprobs_workspace_bytes(rmax, V),), dtype=torch.uint8,
+            vw = self.V_shard if self.vocab_parallel else V
+            self.ws = torch.empty((lm.logprobs_workspace_bytes(rmax, vw),), dtype=torch.uint8,
                                   device=device)
+            if self.vocab_parallel:
+                self.stats = {r: torch.empty((r, 3), dtype=torch.float32, device=device)
+                              for r in rows_list}
         self.calls = 0
 
     def call(self, r: int, hidden=None, out=None, stream=None):
@@ -232,6 +261,10 @@ class Workload:
         o = self.outs[r] if out is None else out
         if self.nvfp4:
             lm.logits_w4a16_nvfp4(h, w[0], w[1], self.g, self.alpha, out=o, stream=stream)
+        elif self.vocab_parallel:
+            lm.logprobs_vocab_parallel(h, w, self.v_begin, self.targets[:r], self.alpha,
+                                       workspace=self.ws, stats=self.stats[r],
+                                       out=(o, self.lse[r]), stream=stream)
         elif self.logprobs:
             lm.logprobs_f32(h, w, self.targets[:r], self.alpha, workspace=self.ws,
                             out=(o, self.lse[r]), stream=stream)
@@ -246,12 +279,19 @@ class Workload:
             return 2 * V * H * 2 + V * H // 2 + V * H // 16 + 4
         if self.nvfp4:
             return V * H // 2 + V * H // 16 + 4 + r * H * 2 + r * V * 2
+        if self.vocab_parallel:  # this rank's slice; the stats out, gathered, read by the merge
+            n = self.V_shard
+            n_chunks = 4 * ((n + 127) // 128)
+            return (n * H * 2 + r * H * 2 + r * 4 + 2 * r * n_chunks * 8 + r * 12
+                    + 2 * self.world * r * 12 + r * 8)
         if self.logprobs:  # W, hidden, targets in; the chunk pairs out and back; lp, lse out
             n_chunks = 4 * ((V + 127) // 128)
             return V * H * 2 + r * H * 2 + r * 4 + 2 * r * n_chunks * 8 + r * 8
         return V * H * 2 + r * H * 2 + r * V * 4 + (V * 2 if self.bias is not None else 0)
 
     def flops_of(self, r: int) -> int:
+        if self.vocab_parallel:
+            return 2 * r * self.H * self.V_shard
         return 0 if self.quantize else 2 * r * self.H * self.V
 
 
@@ -312,7 +352,7 @@ def run_ours(args) -> dict | None:
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
-    wl = Workload(args.workload, dev)
+    wl = Workload(args.workload, dev, world, rank)
     stream = torch.cuda.current_stream()
     rl = wl.rows_list
     calls_per_step = len(rl)
@@ -359,7 +399,8 @@ def run_ours(args) -> dict | None:
         tot_bytes += b
         tot_flops += fl
         tot_ms += mean_ms
-    tensor_bound = args.workload.startswith("prefill")  # prefill, its profiling case, log-probs
+    # prefill, its profiling case, log-probs, vocab-parallel log-probs
+    tensor_bound = args.workload.startswith("prefill") or wl.vocab_parallel
     if tensor_bound:
         achieved = tot_flops / (tot_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -380,22 +421,27 @@ def run_ours(args) -> dict | None:
     # ---- end to end through the C ABI: pinned host hidden -> device, call, logits -> pinned host
     e2e = run_e2e(args, wl, world)
 
-    value = job_us_per_call(elapsed_ms, args.steps, calls_per_step, world)
+    # Replicas: every rank makes whole calls. Vocab-parallel: the ranks make each call together.
+    value = job_us_per_call(elapsed_ms, args.steps, calls_per_step,
+                            1 if wl.vocab_parallel else world)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if wl.vocab_parallel else "weak", "vs_baseline": None,
         "dtype": ("f32" if wl.quantize else "e2m1xbf16" if wl.nvfp4 else
                   "f16" if wl.dtype == torch.float16 else "bf16"),
         "data": "synthetic (seeded N(0,1) hidden, N(0,std) weights; no dataset on the pages)",
         "config": {"workload": WORKLOAD_TEXT[args.workload],
                    "l2": "weights 2x larger than L2 per call; two weight copies alternated",
-                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "parallelism": (f"vocab-parallel x{world} (all-gather of the row stats)"
+                                   if wl.vocab_parallel else
+                                   f"replicas x{world} (no data-path collective)"),
                    "calls_per_step": calls_per_step, "per_rows": detail},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": n_ev * (2 if (wl.quantize or wl.logprobs) else 1),
+        "gpu_launches": n_ev * (3 if wl.vocab_parallel else
+                                2 if (wl.quantize or wl.logprobs) else 1),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -435,7 +481,8 @@ def run_e2e(args, wl, world: int) -> dict:
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = sum(h_host[r].numel() * h_host[r].element_size() for r in rl)
     d2h = sum(o_host[r].numel() * o_host[r].element_size() for r in rl)
-    return {"value": round(ms * 1e3 / (steps * len(rl) * world), 3), "unit": UNIT,
+    share = 1 if wl.vocab_parallel else world   # calls made together count once
+    return {"value": round(ms * 1e3 / (steps * len(rl) * share), 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 

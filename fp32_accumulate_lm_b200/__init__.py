@@ -19,7 +19,9 @@ import threading
 
 __all__ = [
     "LmheadError", "load_library", "library_path", "logits_bf16_f32", "logits_f32", "logprobs_f32",
-    "lmhead_logprobs_f32", "logprobs_workspace_bytes",
+    "lmhead_logprobs_f32", "logprobs_workspace_bytes", "lmhead_logprobs_shard_stats_f32",
+    "lmhead_logprobs_merge_shards", "logprobs_shard_stats_f32", "logprobs_merge_shards",
+    "vocab_shard", "gather_shard_stats", "logprobs_vocab_parallel",
     "logits_w4a16_nvfp4", "lmhead_logits_bf16_f32", "lmhead_logits_f32",
     "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "lmhead_nvfp4_quantize_noalloc",
     "nvfp4_quantize",
@@ -72,6 +74,11 @@ def load_library():
         lib.lmhead_logprobs_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp, vp, vp,
                                             ctypes.c_size_t, vp]
         lib.lmhead_logprobs_f32.restype = i32
+        lib.lmhead_logprobs_shard_stats_f32.argtypes = [vp, i32, i64, i64, vp, i64, i64, f32, vp,
+                                                        vp, vp, vp, ctypes.c_size_t, vp]
+        lib.lmhead_logprobs_shard_stats_f32.restype = i32
+        lib.lmhead_logprobs_merge_shards.argtypes = [vp, i64, i64, vp, vp, vp]
+        lib.lmhead_logprobs_merge_shards.restype = i32
         lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
         lib.lmhead_logits_w4a16_nvfp4.restype = i32
         lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
@@ -120,6 +127,22 @@ def lmhead_logprobs_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: i
                                                bias_ptr or None, targets_ptr, logprobs_ptr,
                                                lse_ptr or None, workspace_ptr, workspace_bytes,
                                                stream)
+
+
+def lmhead_logprobs_shard_stats_f32(hidden_ptr: int, dtype: int, rows: int, H: int,
+                                    w_shard_ptr: int, V_shard: int, v_begin: int, alpha: float,
+                                    bias_shard_ptr: int, targets_ptr: int, stats_ptr: int,
+                                    workspace_ptr: int, workspace_bytes: int,
+                                    stream: int = 0) -> int:
+    return load_library().lmhead_logprobs_shard_stats_f32(
+        hidden_ptr, dtype, rows, H, w_shard_ptr, V_shard, v_begin, alpha, bias_shard_ptr or None,
+        targets_ptr, stats_ptr, workspace_ptr, workspace_bytes, stream)
+
+
+def lmhead_logprobs_merge_shards(stats_ptr: int, shards: int, rows: int, logprobs_ptr: int,
+                                 lse_ptr: int, stream: int = 0) -> int:
+    return load_library().lmhead_logprobs_merge_shards(stats_ptr, shards, rows, logprobs_ptr,
+                                                       lse_ptr or None, stream)
 
 
 def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
@@ -303,6 +326,105 @@ def logprobs_f32(hidden, W, targets, alpha: float = 1.0, bias=None, workspace=No
     if st != LMHEAD_OK:
         raise LmheadError(st, "lmhead_logprobs_f32")
     return lp, lse
+
+
+def vocab_shard(V: int, world: int, rank: int):
+    """(v_begin, V_shard): the contiguous slice of W's V rows that GPU ``rank`` of ``world`` holds
+    for the vocab-parallel head. The first V % world ranks hold one row more; V >= world."""
+    _check(world >= 1 and 0 <= rank < world and V >= world, "need V >= world > rank >= 0")
+    base, extra = divmod(V, world)
+    return rank * base + min(rank, extra), base + (1 if rank < extra else 0)
+
+
+def logprobs_shard_stats_f32(hidden, W_shard, v_begin: int, targets, alpha: float = 1.0,
+                             bias_shard=None, workspace=None, out=None, stream=None):
+    """fp32 [rows, 3] per-row (max, sum of exp(z - max), target logit or NaN) over the logits of
+    this GPU's vocab slice W_shard = W[v_begin : v_begin + V_shard] (targets are global ids)."""
+    import torch
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}.get(hidden.dtype)
+    _check(dt is not None and W_shard.dtype == hidden.dtype,
+           "bf16 or fp16 operands of one dtype required")
+    _check(hidden.dim() == 2 and W_shard.dim() == 2 and hidden.shape[1] == W_shard.shape[1],
+           "shape mismatch")
+    _check(hidden.is_cuda and W_shard.is_cuda and hidden.is_contiguous()
+           and W_shard.is_contiguous(), "contiguous CUDA tensors required")
+    rows, H = hidden.shape
+    V_shard = W_shard.shape[0]
+    _check(targets.dtype == torch.int32 and targets.is_cuda and targets.is_contiguous()
+           and tuple(targets.shape) == (rows,), "targets must be a contiguous int32 [rows] tensor")
+    if bias_shard is not None:
+        _check(bias_shard.dtype == hidden.dtype and bias_shard.is_cuda
+               and bias_shard.is_contiguous() and tuple(bias_shard.shape) == (V_shard,),
+               "bias_shard must be a contiguous [V_shard] tensor of the dtype")
+    if out is None:
+        out = torch.empty((rows, 3), dtype=torch.float32, device=hidden.device)
+    _check(out.dtype == torch.float32 and out.is_contiguous() and out.numel() == rows * 3,
+           "out must be a contiguous fp32 [rows, 3] tensor")
+    need = logprobs_workspace_bytes(rows, V_shard)
+    if workspace is None:
+        workspace = torch.empty((max(need, 8),), dtype=torch.uint8, device=hidden.device)
+    st = lmhead_logprobs_shard_stats_f32(
+        hidden.data_ptr(), dt, rows, H, W_shard.data_ptr(), V_shard, int(v_begin), float(alpha),
+        0 if bias_shard is None else bias_shard.data_ptr(), targets.data_ptr(), out.data_ptr(),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logprobs_shard_stats_f32")
+    return out
+
+
+def logprobs_merge_shards(stats, out=None, stream=None):
+    """(logprobs [rows], lse [rows]) fp32 from the gathered shard stats, fp32 [g, rows, 3] in
+    shard order."""
+    import torch
+    _check(stats.dtype == torch.float32 and stats.is_cuda and stats.is_contiguous()
+           and stats.dim() == 3 and stats.shape[2] == 3, "stats must be a contiguous fp32 "
+           "[g, rows, 3] CUDA tensor")
+    g, rows = stats.shape[0], stats.shape[1]
+    if out is None:
+        lp = torch.empty((rows,), dtype=torch.float32, device=stats.device)
+        lse = torch.empty((rows,), dtype=torch.float32, device=stats.device)
+    else:
+        lp, lse = out
+    st = lmhead_logprobs_merge_shards(stats.data_ptr(), g, rows, lp.data_ptr(),
+                                      0 if lse is None else lse.data_ptr(),
+                                      _stream_handle(stream))
+    if st != LMHEAD_OK:
+        raise LmheadError(st, "lmhead_logprobs_merge_shards")
+    return lp, lse
+
+
+def gather_shard_stats(stats, group=None):
+    """The exchange of the vocab-parallel log-probs: every rank's [rows, 3] stats gathered into
+    [world, rows, 3] in rank order (one all-gather of rows * 12 bytes per rank; NCCL for CUDA
+    tensors). Rank r must hold the r-th vocab slice."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return stats.view(1, *stats.shape)   # a single process holds the whole vocabulary
+    world = dist.get_world_size(group)
+    flat = stats.reshape(-1)
+    out = torch.empty((world * flat.numel(),), dtype=stats.dtype, device=stats.device)
+    dist.all_gather_into_tensor(out, flat, group=group)
+    return out.view(world, *stats.shape)
+
+
+def logprobs_vocab_parallel(hidden, W_shard, v_begin: int, targets, alpha: float = 1.0,
+                            bias_shard=None, group=None, workspace=None, stats=None, out=None,
+                            stream=None):
+    """(logprobs [rows], lse [rows]) of the whole vocabulary on every rank of ``group``, each
+    rank holding its slice W_shard = W[v_begin : v_begin + V_shard] (vocab_shard gives the
+    split) and the same hidden rows and targets: shard stats, one all-gather, merge. Without a
+    process group the caller is the only rank. ``workspace``, ``stats`` ([rows, 3]) and ``out``
+    are allocated here unless given."""
+    import torch
+    _check(stream is None or isinstance(stream, torch.cuda.Stream),
+           "stream must be a torch.cuda.Stream (the all-gather is ordered on it)")
+    stats = logprobs_shard_stats_f32(hidden, W_shard, v_begin, targets, alpha, bias_shard,
+                                     workspace=workspace, out=stats, stream=stream)
+    with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+        gathered = gather_shard_stats(stats, group)
+    return logprobs_merge_shards(gathered, out=out, stream=stream)
 
 
 def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha: float = 1.0,

@@ -384,6 +384,8 @@ struct LogprobArgs {
   float* logprobs;
   float* lse;
   void* workspace;
+  int64_t v_begin;  // vocab id of W's first row
+  float* stats;     // vocab-shard mode: per-row (max, sum, target logit) instead of logprobs
 };
 
 int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W, int64_t V,
@@ -402,7 +404,11 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   p.n_chunks = (int32_t)(4 * ((V + lmh::kBM - 1) / lmh::kBM));
   p.partials = lp != nullptr ? reinterpret_cast<float2*>(lp->workspace) : nullptr;
   p.targets = lp != nullptr ? lp->targets : nullptr;
-  p.target_z = lp != nullptr ? lp->logprobs : nullptr;
+  p.target_base = lp != nullptr ? lp->v_begin : 0;
+  // The target's logit is parked where the combine kernel reads it: the logprobs slot of the
+  // row, or the third word of the row's shard stats.
+  p.target_z = lp == nullptr ? nullptr : lp->stats != nullptr ? lp->stats + 2 : lp->logprobs;
+  p.tz_stride = lp != nullptr && lp->stats != nullptr ? 3 : 1;
   p.bias = reinterpret_cast<const uint16_t*>(bias);
   p.alpha = alpha;
   p.fp16 = dtype == LMHEAD_DTYPE_F16 ? 1 : 0;
@@ -441,7 +447,8 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   if (lp != nullptr) {
     const int64_t blocks = (rows + lmh::kCombineRows - 1) / lmh::kCombineRows;
     lmh::lmhead_logprob_combine_kernel<<<(unsigned)blocks, 1024, 0, (cudaStream_t)stream>>>(
-        p.partials, p.n_chunks, rows, V, lp->targets, lp->logprobs, lp->lse);
+        p.partials, p.n_chunks, rows, V, lp->targets, lp->logprobs, lp->lse, lp->v_begin,
+        lp->stats);
   }
   return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
@@ -508,8 +515,64 @@ int lmhead_logprobs_f32(const void* hidden, int dtype, int64_t rows, int64_t H, 
       if (&o2 != &o && o2.p != nullptr && overlaps(o.p, o.bytes, o2.p, o2.bytes))
         return LMHEAD_ERR_ALIAS;
   }
-  const LogprobArgs lp{targets, logprobs, lse, workspace};
+  const LogprobArgs lp{targets, logprobs, lse, workspace, 0, nullptr};
   return run_f32_head(hidden, dtype, rows, H, W, V, alpha, bias, nullptr, &lp, stream);
+}
+
+int lmhead_logprobs_shard_stats_f32(const void* hidden, int dtype, int64_t rows, int64_t H,
+                                    const void* W_shard, int64_t V_shard, int64_t v_begin,
+                                    float alpha, const void* bias_shard, const int32_t* targets,
+                                    float* stats, void* workspace, size_t workspace_bytes,
+                                    lmhead_stream_t stream) {
+  const int st = check_f32_head_args(hidden, dtype, rows, H, W_shard, V_shard, bias_shard);
+  if (st != LMHEAD_OK) return st;
+  // Token ids are int32: the shard must lie inside [0, 2^31).
+  if (v_begin < 0 || v_begin > kInt32Max || V_shard > (int64_t)kInt32Max + 1 - v_begin)
+    return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (targets == nullptr || stats == nullptr || workspace == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(targets, 4) || !aligned(stats, 4) || !aligned(workspace, 8))
+    return LMHEAD_ERR_ALIGN;
+  if (workspace_bytes < lmhead_logprobs_workspace_bytes(rows, V_shard)) return LMHEAD_ERR_SHAPE;
+  const struct { const void* p; int64_t bytes; } in[4] = {
+      {hidden, rows * H * 2},
+      {W_shard, V_shard * H * 2},
+      {bias_shard, bias_shard ? V_shard * 2 : 0},
+      {targets, rows * 4}};
+  const int64_t stats_bytes = rows * 12;
+  for (const auto& i : in) {
+    if (i.p == nullptr) continue;
+    if (overlaps(stats, stats_bytes, i.p, i.bytes) ||
+        overlaps(workspace, (int64_t)workspace_bytes, i.p, i.bytes))
+      return LMHEAD_ERR_ALIAS;
+  }
+  if (overlaps(stats, stats_bytes, workspace, (int64_t)workspace_bytes)) return LMHEAD_ERR_ALIAS;
+  const LogprobArgs lp{targets, nullptr, nullptr, workspace, v_begin, stats};
+  return run_f32_head(hidden, dtype, rows, H, W_shard, V_shard, alpha, bias_shard, nullptr, &lp,
+                      stream);
+}
+
+int lmhead_logprobs_merge_shards(const float* stats, int64_t shards, int64_t rows,
+                                 float* logprobs, float* lse, lmhead_stream_t stream) {
+  if (shards <= 0 || shards > kInt32Max || rows < 0) return LMHEAD_ERR_SHAPE;
+  if (rows > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (stats == nullptr || logprobs == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(stats, 4) || !aligned(logprobs, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return LMHEAD_ERR_ALIGN;
+  const int64_t stats_bytes = shards * rows * 12;
+  if (overlaps(logprobs, rows * 4, stats, stats_bytes) ||
+      (lse != nullptr && (overlaps(lse, rows * 4, stats, stats_bytes) ||
+                          overlaps(lse, rows * 4, logprobs, rows * 4))))
+    return LMHEAD_ERR_ALIAS;
+  DeviceInfo dev;
+  const int st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+  const int64_t blocks = (rows + lmh::kMergeThreads - 1) / lmh::kMergeThreads;
+  lmh::lmhead_logprob_merge_shards_kernel<<<(unsigned)blocks, lmh::kMergeThreads, 0,
+                                            (cudaStream_t)stream>>>(stats, (int32_t)shards, rows,
+                                                                    logprobs, lse);
+  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
 int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,

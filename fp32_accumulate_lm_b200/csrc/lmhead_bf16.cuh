@@ -50,7 +50,9 @@ struct Bf16HeadParams {
   int32_t n_chunks;         // 32-entry vocab chunks per row: 4 * ceil(V / 128)
   float2* partials;         // [n_chunks, rows] (max, sum of exp(z - max)) per chunk and row
   const int32_t* targets;   // [rows] token ids
-  float* target_z;          // [rows] the target's logit (written by the chunk that holds it)
+  int64_t target_base;      // vocab id of W's first row (a vocab shard's offset; 0 otherwise)
+  float* target_z;          // the target's logit, row r at target_z[r * tz_stride] (written by
+  int32_t tz_stride;        // the chunk that holds it)
   WaitCfg wait;
 };
 
@@ -71,11 +73,17 @@ __device__ __forceinline__ void merge_max_sum(float m1, float s1, float m2, floa
 // warps serves 32 rows: lane i is row i; warp w folds chunk segment w in order (coalesced reads
 // of the chunk-major pairs), then warp 0 folds the 32 segment pairs of its row in order. The
 // result depends only on the row's logits and V.
+//
+// With `stats` set (one vocab shard of a larger head, whose first row is vocab id v_begin), the
+// row's pair and target logit are written instead: stats[3 r .. 3 r + 2] = (max, sum of
+// exp(z - max), z[target]), the last NaN when the shard does not hold the target. The main
+// kernel left z[target] in stats[3 r + 2].
 constexpr int kCombineRows = 32;
 __global__ void __launch_bounds__(1024)
     lmhead_logprob_combine_kernel(const float2* __restrict__ partials, int32_t n_chunks,
                                   int64_t rows, int64_t V, const int32_t* __restrict__ targets,
-                                  float* logprobs, float* lse_out) {
+                                  float* logprobs, float* lse_out, int64_t v_begin,
+                                  float* stats) {
   __shared__ float2 seg[32][kCombineRows + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kCombineRows + lane;
@@ -95,11 +103,44 @@ __global__ void __launch_bounds__(1024)
     m = -INFINITY;
     s = 0.0f;
     for (int w = 0; w < 32; ++w) merge_max_sum(m, s, seg[w][lane].x, seg[w][lane].y, m, s);
+    const int64_t t = (int64_t)targets[row] - v_begin;
+    const bool held = t >= 0 && t < V;
+    if (stats != nullptr) {
+      stats[3 * row] = m;
+      stats[3 * row + 1] = s;
+      if (!held) stats[3 * row + 2] = __int_as_float(0x7fc00000);
+      return;
+    }
     const float l = __fadd_rn(m, logf(s));
     if (lse_out != nullptr) lse_out[row] = l;
-    const int32_t t = targets[row];
-    logprobs[row] = (t >= 0 && t < V) ? __fsub_rn(logprobs[row], l) : __int_as_float(0x7fc00000);
+    logprobs[row] = held ? __fsub_rn(logprobs[row], l) : __int_as_float(0x7fc00000);
   }
+}
+
+// The vocab-parallel finish: stats [shards][rows][3] holds each shard's (max, sum, target logit)
+// of every row; fold the shards in order into the row's pair, then lse = max + log(sum) and
+// logprob = z[target] - lse, taking z[target] from the first shard that holds it (NaN if none).
+// One thread per row; the reads of a warp are 12-byte strided, a few KB per call.
+constexpr int kMergeThreads = 256;
+__global__ void __launch_bounds__(kMergeThreads)
+    lmhead_logprob_merge_shards_kernel(const float* __restrict__ stats, int32_t shards,
+                                       int64_t rows, float* logprobs, float* lse_out) {
+  const int64_t row = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  if (row >= rows) return;
+  float m = -INFINITY, s = 0.0f, zt = __int_as_float(0x7fc00000);
+  bool found = false;
+  for (int g = 0; g < shards; ++g) {
+    const float* q = stats + 3 * ((int64_t)g * rows + row);
+    merge_max_sum(m, s, q[0], q[1], m, s);
+    const float z = q[2];
+    if (!found && !isnan(z)) {
+      zt = z;
+      found = true;
+    }
+  }
+  const float l = __fadd_rn(m, logf(s));
+  if (lse_out != nullptr) lse_out[row] = l;
+  logprobs[row] = __fsub_rn(zt, l);
 }
 
 template <int NSUB>
@@ -292,7 +333,12 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           // over the lanes, so lanes 2i and 2i + 1 both hold row i's pair.
           const int32_t chunk = (int32_t)(tc.v0 / kBM) * 4 + quarter;
           const int64_t rl = r0 + c + lane;
-          const int32_t tgt = (lane < 16 && rl < p.rows) ? p.targets[rl] : -1;
+          // The target as an index into this call's W (-1 when W does not hold it).
+          int32_t tgt = -1;
+          if (lane < 16 && rl < p.rows) {
+            const int64_t tv = (int64_t)p.targets[rl] - p.target_base;
+            tgt = (tv >= 0 && tv < p.V) ? (int32_t)tv : -1;
+          }
           // Which of these 16 rows has its target among this warp's 32 entries (usually none).
           const int64_t wv0 = tc.v0 + quarter * 32;
           const uint32_t hits = __ballot_sync(0xffffffffu, tgt >= wv0 && tgt < wv0 + 32);
@@ -305,7 +351,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
                                                 : __fmul_rn(p.alpha, __fadd_rn(a, b));
             if (hits & (1u << j)) {  // warp-uniform
               const int32_t tj = __shfl_sync(0xffffffffu, tgt, j);
-              if (v_ok && v == (int64_t)tj) p.target_z[r0 + c + j] = z;
+              if (v_ok && v == (int64_t)tj) p.target_z[(r0 + c + j) * p.tz_stride] = z;
             }
             zz[j] = z;
             pm[j] = z;

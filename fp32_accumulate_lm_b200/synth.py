@@ -43,6 +43,8 @@ WORKLOADS = {
     "nvfp4": ([1, 16, 64, 65, 256], 2048, 151936, 0.02, 1.0 / 8),
     # the prefill shape computing log-probabilities of one target token per row (no logits out)
     "prefill_logprobs": ([8192], 4096, 151936, 0.02, 1.0 / 8),
+    # the prefill log-probabilities with W's rows split over the GPUs (each holds one slice)
+    "vocab_parallel_logprobs": ([8192], 4096, 151936, 0.02, 1.0 / 8),
     # the NVFP4 quantiser on the NVFP4 head's weight shape (rows = the V rows quantised per call)
     "nvfp4_quantize": ([151936], 2048, 151936, 0.02, 1.0),
     # the decode shape with fp16 operands and an fp16 embedding bias

@@ -132,6 +132,46 @@ int lmhead_logprobs_f32(const void* hidden, int dtype, int64_t rows, int64_t H, 
                         lmhead_stream_t stream);
 
 /*
+ * Vocab-parallel log-probabilities, in two calls around one exchange. "FP32 LM head skip FP32
+ * cast" (key source excerpt, `_compute_lm_head`) takes the head as a VocabParallelEmbedding: each
+ * of g GPUs holds a contiguous slice of W's rows, and the log-softmax of a row needs all of them.
+ * lm_head_nvfp4_rows.rs (its install guard) keeps its own head to one GPU (tp_world_size 1);
+ * this pair is for the fp32 head.
+ *
+ * 1. lmhead_logprobs_shard_stats_f32: on the GPU holding W_shard = W[v_begin, v_begin + V_shard),
+ *    for each row r, with z the fp32 logits lmhead_logits_f32 would write for that slice (same
+ *    bits as the same columns of the whole head):
+ *      stats[3 r]     = m = max_v z[r, v]
+ *      stats[3 r + 1] = s = sum_v exp(z[r, v] - m)          (fp32, fixed order)
+ *      stats[3 r + 2] = z[r, targets[r]] if v_begin <= targets[r] < v_begin + V_shard, else NaN
+ *    targets are global token ids. bias_shard is the slice of the bias (or NULL). The workspace
+ *    is as lmhead_logprobs_f32's for V_shard rows of W. Two kernels are enqueued.
+ * 2. The caller gathers the g stats arrays into one [g][rows][3] array in shard order (an
+ *    all-gather of rows * 12 bytes per GPU).
+ * 3. lmhead_logprobs_merge_shards folds the shards of each row in order:
+ *      (m, s) = union of the shards' pairs,  lse[r] = m + log s,
+ *      logprobs[r] = z[r, targets[r]] - lse[r]   (from the first shard that holds the target;
+ *                                                 NaN when none does)
+ *    One kernel is enqueued.
+ * Results are deterministic for a given split; against the exact values over the same fp32
+ * logits they are as accurate as lmhead_logprobs_f32's (one more fold per shard).
+ *
+ *   v_begin    >= 0; v_begin + V_shard <= 2^31 (token ids are int32), else LMHEAD_ERR_SHAPE
+ *   stats      fp32 [rows][3], 4-byte aligned (output of 1, input of 3)
+ *   shards     g >= 1
+ *   logprobs   fp32 [rows]; lse fp32 [rows] or NULL; 4-byte aligned (outputs of 3)
+ * Outputs must not overlap the inputs, the workspace or each other. Each returns an
+ * lmhead_status.
+ */
+int lmhead_logprobs_shard_stats_f32(const void* hidden, int dtype, int64_t rows, int64_t H,
+                                    const void* W_shard, int64_t V_shard, int64_t v_begin,
+                                    float alpha, const void* bias_shard, const int32_t* targets,
+                                    float* stats, void* workspace, size_t workspace_bytes,
+                                    lmhead_stream_t stream);
+int lmhead_logprobs_merge_shards(const float* stats, int64_t shards, int64_t rows,
+                                 float* logprobs, float* lse, lmhead_stream_t stream);
+
+/*
  * Entry 2: bf16 logits from the W4A16 NVFP4 head.
  *   W[v, k]      = e2m1(code[v, k]) * e4m3(w_scales[v, k / 16])      (exact in bf16)
  *   logits[r, v] = bf16_rn( fl32( fl32(acc[r, v] * w_global_scale) * alpha ) ),

@@ -171,3 +171,55 @@ def test_torch_wrapper_rejects_wrong_dtypes():
     w = torch.zeros(8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         lm.logits_bf16_f32(h, w, 1.0)
+
+
+def test_vocab_shard_argument_errors(lib):
+    """lmhead_logprobs_shard_stats_f32 / lmhead_logprobs_merge_shards: the shard must lie inside
+    the int32 token-id range, and outputs may not overlap inputs, the workspace or each other."""
+    f = lm.lmhead_logprobs_shard_stats_f32
+    T, ST, WS = 0x60000000, 0x61000000, 0x63000000
+    need = lm.logprobs_workspace_bytes(4, 300)
+    args = lambda **kw: dict(dict(h=A16, dt=0, rows=4, H=64, w=B16, V=300, v0=1000, alpha=1.0,
+                                  bias=0, t=T, st=ST, ws=WS, nb=need), **kw)
+    call = lambda a: f(a["h"], a["dt"], a["rows"], a["H"], a["w"], a["V"], a["v0"], a["alpha"],
+                       a["bias"], a["t"], a["st"], a["ws"], a["nb"], 0)
+    assert call(args()) not in (1, 2, 3, 7)                  # valid: reaches the device check
+    assert call(args(v0=-1)) == 2
+    assert call(args(v0=2 ** 31 - 300)) not in (1, 2, 3, 7)  # last id 2^31 - 1: still valid
+    assert call(args(v0=2 ** 31 - 299)) == 2                 # one past the int32 ids
+    assert call(args(dt=3)) == 2
+    assert call(args(t=0)) == 1 and call(args(st=0)) == 1 and call(args(ws=0)) == 1
+    assert call(args(nb=need - 8)) == 2
+    assert call(args(t=T + 2)) == 3 and call(args(st=ST + 2)) == 3 and call(args(ws=WS + 4)) == 3
+    assert call(args(st=B16 + 64)) == 7                      # stats over the weight slice
+    assert call(args(st=T)) == 7                             # stats over the targets
+    assert call(args(st=WS + 8)) == 7                        # stats inside the workspace
+    assert call(args(ws=A16)) == 7                           # workspace over hidden
+    assert call(args(rows=0, h=0, w=0, t=0, st=0, ws=0)) == 0
+    m = lm.lmhead_logprobs_merge_shards
+    LP, LSE = 0x64000000, 0x65000000
+    assert m(ST, 0, 4, LP, LSE, 0) == 2                      # no shards
+    assert m(ST, 2, -1, LP, LSE, 0) == 2
+    assert m(0, 2, 4, LP, LSE, 0) == 1 and m(ST, 2, 4, 0, LSE, 0) == 1
+    assert m(ST + 2, 2, 4, LP, LSE, 0) == 3 and m(ST, 2, 4, LP + 1, LSE, 0) == 3
+    assert m(ST, 2, 4, ST + 88, LSE, 0) == 7                 # logprobs inside the 96-byte stats
+    assert m(ST, 2, 4, LP, LP + 4, 0) == 7                   # lse over logprobs
+    assert m(ST, 2, 4, LP, 0, 0) not in (1, 2, 3, 7)         # lse is optional
+    assert m(0, 3, 0, 0, 0, 0) == 0                          # rows == 0
+
+
+def test_vocab_shard_split():
+    """vocab_shard: contiguous, disjoint, covering slices whose sizes differ by at most one."""
+    for V in (8, 1000, 128256, 151936):
+        for world in range(1, 9):
+            parts = [lm.vocab_shard(V, world, r) for r in range(world)]
+            assert parts[0][0] == 0
+            for (b0, n0), (b1, _) in zip(parts, parts[1:]):
+                assert b0 + n0 == b1
+            assert parts[-1][0] + parts[-1][1] == V
+            sizes = [n for _, n in parts]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    with pytest.raises(ValueError):
+        lm.vocab_shard(3, 4, 0)
+    with pytest.raises(ValueError):
+        lm.vocab_shard(100, 2, 2)

@@ -17,7 +17,8 @@ KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "
 
 
 @pytest.mark.parametrize("workload", ["decode", "spec_verify", "nvfp4", "decode_f16_bias",
-                                      "prefill", "prefill_logprobs", "nvfp4_quantize"])
+                                      "prefill", "prefill_logprobs", "nvfp4_quantize",
+                                      "vocab_parallel_logprobs"])
 def test_bench_line(workload):
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", workload,
                           "--steps", "1", "--warmup", "3", "--no-cpu-baseline"],
