@@ -1,5 +1,6 @@
 // C ABI of the LM-head library (declared in include/lmhead.h): argument validation, TMA
-// descriptor set-up and the launch of one kernel per call on the caller's stream.
+// descriptor set-up and the launches on the caller's stream (one kernel per head call; two for
+// the log-probabilities and for the quantiser; one for the vocab-slice merge).
 //
 // The operation: logits = alpha * hidden @ W^T with bf16 inputs, fp32 accumulation and alpha in
 // the epilogue ("[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)",

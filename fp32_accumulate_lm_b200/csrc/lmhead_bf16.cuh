@@ -24,7 +24,9 @@
 //              IEEE fp32 multiply by alpha, store. In log-prob mode the logits are not stored:
 //              each warp reduces its 32 vocab entries to (max, sum of exp(z - max)) per row
 //              and writes that pair to the workspace, and the lane holding a row's target token
-//              writes that logit; a combine kernel (lmhead_logprob_combine_kernel) finishes.
+//              writes that logit; a combine kernel (lmhead_logprob_combine_kernel) finishes,
+//              or, when W is one vocab slice of a larger head, writes the row's (max, sum,
+//              target logit) for lmhead_logprob_merge_shards_kernel to fold across slices.
 // Tile ownership: see TileSched.
 #pragma once
 

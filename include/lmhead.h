@@ -4,9 +4,11 @@
  *   logits[rows, V] = alpha * (hidden[rows, H] @ W[V, H]^T)
  *
  * Entry 1 takes bf16 hidden and W, accumulates in fp32 and writes fp32 logits; no fp32 copy of
- * either operand is ever made. Its general form also takes fp16 operands and an embedding bias. Entry 2 is the W4A16 NVFP4 head: E2M1 weights with per-16 E4M3
- * block scales and one fp32 per-tensor scale, bf16 activations that are never quantised, bf16
- * logits.
+ * either operand is ever made. Its general form also takes fp16 operands and an embedding bias.
+ * Entry 2 is the W4A16 NVFP4 head: E2M1 weights with per-16 E4M3 block scales and one fp32
+ * per-tensor scale, bf16 activations that are never quantised, bf16 logits. Around them: the
+ * log-probabilities of given tokens over the fp32 logits (whole vocabulary, or one vocab slice
+ * per GPU plus a merge), and the NVFP4 quantiser.
  *
  * The operation comes from these pages:
  *  - "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)", "Purpose" and
@@ -27,8 +29,9 @@
  *  - Matrices are row-major and contiguous: hidden [rows, H], W [V, H] (used transposed), logits
  *    [rows, V].
  *  - A call validates its arguments synchronously on the host and launches nothing on error; it
- *    then enqueues its kernel (two for the quantiser) on `stream` and returns without waiting. Faults surface at the
- *    caller's next synchronisation. There is no fallback path of any kind.
+ *    then enqueues its kernel (two for the log-probabilities and for the quantiser) on `stream`
+ *    and returns without waiting. Faults surface at the caller's next synchronisation. There is
+ *    no fallback path of any kind.
  *  - rows == 0 is valid and launches nothing.
  *  - Determinism: the same inputs give the same bits on every run (no atomics, no split-K). Each
  *    output element is one fp32 accumulator chain over k in ascending 16-element steps, the same
