@@ -635,7 +635,8 @@ def run_reference(args) -> dict | None:
         "metric": METRIC, "value": round(us_per_call, 1), "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "strong" if args.workload == "vocab_parallel_logprobs" else "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "parallelism": "host cores"},
         "impl": "reference",
         "cpu_baseline": {"value": round(us_per_call, 1), "unit": UNIT, "cores": cores,
