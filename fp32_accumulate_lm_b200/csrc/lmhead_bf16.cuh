@@ -7,8 +7,8 @@
 //
 // One persistent, warp-specialised tcgen05 kernel serves every row count (decode, speculative
 // verify and prefill alike), so a row's reduction order never depends on how many rows a call
-// carries ("A row's logits here do not depend on the row count", lm_head_nvfp4_rows.rs, module
-// doc -- applied here to the bf16 head as well).
+// carries. lm_head_nvfp4_rows.rs (module doc) promises this for its NVFP4 head; it is applied
+// here to the bf16 head as well.
 //
 // Orientation ("swap-AB"): W supplies the MMA's M = 128 side and the hidden rows the N side, so
 // a handful of decode rows pads N (16..256 in steps of 16), never M, and each TMEM lane holds one

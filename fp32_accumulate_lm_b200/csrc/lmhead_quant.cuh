@@ -1,7 +1,7 @@
-// NVFP4 quantiser for the W4A16 head's weights: an absmax pass, then an encode pass, as the
-// two kernels lm_head_nvfp4_rows.rs / mtp_head/new_bf16_moe.rs name ("quantize_to_nvfp4(w, n, k,
-// gpu, absmax_k, nvfp4_k, stream)"). The pages print no rules; this library's reading takes every
-// decision as one IEEE binary32 operation, so a CPU re-implementation can match it bit for bit:
+// NVFP4 quantiser for the W4A16 head's weights: an absmax pass, then an encode pass, the two
+// kernels that lm_head_nvfp4_rows.rs / mtp_head/new_bf16_moe.rs hand to `quantize_to_nvfp4`.
+// The pages print no rules; this library's reading takes every decision as one IEEE binary32
+// operation, so a CPU re-implementation can match it bit for bit:
 //   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
 //   per 16-element block:  s = RN_e4m3(bmax / (6 * g)), saturating at 448
 //   per element:           q = RN_e2m1(w / (e4m3(s) * g)), saturating at 6; the sign is kept

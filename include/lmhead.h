@@ -19,9 +19,10 @@
  *  - "FP32 LM head skip FP32 cast" (SGLang PR #32370 summary), implementation breakdown:
  *    torch.mm(hidden, W.T, out_dtype=float32) -- bf16 x bf16 -> fp32 with an fp32 accumulator,
  *    replacing a cast of both operands to fp32.
- *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head at its
- *    declared W4A16 precision, bf16 logits[rows, vocab], row-major hidden and logits, launching
- *    nothing unless the head can run, and a row's logits that do not depend on the row count.
+ *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head kept at the
+ *    W4A16 precision its checkpoint declares, bf16 logits[rows, vocab], row-major hidden and
+ *    logits, launching nothing unless the head can run, and logits of a row that are the same
+ *    whatever the number of rows in the call.
  *
  * Conventions for every entry point:
  *  - All array arguments are DEVICE pointers owned by the caller. The library keeps no reference
@@ -114,8 +115,8 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
  * avoids writing rows * V * 4 bytes of logits (5 GB at 8192 x 151936).
  * The head's epilogue reduces every 32-entry vocab chunk of a row to (max, sum of exp(z - max))
  * in fp32 and stores that pair in `workspace` (chunk-major); a second kernel folds a row's pairs
- * in a fixed order. So a row's results do not depend on the row count, and they are
- * reproducible.
+ * in a fixed order. So a row's results are the same whatever other rows the call carries, and
+ * they are reproducible.
  * Accuracy: lse and logprobs are fp32 sums of expf terms; against the exact values over the same
  * fp32 logits they are good to a few units in 1e-6 relative.
  *
@@ -199,8 +200,8 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
 /*
  * NVFP4 quantiser: bf16 W -> the three inputs of lmhead_logits_w4a16_nvfp4. The pages name a
  * two-kernel quantiser, an absmax pass then an encode pass (lm_head_nvfp4_rows.rs and
- * mtp_head/new_bf16_moe.rs, quantize_to_nvfp4(w, n, k, gpu, absmax_k, nvfp4_k, stream)), but print
- * no rules. This library's rules take every decision as one IEEE binary32 operation:
+ * mtp_head/new_bf16_moe.rs: `quantize_to_nvfp4` is handed the weight, its shape, the device, the
+ * two kernels and a stream), but print no rules. This library's rules take every decision as one IEEE binary32 operation:
  *   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
  *   w_scales[v, j]  = RN_e4m3(max_{k in block j} |w[v, k]| / (6 * g)), saturating at 448
  *   code[v, k]      = RN_e2m1(w[v, k] / (e4m3(w_scales[v, k/16]) * g)), saturating at +-6,

@@ -20,11 +20,12 @@
  *    product with an fp32 accumulator; the path's predicate admits float16 as well as bfloat16
  *    hidden states, of the same dtype as the weight.
  *  - The first page's "Purpose" lists the embedding bias among the cases the fused multiply does
- *    not cover; there the head is the projection with its bias, then the elementwise multiply by
+ *    not cover; there the head projects with its bias and then multiplies every logit by
  *    1/mup, read here as alpha * (hidden @ w.t() + bias), the bias in the weight's dtype.
- *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head at its declared
- *    W4A16 precision (16-bit activations, never cast to E4M3), bf16 logits[rows, vocab], row-major
- *    layouts (row offsets done*h*2 and done*v*2 bytes), values independent of the row count.
+ *  - lm_head_nvfp4_rows.rs, module doc and lm_head_nvfp4_rows_run: the NVFP4 head kept at the
+ *    W4A16 precision its checkpoint declares (16-bit activations, never cast to E4M3), bf16
+ *    logits[rows, vocab], row-major layouts (row offsets done*h*2 and done*v*2 bytes), values
+ *    independent of the row count.
  *
  * Readings where the pages are silent (the NVFP4 layout is not printed anywhere):
  *  - bf16 decode: the 16 bits are the top half of an IEEE binary32.
@@ -47,8 +48,8 @@
  * [0, V) gives NaN.
  *
  * NVFP4 quantiser (oracle_nvfp4_quantize). lm_head_nvfp4_rows.rs and mtp_head/new_bf16_moe.rs
- * ("quantize_to_nvfp4(w, n, k, gpu, absmax_k, nvfp4_k, stream)": an absmax kernel, then an encode
- * kernel) name it but print no rules. Reading, with every step one IEEE binary32 operation so that
+ * name it (`quantize_to_nvfp4`, handed an absmax kernel and an encode kernel) but print no
+ * rules. Reading, with every step one IEEE binary32 operation so that
  * a GPU implementation can take the same decisions bit for bit:
  *   amax = max |w| over the tensor;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
  *   per 16-element block: t = bmax / (6 * g);  s = RN_e4m3(t), saturating at 448

@@ -7,8 +7,8 @@
 Floating-point results are compared element by element within the bound in tolerance.py;
 cases where every summation order is exact (small integers, one-hot rows, zero and identity
 weights) are compared bit for bit, as are the properties the method promises exactly: the
-alpha fold equals a separate fp32 multiply, and a row's logits do not depend on the row count
-(lm_head_nvfp4_rows.rs, module doc).
+alpha fold equals a separate fp32 multiply, and a row's logits are the same whatever the number
+of rows in the call (lm_head_nvfp4_rows.rs, module doc).
 """
 import numpy as np
 import pytest
@@ -193,7 +193,7 @@ def test_decode_workload_matches_oracle(decode_inputs):
 def test_spec_verify_workload():
     """32 sequences x (1 target + 3 draft) rows = 128, ragged 97, and the 32-row draft-head call
     (rows 4s): H = 4096, V = 128256, alpha = 1/16. Shared rows must be bit-identical between
-    the target and draft calls (page 1: the MTP draft must match the target)."""
+    the target and draft calls (page 1 requires draft and target logits to agree)."""
     rows_list, H, V, std, alpha = synth.WORKLOADS["spec_verify"]
     h = synth.hidden(128, H, synth.SEED_SPEC)
     w = synth.weight(V, H, std, synth.SEED_SPEC)
