@@ -162,3 +162,23 @@ def test_through_a_one_rank_nccl_group():
         check_status()
     finally:
         dist.destroy_process_group()
+
+
+def test_rows_past_the_first_row_tile():
+    """300 rows span two 256-row tiles: every row's slice max and target logit are the slice
+    logits' bits, and the merged result agrees with the one-GPU entry."""
+    rows, H, V = 300, 256, 5000
+    _, (hd, wd, bd, td) = make(rows, H, V, 50, "bf16", True)
+    t = td.cpu().numpy()
+    stats, lp, lse = split_run(hd, wd, bd, td, 0.5, 3)
+    for i, (b0, n) in enumerate(slices(V, 3)):
+        z = lm.logits_f32(hd, wd[b0:b0 + n].contiguous(), 0.5,
+                          bias=bd[b0:b0 + n].contiguous()).cpu().numpy()
+        assert np.array_equal(stats[i, :, 0], z.max(axis=1)), i
+        held = (t >= b0) & (t < b0 + n)
+        assert np.array_equal(stats[i, held, 2], z[np.nonzero(held)[0], t[held] - b0]), i
+        assert np.isnan(stats[i, ~held, 2]).all(), i
+    lp1, lse1 = lm.logprobs_f32(hd, wd, td, 0.5, bias=bd)
+    bound = 2 * merged_bound(lse1.cpu().numpy().astype(np.float64), 1667, 3)
+    assert np.all(np.abs(lp - lp1.cpu().numpy()) <= bound)
+    assert np.all(np.abs(lse - lse1.cpu().numpy()) <= bound)
