@@ -9,6 +9,9 @@ this module only compiles it with gcc and marshals numpy arrays through ctypes. 
     fp32 head:  logits[r, v] = RN_fp32(alpha * (sum_k hidden[r, k] * W[v, k] + bias[v]))
                 (bf16 or fp16 inputs; bias optional)
     NVFP4 head: logits[r, v] = RN_bf16(alpha * sum_k hidden[r, k] * e2m1(q[v, k]) * e4m3(s[v, k/16]) * g)
+    log-probs:  logprob[r] = z[r, t_r] - log sum_v exp z[r, v] over the fp32 logits z, whole or
+                from per-slice (max, sum, target logit) stats merged in double
+    quantiser:  the NVFP4 codes, block scales and global scale of a bf16 W
 
 following "[Model] Honor fp32 head_dtype in Inkling muP logits (target + MTP draft)" ("Purpose";
 "muP is folded into the fp32 GEMM"), "FP32 LM head skip FP32 cast" (implementation breakdown) and

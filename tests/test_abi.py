@@ -223,3 +223,18 @@ def test_vocab_shard_split():
         lm.vocab_shard(3, 4, 0)
     with pytest.raises(ValueError):
         lm.vocab_shard(100, 2, 2)
+
+
+def test_vocab_parallel_wrappers_reject_bad_tensors():
+    import torch
+    h = torch.zeros(2, 64, dtype=torch.bfloat16)
+    w = torch.zeros(8, 64, dtype=torch.bfloat16)
+    t = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):                      # host tensors
+        lm.logprobs_shard_stats_f32(h, w, 0, t)
+    with pytest.raises(ValueError):                      # mixed operand dtypes
+        lm.logprobs_shard_stats_f32(h, w.half(), 0, t)
+    with pytest.raises(ValueError):                      # stats must be [g, rows, 3] fp32
+        lm.logprobs_merge_shards(torch.zeros(2, 4, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        lm.logprobs_merge_shards(torch.zeros(2, 4, 3, dtype=torch.float64))
