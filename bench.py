@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Workloads (seeded synthetic inputs from fp32_accumulate_lm_b200.synth; the pages use no dataset):
+Workloads (seeded synthetic inputs from tests/synth.py; the pages use no dataset):
   decode       (default) rows in {1,2,4,8,16,32,64}, H = 2048, V = 151936, bf16 -> fp32,
                alpha = 1/8. One step = one call per row count (7 calls).
   spec_verify  rows in {128, 97, 32}, H = 4096, V = 128256, alpha = 1/16 (3 calls per step).
@@ -38,8 +38,9 @@ import threading
 import time
 
 _ROOT = os.path.dirname(os.path.abspath(__file__))
-if _ROOT not in sys.path:
-    sys.path.insert(0, _ROOT)
+for _p in (_ROOT, os.path.join(_ROOT, "tests")):   # tests/ holds the seeded input generator
+    if _p not in sys.path:
+        sys.path.insert(0, _p)
 
 METRIC = "LM-head µs/call and achieved % of roofline (HBM GB/s decode, TFLOP/s prefill)"
 UNIT = "us/call"
@@ -172,7 +173,7 @@ class Workload:
 
     def __init__(self, name: str, device, world: int = 1, rank: int = 0):
         import torch
-        from fp32_accumulate_lm_b200 import synth
+        import synth
         self.name = name
         rows_list, H, V, std, alpha = synth.WORKLOADS[name]
         self.rows_list, self.H, self.V, self.alpha = rows_list, H, V, alpha
@@ -345,14 +346,38 @@ def job_us_per_call(elapsed_ms: float, steps: int, calls_per_step: int, world: i
     return elapsed_ms * 1e3 / (steps * calls_per_step * world)
 
 
-def run_ours(args) -> dict | None:
+# The default run measures the decode head as the headline `value`, then every other workload of
+# the library into the line's "workloads" map, each with its own roofline, e2e, clocks and CPU
+# baseline, so one run covers the whole metric (HBM-bound decode shapes, tensor-bound prefill).
+PRIMARY = "decode"
+SECONDARY = ["spec_verify", "prefill", "nvfp4", "decode_f16_bias", "prefill_logprobs",
+             "vocab_parallel_logprobs", "nvfp4_quantize"]
+# A timed region at least this long is "a long step": the sustained bf16 peak applies.
+SUSTAINED_REGION_S = 1.0
+
+
+def config_of(name: str, world: int) -> dict:
+    """The workload's description: the same keys and values in both arms of the bench."""
+    import synth
+    rows_list = synth.WORKLOADS[name][0]
+    vp = name == "vocab_parallel_logprobs"
+    return {"workload": WORKLOAD_TEXT[name],
+            "l2": "weights 2x larger than L2 per call; two weight copies alternated",
+            "parallelism": (f"vocab-parallel x{world} (all-gather of the row stats)" if vp else
+                            f"replicas x{world} (no data-path collective)"),
+            "calls_per_step": len(rows_list),
+            "rows_per_call": list(rows_list)}
+
+
+def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: float) -> dict:
+    """Warm-up, then a timed region of args.steps steps of workload `name`: per-launch CUDA events
+    on the launching stream, barrier + synchronize on both sides, max over ranks. Returns the
+    workload's record (its inputs are freed before returning)."""
     import torch
     import fp32_accumulate_lm_b200 as lm
 
-    world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
-    peaks = load_peaks()
-    wl = Workload(args.workload, dev, world, rank)
+    wl = Workload(name, dev, world, rank)
     stream = torch.cuda.current_stream()
     rl = wl.rows_list
     calls_per_step = len(rl)
@@ -362,9 +387,8 @@ def run_ours(args) -> dict | None:
             wl.call(r)
     torch.cuda.synchronize()
     if lm.device_status(clear=True) != 0:
-        raise RuntimeError("device status word set during warm-up")
+        raise RuntimeError(f"{name}: device status word set during warm-up")
 
-    # ---- timed region: K steps, per-launch events on the launching stream
     n_ev = args.steps * calls_per_step
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
     sampler = ClockSampler(torch.cuda.current_device())
@@ -381,7 +405,7 @@ def run_ours(args) -> dict | None:
     clocks = sampler.stop()
     barrier(world)
     if lm.device_status(clear=True) != 0:
-        raise RuntimeError("device status word set during the timed region")
+        raise RuntimeError(f"{name}: device status word set during the timed region")
     elapsed_ms = ev[0].elapsed_time(ev[n_ev])
     per_call_ms = [ev[j].elapsed_time(ev[j + 1]) for j in range(n_ev)]
     elapsed_ms = max_over_ranks(elapsed_ms, world)
@@ -400,13 +424,15 @@ def run_ours(args) -> dict | None:
         tot_flops += fl
         tot_ms += mean_ms
     # prefill, its profiling case, log-probs, vocab-parallel log-probs
-    tensor_bound = args.workload.startswith("prefill") or wl.vocab_parallel
+    tensor_bound = name.startswith("prefill") or wl.vocab_parallel
     if tensor_bound:
         achieved = tot_flops / (tot_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        long_region = elapsed_ms >= SUSTAINED_REGION_S * 1e3
+        peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),
-                "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
+                "peak_kind": ("bf16 dense, sustained" if long_region else "bf16 dense, burst") +
+                             f" ({peaks['source']}; timed region {elapsed_ms / 1e3:.2f} s)"}
     else:
         achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
@@ -414,38 +440,61 @@ def run_ours(args) -> dict | None:
                 "frac": round(achieved / peak, 4), "peak_kind": f"HBM copy ({peaks['source']})"}
     roof["kernel"] = ("nvfp4_encode_kernel + nvfp4_absmax_kernel" if wl.quantize else
                       "lmhead_w4a16_nvfp4_kernel" if wl.nvfp4 else "lmhead_bf16_f32_kernel")
-    roof["traffic"] = recorded_traffic(roof["kernel"], args.workload)
+    roof["traffic"] = recorded_traffic(roof["kernel"], name)
     roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
     roof["source_hash"] = kernel_source_hash()
 
-    # ---- end to end through the C ABI: pinned host hidden -> device, call, logits -> pinned host
+    # end to end through the C ABI: pinned host hidden -> device, call, outputs -> pinned host
     e2e = run_e2e(args, wl, world)
 
     # Replicas: every rank makes whole calls. Vocab-parallel: the ranks make each call together.
     value = job_us_per_call(elapsed_ms, args.steps, calls_per_step,
                             1 if wl.vocab_parallel else world)
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": False,
-        "scaling": "strong" if wl.vocab_parallel else "weak", "vs_baseline": None,
+    rec = {
+        "value": round(value, 3), "unit": UNIT, "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "scaling": "strong" if wl.vocab_parallel else "weak",
         "dtype": ("f32" if wl.quantize else "e2m1xbf16" if wl.nvfp4 else
                   "f16" if wl.dtype == torch.float16 else "bf16"),
-        "data": "synthetic (seeded N(0,1) hidden, N(0,std) weights; no dataset on the pages)",
-        "config": {"workload": WORKLOAD_TEXT[args.workload],
-                   "l2": "weights 2x larger than L2 per call; two weight copies alternated",
-                   "parallelism": (f"vocab-parallel x{world} (all-gather of the row stats)"
-                                   if wl.vocab_parallel else
-                                   f"replicas x{world} (no data-path collective)"),
-                   "calls_per_step": calls_per_step, "per_rows": detail},
+        "config": config_of(name, world),
+        "per_rows": detail,
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": n_ev * (3 if wl.vocab_parallel else
                                 2 if (wl.quantize or wl.logprobs) else 1),
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, wl)
+    if rank == 0 and world == 1 and cpu_budget_s > 0:
+        rec["cpu_baseline"] = cpu_baseline(name, wl, cpu_budget_s)
+    del wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args) -> dict | None:
+    world, rank, local = dist_setup(args.gpus)
+    peaks = load_peaks()
+    budget = 0.0 if args.no_cpu_baseline else 10.0
+    main = measure(args.workload, args, world, rank, peaks, budget)
+    line = {
+        "metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+        "higher_is_better": False, "scaling": main["scaling"], "vs_baseline": None,
+        "dtype": main["dtype"],
+        "data": "synthetic (seeded N(0,1) hidden, N(0,std) weights; no dataset on the pages)",
+        "config": main["config"],
+        "per_rows": main["per_rows"],
+        "roofline": main["roofline"],
+        "e2e": main["e2e"],
+        "gpu_launches": main["gpu_launches"],
+        "clocks": main["clocks"],
+    }
+    if "cpu_baseline" in main:
+        line["cpu_baseline"] = main["cpu_baseline"]
+    if args.workload == PRIMARY and not args.only:
+        # every rank runs the same workloads in the same order (vocab-parallel has a collective)
+        line["workloads"] = {name: measure(name, args, world, rank, peaks, budget / 2)
+                             for name in SECONDARY}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -487,157 +536,139 @@ def run_e2e(args, wl, world: int) -> dict:
 
 
 # ---------------------------------------------------------------- CPU oracle (baseline arm)
+#
+# Both CPU legs -- the repo arm's cpu_baseline and the reference arm -- time the oracle the same
+# way: the step's first n distinct hidden rows (n <= 64) against the first `vslice` rows of W,
+# scaled by V / vslice and by the step's total rows / n, per call. The oracle decodes W once per
+# call, so timing the distinct rows together amortises that decode as a real call would.
 
-_SAMPLES: dict = {}
-
-
-def _oracle_sample(workload: str, rows: int, vocab_slice: int, wl=None):
-    """Time the oracle on `rows` rows against the first `vocab_slice` weight rows; returns
-    (seconds, multiply-adds done). Inputs are generated once and reused; only the oracle call is
-    timed."""
-    import oracle
-    from fp32_accumulate_lm_b200 import synth
-    rows_list, H, V, std, alpha = synth.WORKLOADS[workload]
-    key = (workload, rows, vocab_slice)
-    f16 = workload == "decode_f16_bias"
-    if key not in _SAMPLES:
-        import torch
-        dt = torch.float16 if f16 else torch.bfloat16
-        h = synth.hidden(rows, H, 7, dtype=dt)
-        if workload == "nvfp4":
-            _SAMPLES[key] = (h, synth.nvfp4_weights(vocab_slice, H, std, 7))
-        else:
-            _SAMPLES[key] = (h, (synth.weight(vocab_slice, H, std, 7, dtype=dt),
-                                 synth.bias(vocab_slice, 7, dtype=dt) if f16 else None))
-    h, w = _SAMPLES[key]
-    t0 = time.perf_counter()
-    if workload == "nvfp4":
-        packed, scales, g = w
-        oracle.logits_w4a16_nvfp4(h, packed, scales, g, alpha)
-    else:
-        oracle.logits_f32(h, w[0], alpha, bias_bits=w[1], dtype="f16" if f16 else "bf16")
-    return time.perf_counter() - t0, rows * vocab_slice * H
+ORACLE_MAX_ROWS = 64
 
 
-def cpu_baseline(workload: str, wl) -> dict:
-    """The oracle on the host cores, on the bench's own inputs: as many of the step's rows as fit
-    in about 10 s (all of them for the decode workload), against the full vocabulary, scaled by
-    rows to the step and reported per call."""
+def _oracle_inputs(name: str, n_rows: int, vslice: int, wl=None) -> dict:
+    """numpy inputs for the oracle: hidden rows [n_rows, H] and the first vslice rows of the
+    weights (NVFP4 codes and scales for the NVFP4 head), from the GPU workload's own tensors
+    when `wl` is given, else regenerated on the host with the workload's seeds."""
     import numpy as np
-    import oracle
     import torch
-    cores = oracle.default_threads()
-    H, V = wl.H, wl.V
-    if wl.quantize:  # the oracle quantiser is single-threaded: time a slice of W's rows
-        w = wl.weights[0].view(torch.int16).cpu().numpy().view(np.uint16)
-        n = 4096
-        t0 = time.perf_counter()
-        oracle.nvfp4_quantize(w[:n])
-        secs = time.perf_counter() - t0
-        return {"value": round(1e6 * secs * V / n, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
-                "sample": f"{n} of W's {V} rows x H={H} ({secs:.1f} s), scaled by rows"}
-    rows_in_step = sum(wl.rows_list)
-    h_all = wl.hidden.view(torch.int16).cpu().numpy().view(np.uint16)
-    if wl.nvfp4:
-        packed = wl.weights[0][0].cpu().numpy()
-        scales = wl.weights[0][1].cpu().numpy()
-
-        def run(h, vrows):
-            oracle.logits_w4a16_nvfp4(h, packed[:vrows], scales[:vrows], wl.g, wl.alpha)
-    else:
-        w = wl.weights[0].view(torch.int16).cpu().numpy().view(np.uint16)
-        b = None if wl.bias is None else wl.bias.view(torch.int16).cpu().numpy().view(np.uint16)
-        dt = "f16" if wl.dtype == torch.float16 else "bf16"
-
-        tg = wl.targets.cpu().numpy() if wl.logprobs else None
-
-        def run(h, vrows):
-            if wl.logprobs:
-                oracle.logprobs_f32(h, w[:vrows], wl.alpha, np.minimum(tg[:h.shape[0]], vrows - 1),
-                                    dtype=dt)
-            else:
-                oracle.logits_f32(h, w[:vrows], wl.alpha,
-                                  bias_bits=None if b is None else b[:vrows], dtype=dt)
-    probe_v = min(V, 4096)
-    t0 = time.perf_counter()
-    run(h_all[:1], probe_v)
-    t_row = (time.perf_counter() - t0) * V / probe_v
-    n_rows = int(max(1, min(rows_in_step, h_all.shape[0], 10.0 / max(t_row, 1e-9))))
-    t0 = time.perf_counter()
-    run(h_all[:n_rows], V)
-    secs = time.perf_counter() - t0
-    us_per_call = 1e6 * secs * (rows_in_step / n_rows) / len(wl.rows_list)
-    return {"value": round(us_per_call, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n_rows} of the step's {rows_in_step} rows x full V={V} x H={H} "
-                      f"({secs:.1f} s), scaled by rows to the step, per call"}
+    import synth
+    rows_list, H, V, std, alpha = synth.WORKLOADS[name]
+    seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
+            "nvfp4": synth.SEED_NVFP4, "decode_f16_bias": synth.SEED_F16,
+            "nvfp4_quantize": synth.SEED_NVFP4}.get(name, synth.SEED_PREFILL)
+    f16 = name == "decode_f16_bias"
+    dt = torch.float16 if f16 else torch.bfloat16
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    d = {"name": name, "H": H, "V": V, "alpha": alpha, "f16": f16}
+    if name == "nvfp4_quantize":
+        d["w"] = (bits(wl.weights[0][:vslice]) if wl is not None
+                  else synth.weight(vslice, H, std, seed, dtype=dt))
+        return d
+    d["h"] = (bits(wl.hidden[:n_rows]) if wl is not None
+              else synth.hidden(n_rows, H, seed, dtype=dt))
+    if name == "nvfp4":
+        if wl is not None:
+            d["packed"] = wl.weights[0][0][:vslice].cpu().numpy()
+            d["scales"] = wl.weights[0][1][:vslice].cpu().numpy()
+            d["g"] = wl.g
+        else:
+            d["packed"], d["scales"] = synth.random_nvfp4_codes(vslice, H, seed)
+            d["g"] = 1.0 / 4096
+        return d
+    d["w"] = bits(wl.weights[0][:vslice]) if wl is not None else synth.weight(vslice, H, std,
+                                                                               seed, dtype=dt)
+    d["b"] = ((bits(wl.bias[:vslice]) if wl is not None else synth.bias(vslice, synth.SEED_BIAS,
+                                                                        dtype=dt))
+              if f16 else None)
+    if name in ("prefill_logprobs", "vocab_parallel_logprobs"):
+        gen = torch.Generator(device="cpu")
+        gen.manual_seed(seed + 700_000)
+        d["t"] = torch.randint(0, vslice, (n_rows,), generator=gen, dtype=torch.int32).numpy()
+    return d
 
 
-def _reference_quantize(args, H: int, V: int) -> dict:
-    """The oracle quantiser as the reference arm: each step quantises a slice of W's rows, scaled
-    by rows to one call."""
+def _oracle_run(d: dict) -> float:
+    """Seconds of one oracle call on the prepared inputs."""
     import oracle
-    from fp32_accumulate_lm_b200 import synth
-    n = 2048
-    w = synth.weight(n, H, 0.02, 7)
-    for _ in range(args.warmup):
-        oracle.nvfp4_quantize(w)
-    times = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle.nvfp4_quantize(w)
-        times.append(time.perf_counter() - t0)
-    total = sum(times)
-    us = 1e6 * total / args.steps * V / n
-    sample = f"per step: {n} of W's {V} rows x H={H}, scaled by rows to one call"
-    return {
-        "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "parallelism": "host core"},
-        "impl": "reference",
-        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
-        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
+    t0 = time.perf_counter()
+    if d["name"] == "nvfp4_quantize":
+        oracle.nvfp4_quantize(d["w"])
+    elif d["name"] == "nvfp4":
+        oracle.logits_w4a16_nvfp4(d["h"], d["packed"], d["scales"], d["g"], d["alpha"])
+    elif "t" in d:
+        oracle.logprobs_f32(d["h"], d["w"], d["alpha"], d["t"])
+    else:
+        oracle.logits_f32(d["h"], d["w"], d["alpha"], bias_bits=d["b"],
+                          dtype="f16" if d["f16"] else "bf16")
+    return time.perf_counter() - t0
+
+
+def _oracle_plan(name: str, budget_s: float, wl=None):
+    """(n_rows, vslice, per-call scale) for oracle calls of about budget_s seconds each: the
+    step's distinct rows (at most 64), and as much of the vocabulary as the budget allows."""
+    import synth
+    rows_list, H, V, _, _ = synth.WORKLOADS[name]
+    if name == "nvfp4_quantize":
+        probe = 1024
+        t = _oracle_run(_oracle_inputs(name, 0, probe, wl))
+        vslice = int(max(probe, min(V, probe * budget_s / max(t, 1e-6))))
+        return 0, vslice, V / vslice
+    n_rows = min(max(rows_list), ORACLE_MAX_ROWS)
+    probe = min(V, 2048)
+    t = _oracle_run(_oracle_inputs(name, n_rows, probe, wl))
+    vslice = int(max(probe, min(V, probe * budget_s / max(t, 1e-6))))
+    scale = (V / vslice) * (sum(rows_list) / n_rows) / len(rows_list)
+    return n_rows, vslice, scale
+
+
+def _oracle_sample_text(name: str, n_rows: int, vslice: int, secs: float) -> str:
+    import synth
+    rows_list, H, V, _, _ = synth.WORKLOADS[name]
+    if name == "nvfp4_quantize":
+        return (f"{vslice} of W's {V} rows x H={H} ({secs:.1f} s per sample), scaled by rows to "
+                "one call")
+    return (f"the step's first {n_rows} distinct rows (of {sum(rows_list)} rows in "
+            f"{len(rows_list)} calls) x {vslice} of V={V} vocab rows x H={H} ({secs:.1f} s per "
+            "sample), scaled by V and by rows, per call")
+
+
+def cpu_baseline(name: str, wl, budget_s: float = 10.0) -> dict:
+    """The oracle as it stands, on the host cores, on the bench's own inputs (rank 0, N = 1)."""
+    import oracle
+    n_rows, vslice, scale = _oracle_plan(name, budget_s, wl)
+    d = _oracle_inputs(name, n_rows, vslice, wl)
+    secs = _oracle_run(d)
+    cores = 1 if name == "nvfp4_quantize" else oracle.default_threads()
+    return {"value": round(1e6 * secs * scale, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": _oracle_sample_text(name, n_rows, vslice, secs)}
 
 
 def run_reference(args) -> dict | None:
+    """The reference arm: the CPU oracle (this build has no installable reference; the pages hold
+    no code) timed as cpu_baseline times it, each step one bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
     if rank != 0:
         return None
     import oracle
-    from fp32_accumulate_lm_b200 import synth
-    rows_list, H, V, std, alpha = synth.WORKLOADS[args.workload]
-    cores = oracle.default_threads()
-    if args.workload == "nvfp4_quantize":
-        return _reference_quantize(args, H, V)
-    mean_macs_per_call = sum(r * H * V for r in rows_list) / len(rows_list)
-    # bounded per-step sample sized so warm-up + steps stay near a minute of CPU time
-    vslice = 256
-    t_probe, m_probe = _oracle_sample(args.workload, 1, vslice)
-    budget_s = 60.0
-    per_step_s = budget_s / max(1, args.steps + args.warmup)
-    vslice = int(max(128, min(V, vslice * per_step_s / max(t_probe, 1e-6))))
+    name = args.workload
+    per_step_s = min(10.0, 90.0 / max(1, args.steps + args.warmup))
+    n_rows, vslice, scale = _oracle_plan(name, per_step_s)
+    d = _oracle_inputs(name, n_rows, vslice)
     for _ in range(args.warmup):
-        _oracle_sample(args.workload, 1, vslice)
-    times = []
-    macs = 0
-    for _ in range(args.steps):
-        s, m = _oracle_sample(args.workload, 1, vslice)
-        times.append(s)
-        macs = m
+        _oracle_run(d)
+    times = [_oracle_run(d) for _ in range(args.steps)]
     total = sum(times)
-    us_per_call = 1e6 * (total / (args.steps * macs)) * mean_macs_per_call
-    sample = f"per step: 1 row x {vslice} vocab rows x H={H}, scaled by multiply-adds to the mean call"
+    us_per_call = 1e6 * (total / args.steps) * scale
+    cores = 1 if name == "nvfp4_quantize" else oracle.default_threads()
+    sample = "per step: " + _oracle_sample_text(name, n_rows, vslice, total / args.steps)
     return {
         "metric": METRIC, "value": round(us_per_call, 1), "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": False,
-        "scaling": "strong" if args.workload == "vocab_parallel_logprobs" else "weak",
+        "scaling": "strong" if name == "vocab_parallel_logprobs" else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "parallelism": "host cores"},
+        "config": config_of(name, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(us_per_call, 1), "unit": UNIT, "cores": cores,
                          "kind": "oracle", "sample": sample},
@@ -654,6 +685,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true",
+                    help="measure only --workload (the default run adds every other workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -10,9 +10,18 @@ logits (lm_head_nvfp4_rows.rs, lm_head_nvfp4_rows_run).
 This module only marshals arguments: every step of the computation runs in the CUDA library
 ``liblmhead.so`` built in-tree by ``fp32_accumulate_lm_b200._build``. If that library is
 missing or fails to load, every call raises; there is no other code path.
+
+Calls are asynchronous. A kernel that gives up on one of its bounded waits records a timeout in
+a per-device status word instead of faulting; pass ``check=True`` to a wrapper (or call
+``check(stream)``) to synchronise and raise ``LmheadError`` if that happened.
+
+``test_hooks()`` routes every call to ``liblmhead_test.so`` (the same kernels plus two
+host-side test knobs, see ``set_fault_injection`` and ``set_nvfp4_conversion``); only the tests
+use it.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -26,7 +35,8 @@ __all__ = [
     "lmhead_logits_w4a16_nvfp4", "lmhead_nvfp4_quantize", "lmhead_nvfp4_quantize_noalloc",
     "nvfp4_quantize",
     "nvfp4_quantize_workspace_bytes", "status_string", "device_status", "DTYPE_BF16", "DTYPE_F16",
-    "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS",
+    "version", "set_fault_injection", "set_nvfp4_conversion", "STATUS", "lmhead_stream_status",
+    "stream_status", "check", "test_hooks", "load_test_library",
 ]
 
 STATUS = {
@@ -40,8 +50,11 @@ DTYPE_F16 = 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liblmhead.so")
+_TEST_LIB_PATH = os.path.join(_HERE, "liblmhead_test.so")
 _lock = threading.Lock()
 _lib = None
+_test_lib = None
+_use_test = False
 
 
 class LmheadError(RuntimeError):
@@ -54,6 +67,46 @@ def library_path() -> str:
     return _LIB_PATH
 
 
+def _bind(lib, test: bool):
+    vp, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+    lib.lmhead_logits_bf16_f32.argtypes = [vp, i64, i64, vp, i64, f32, vp, vp]
+    lib.lmhead_logits_bf16_f32.restype = i32
+    lib.lmhead_logits_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp]
+    lib.lmhead_logits_f32.restype = i32
+    lib.lmhead_logprobs_workspace_bytes.argtypes = [i64, i64]
+    lib.lmhead_logprobs_workspace_bytes.restype = ctypes.c_size_t
+    lib.lmhead_logprobs_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
+    lib.lmhead_logprobs_f32.restype = i32
+    lib.lmhead_logprobs_shard_stats_f32.argtypes = [vp, i32, i64, i64, vp, i64, i64, f32, vp,
+                                                    vp, vp, vp, ctypes.c_size_t, vp]
+    lib.lmhead_logprobs_shard_stats_f32.restype = i32
+    lib.lmhead_logprobs_merge_shards.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.lmhead_logprobs_merge_shards.restype = i32
+    lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
+    lib.lmhead_logits_w4a16_nvfp4.restype = i32
+    lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
+    lib.lmhead_nvfp4_quantize_workspace_bytes.restype = ctypes.c_size_t
+    lib.lmhead_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.lmhead_nvfp4_quantize.restype = i32
+    lib.lmhead_nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+    lib.lmhead_nvfp4_quantize_noalloc.restype = i32
+    lib.lmhead_status_string.argtypes = [i32]
+    lib.lmhead_status_string.restype = ctypes.c_char_p
+    lib.lmhead_device_status.argtypes = [i32]
+    lib.lmhead_device_status.restype = i32
+    lib.lmhead_stream_status.argtypes = [vp]
+    lib.lmhead_stream_status.restype = i32
+    lib.lmhead_version.argtypes = []
+    lib.lmhead_version.restype = i32
+    if test:
+        lib.lmhead_debug_set_fault_injection.argtypes = [i32, ctypes.c_uint64]
+        lib.lmhead_debug_set_fault_injection.restype = None
+        lib.lmhead_debug_set_nvfp4_conversion.argtypes = [i32]
+        lib.lmhead_debug_set_nvfp4_conversion.restype = None
+    return lib
+
+
 def load_library():
     """Load liblmhead.so (raises if it has not been built)."""
     global _lib
@@ -63,67 +116,64 @@ def load_library():
         if not os.path.exists(_LIB_PATH):
             raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
                                "`python -m fp32_accumulate_lm_b200._build`")
-        lib = ctypes.CDLL(_LIB_PATH)
-        vp, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
-        lib.lmhead_logits_bf16_f32.argtypes = [vp, i64, i64, vp, i64, f32, vp, vp]
-        lib.lmhead_logits_bf16_f32.restype = i32
-        lib.lmhead_logits_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp]
-        lib.lmhead_logits_f32.restype = i32
-        lib.lmhead_logprobs_workspace_bytes.argtypes = [i64, i64]
-        lib.lmhead_logprobs_workspace_bytes.restype = ctypes.c_size_t
-        lib.lmhead_logprobs_f32.argtypes = [vp, i32, i64, i64, vp, i64, f32, vp, vp, vp, vp, vp,
-                                            ctypes.c_size_t, vp]
-        lib.lmhead_logprobs_f32.restype = i32
-        lib.lmhead_logprobs_shard_stats_f32.argtypes = [vp, i32, i64, i64, vp, i64, i64, f32, vp,
-                                                        vp, vp, vp, ctypes.c_size_t, vp]
-        lib.lmhead_logprobs_shard_stats_f32.restype = i32
-        lib.lmhead_logprobs_merge_shards.argtypes = [vp, i64, i64, vp, vp, vp]
-        lib.lmhead_logprobs_merge_shards.restype = i32
-        lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
-        lib.lmhead_logits_w4a16_nvfp4.restype = i32
-        lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
-        lib.lmhead_nvfp4_quantize_workspace_bytes.restype = ctypes.c_size_t
-        lib.lmhead_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
-        lib.lmhead_nvfp4_quantize.restype = i32
-        lib.lmhead_nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
-        lib.lmhead_nvfp4_quantize_noalloc.restype = i32
-        lib.lmhead_status_string.argtypes = [i32]
-        lib.lmhead_status_string.restype = ctypes.c_char_p
-        lib.lmhead_device_status.argtypes = [i32]
-        lib.lmhead_device_status.restype = i32
-        lib.lmhead_version.argtypes = []
-        lib.lmhead_version.restype = i32
-        lib.lmhead_debug_set_fault_injection.argtypes = [i32, ctypes.c_uint64]
-        lib.lmhead_debug_set_fault_injection.restype = None
-        lib.lmhead_debug_set_nvfp4_conversion.argtypes = [i32]
-        lib.lmhead_debug_set_nvfp4_conversion.restype = None
-        _lib = lib
-        return lib
+        _lib = _bind(ctypes.CDLL(_LIB_PATH), test=False)
+        return _lib
+
+
+def load_test_library():
+    """Load liblmhead_test.so, the test build (raises if it has not been built)."""
+    global _test_lib
+    with _lock:
+        if _test_lib is not None:
+            return _test_lib
+        if not os.path.exists(_TEST_LIB_PATH):
+            raise RuntimeError(f"{_TEST_LIB_PATH} is missing: build it with "
+                               "`python -m fp32_accumulate_lm_b200._build`")
+        _test_lib = _bind(ctypes.CDLL(_TEST_LIB_PATH), test=True)
+        return _test_lib
+
+
+def _active():
+    return load_test_library() if _use_test else load_library()
+
+
+@contextlib.contextmanager
+def test_hooks():
+    """Route every call of this module to the test build for the duration (tests only). The test
+    build has its own per-device status word; read it inside the block."""
+    global _use_test
+    load_test_library()
+    prev = _use_test
+    _use_test = True
+    try:
+        yield load_test_library()
+    finally:
+        _use_test = prev
 
 
 # ---------------------------------------------------------------- raw C-ABI (integers in, status out)
 
 def lmhead_logits_bf16_f32(hidden_ptr: int, rows: int, H: int, w_ptr: int, V: int, alpha: float,
                            logits_ptr: int, stream: int = 0) -> int:
-    return load_library().lmhead_logits_bf16_f32(hidden_ptr, rows, H, w_ptr, V, alpha,
+    return _active().lmhead_logits_bf16_f32(hidden_ptr, rows, H, w_ptr, V, alpha,
                                                   logits_ptr, stream)
 
 
 def lmhead_logits_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: int, V: int,
                       alpha: float, bias_ptr: int, logits_ptr: int, stream: int = 0) -> int:
-    return load_library().lmhead_logits_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
+    return _active().lmhead_logits_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
                                              bias_ptr or None, logits_ptr, stream)
 
 
 def logprobs_workspace_bytes(rows: int, V: int) -> int:
-    return int(load_library().lmhead_logprobs_workspace_bytes(rows, V))
+    return int(_active().lmhead_logprobs_workspace_bytes(rows, V))
 
 
 def lmhead_logprobs_f32(hidden_ptr: int, dtype: int, rows: int, H: int, w_ptr: int, V: int,
                         alpha: float, bias_ptr: int, targets_ptr: int, logprobs_ptr: int,
                         lse_ptr: int, workspace_ptr: int, workspace_bytes: int,
                         stream: int = 0) -> int:
-    return load_library().lmhead_logprobs_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
+    return _active().lmhead_logprobs_f32(hidden_ptr, dtype, rows, H, w_ptr, V, alpha,
                                                bias_ptr or None, targets_ptr, logprobs_ptr,
                                                lse_ptr or None, workspace_ptr, workspace_bytes,
                                                stream)
@@ -134,32 +184,32 @@ def lmhead_logprobs_shard_stats_f32(hidden_ptr: int, dtype: int, rows: int, H: i
                                     bias_shard_ptr: int, targets_ptr: int, stats_ptr: int,
                                     workspace_ptr: int, workspace_bytes: int,
                                     stream: int = 0) -> int:
-    return load_library().lmhead_logprobs_shard_stats_f32(
+    return _active().lmhead_logprobs_shard_stats_f32(
         hidden_ptr, dtype, rows, H, w_shard_ptr, V_shard, v_begin, alpha, bias_shard_ptr or None,
         targets_ptr, stats_ptr, workspace_ptr, workspace_bytes, stream)
 
 
 def lmhead_logprobs_merge_shards(stats_ptr: int, shards: int, rows: int, logprobs_ptr: int,
                                  lse_ptr: int, stream: int = 0) -> int:
-    return load_library().lmhead_logprobs_merge_shards(stats_ptr, shards, rows, logprobs_ptr,
+    return _active().lmhead_logprobs_merge_shards(stats_ptr, shards, rows, logprobs_ptr,
                                                        lse_ptr or None, stream)
 
 
 def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
                               scales_ptr: int, w_global_scale: float, V: int, alpha: float,
                               logits_ptr: int, stream: int = 0) -> int:
-    return load_library().lmhead_logits_w4a16_nvfp4(hidden_ptr, rows, H, packed_ptr, scales_ptr,
+    return _active().lmhead_logits_w4a16_nvfp4(hidden_ptr, rows, H, packed_ptr, scales_ptr,
                                                      w_global_scale, V, alpha, logits_ptr, stream)
 
 
 def nvfp4_quantize_workspace_bytes() -> int:
-    return int(load_library().lmhead_nvfp4_quantize_workspace_bytes())
+    return int(_active().lmhead_nvfp4_quantize_workspace_bytes())
 
 
 def lmhead_nvfp4_quantize(w_ptr: int, V: int, H: int, packed_ptr: int, scales_ptr: int,
                           g_ptr: int, workspace_ptr: int, workspace_bytes: int,
                           stream: int = 0) -> int:
-    return load_library().lmhead_nvfp4_quantize(w_ptr, V, H, packed_ptr, scales_ptr, g_ptr,
+    return _active().lmhead_nvfp4_quantize(w_ptr, V, H, packed_ptr, scales_ptr, g_ptr,
                                                 workspace_ptr, workspace_bytes, stream)
 
 
@@ -167,11 +217,11 @@ def lmhead_nvfp4_quantize_noalloc(w_ptr: int, V: int, H: int, packed_ptr: int, s
                                   g_ptr: int, stream: int = 0) -> int:
     """The quantiser for callers that cannot allocate device memory: the library's own 4 KB
     per-GPU scratch replaces the workspace (see include/lmhead.h)."""
-    return load_library().lmhead_nvfp4_quantize_noalloc(w_ptr, V, H, packed_ptr, scales_ptr,
+    return _active().lmhead_nvfp4_quantize_noalloc(w_ptr, V, H, packed_ptr, scales_ptr,
                                                         g_ptr, stream)
 
 
-def nvfp4_quantize(W, workspace=None, out=None, stream=None):
+def nvfp4_quantize(W, workspace=None, out=None, stream=None, check: bool = False):
     """Quantise a bf16 CUDA tensor W [V, H] (H % 16 == 0) for the NVFP4 head. Returns (packed uint8
     [V, H/2], scales uint8 [V, H/16], g: fp32 CUDA tensor of one element), all on W's device;
     runs asynchronously on ``stream``. ``workspace`` (a CUDA tensor of at least
@@ -187,44 +237,74 @@ def nvfp4_quantize(W, workspace=None, out=None, stream=None):
         g = torch.empty((1,), dtype=torch.float32, device=W.device)
     else:
         packed, scales, g = out
-        _check(packed.dtype == torch.uint8 and tuple(packed.shape) == (V, H // 2) and
-               scales.dtype == torch.uint8 and tuple(scales.shape) == (V, H // 16) and
-               g.dtype == torch.float32 and g.numel() == 1, "out = (packed, scales, g) mismatch")
+        _check_out(packed, torch.uint8, (V, H // 2), W.device, "out[0] (packed codes)")
+        _check_out(scales, torch.uint8, (V, H // 16), W.device, "out[1] (block scales)")
+        _check_out(g, torch.float32, (1,), W.device, "out[2] (global scale)")
     need = nvfp4_quantize_workspace_bytes()
     if workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=W.device)
+    _check(workspace.is_cuda and workspace.is_contiguous() and workspace.device == W.device,
+           "workspace must be a contiguous CUDA tensor on W's device")
     nbytes = workspace.numel() * workspace.element_size()
     st = lmhead_nvfp4_quantize(W.data_ptr(), V, H, packed.data_ptr(), scales.data_ptr(),
                                g.data_ptr(), workspace.data_ptr(), nbytes, _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_nvfp4_quantize")
+    _finish(st, "lmhead_nvfp4_quantize", check, stream)
     return packed, scales, g
 
 
 def status_string(status: int) -> str:
     try:
-        return load_library().lmhead_status_string(int(status)).decode()
+        return _active().lmhead_status_string(int(status)).decode()
     except RuntimeError:
         return STATUS.get(status, "unknown status")
 
 
 def device_status(clear: bool = False) -> int:
-    """Status word of the current device (0, or LMHEAD_ERR_TIMEOUT | role << 8)."""
-    return load_library().lmhead_device_status(1 if clear else 0)
+    """Status word of the current device (0, or LMHEAD_ERR_TIMEOUT | role << 8). Does not
+    synchronise: read it after the work of interest has finished."""
+    return _active().lmhead_device_status(1 if clear else 0)
+
+
+def lmhead_stream_status(stream: int = 0) -> int:
+    return _active().lmhead_stream_status(stream)
+
+
+def stream_status(stream=None) -> int:
+    """Synchronise ``stream`` (default: torch's current stream), then return and clear the
+    device's status word (0 when no kernel wait ran out)."""
+    return lmhead_stream_status(_stream_handle(stream))
+
+
+def check(stream=None) -> None:
+    """Synchronise ``stream`` and raise LmheadError if a kernel of this device gave up on one of
+    its waits since the last check (its outputs are undefined) or the stream reported an error."""
+    st = stream_status(stream)
+    if st != LMHEAD_OK:
+        raise LmheadError(st & 0xFF, f"kernel status word {st:#x} (role {(st >> 8) & 0xFF})")
 
 
 def version() -> int:
-    return load_library().lmhead_version()
+    return _active().lmhead_version()
 
 
 def set_nvfp4_conversion(path: int) -> None:
-    """Test hook: 1 pair table, 2 integer spreading, 0 automatic (same bits either way)."""
-    load_library().lmhead_debug_set_nvfp4_conversion(int(path))
+    """Test build only (inside ``test_hooks()``): 1 pair table, 2 integer spreading, 0 automatic
+    (the same bits either way)."""
+    _require_test_build("set_nvfp4_conversion")
+    _active().lmhead_debug_set_nvfp4_conversion(int(path))
 
 
 def set_fault_injection(starve_loads: bool, wait_limit_ns: int = 0) -> None:
-    """Test-only: make launches issue no loads so their waits time out after wait_limit_ns."""
-    load_library().lmhead_debug_set_fault_injection(1 if starve_loads else 0, int(wait_limit_ns))
+    """Test build only (inside ``test_hooks()``): make launches issue no loads, so their waits
+    time out after wait_limit_ns."""
+    _require_test_build("set_fault_injection")
+    _active().lmhead_debug_set_fault_injection(1 if starve_loads else 0, int(wait_limit_ns))
+
+
+def _require_test_build(what: str):
+    if not _use_test:
+        raise RuntimeError(f"{what} exists only in the test build: call it inside "
+                           "fp32_accumulate_lm_b200.test_hooks()")
 
 
 # ---------------------------------------------------------------- torch-tensor convenience wrappers
@@ -243,9 +323,25 @@ def _check(cond: bool, msg: str):
         raise ValueError(msg)
 
 
-def logits_bf16_f32(hidden, W, alpha: float = 1.0, out=None, stream=None):
+def _check_out(t, dtype, shape, device, what: str):
+    """A caller-supplied output must be a contiguous CUDA tensor of this dtype and shape on the
+    inputs' device: the kernels write exactly that many elements and check nothing."""
+    _check(t is not None and t.dtype == dtype and t.is_cuda and t.is_contiguous()
+           and tuple(t.shape) == tuple(shape) and t.device == device,
+           f"{what} must be a contiguous {dtype} CUDA tensor of shape {tuple(shape)} on {device}")
+
+
+def _finish(st: int, what: str, check_after: bool, stream):
+    if st != LMHEAD_OK:
+        raise LmheadError(st, what)
+    if check_after:
+        check(stream)
+
+
+def logits_bf16_f32(hidden, W, alpha: float = 1.0, out=None, stream=None, check: bool = False):
     """fp32 logits[rows, V] = alpha * hidden @ W^T for bf16 CUDA tensors hidden [rows, H] and
-    W [V, H]. Runs asynchronously on ``stream`` (default: torch's current stream)."""
+    W [V, H]. Runs asynchronously on ``stream`` (default: torch's current stream); with
+    ``check`` it synchronises and raises if a kernel wait timed out."""
     import torch
     _check(hidden.dtype == torch.bfloat16 and W.dtype == torch.bfloat16, "bf16 operands required")
     _check(hidden.dim() == 2 and W.dim() == 2 and hidden.shape[1] == W.shape[1], "shape mismatch")
@@ -255,16 +351,16 @@ def logits_bf16_f32(hidden, W, alpha: float = 1.0, out=None, stream=None):
     V = W.shape[0]
     if out is None:
         out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
-    _check(out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (rows, V),
-           "out must be a contiguous fp32 [rows, V] tensor")
+    _check_out(out, torch.float32, (rows, V), hidden.device, "out")
+    _check(W.device == hidden.device, "hidden and W must be on one device")
     st = lmhead_logits_bf16_f32(hidden.data_ptr(), rows, H, W.data_ptr(), V, float(alpha),
                                 out.data_ptr(), _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logits_bf16_f32")
+    _finish(st, "lmhead_logits_bf16_f32", check, stream)
     return out
 
 
-def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None):
+def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None,
+               check: bool = False):
     """fp32 logits[rows, V] = alpha * (hidden @ W^T + bias) for bf16 or fp16 CUDA tensors hidden
     [rows, H], W [V, H] and optional bias [V], all of one dtype. Runs asynchronously on
     ``stream`` (default: torch's current stream)."""
@@ -281,18 +377,17 @@ def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None):
                and tuple(bias.shape) == (V,), "bias must be a contiguous [V] tensor of the dtype")
     if out is None:
         out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
-    _check(out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (rows, V),
-           "out must be a contiguous fp32 [rows, V] tensor")
+    _check_out(out, torch.float32, (rows, V), hidden.device, "out")
+    _check(W.device == hidden.device, "hidden and W must be on one device")
     st = lmhead_logits_f32(hidden.data_ptr(), dt, rows, H, W.data_ptr(), V, float(alpha),
                            0 if bias is None else bias.data_ptr(), out.data_ptr(),
                            _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logits_f32")
+    _finish(st, "lmhead_logits_f32", check, stream)
     return out
 
 
 def logprobs_f32(hidden, W, targets, alpha: float = 1.0, bias=None, workspace=None, out=None,
-                 stream=None):
+                 stream=None, check: bool = False):
     """(logprobs [rows], lse [rows]) fp32: the log-softmax of the fp32 logits alpha * (hidden @
     W^T + bias) at each row's target token (int32 CUDA tensor [rows]), without writing logits.
     The workspace (logprobs_workspace_bytes(rows, V) bytes) and outputs are allocated here unless
@@ -315,16 +410,20 @@ def logprobs_f32(hidden, W, targets, alpha: float = 1.0, bias=None, workspace=No
         lse = torch.empty((rows,), dtype=torch.float32, device=hidden.device)
     else:
         lp, lse = out
+        _check_out(lp, torch.float32, (rows,), hidden.device, "out[0] (logprobs)")
+        if lse is not None:
+            _check_out(lse, torch.float32, (rows,), hidden.device, "out[1] (lse)")
     need = logprobs_workspace_bytes(rows, V)
     if workspace is None:
         workspace = torch.empty((max(need, 8),), dtype=torch.uint8, device=hidden.device)
+    _check(workspace.is_cuda and workspace.is_contiguous() and workspace.device == hidden.device,
+           "workspace must be a contiguous CUDA tensor on the inputs' device")
     st = lmhead_logprobs_f32(hidden.data_ptr(), dt, rows, H, W.data_ptr(), V, float(alpha),
                              0 if bias is None else bias.data_ptr(), targets.data_ptr(),
                              lp.data_ptr(), 0 if lse is None else lse.data_ptr(),
                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                              _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logprobs_f32")
+    _finish(st, "lmhead_logprobs_f32", check, stream)
     return lp, lse
 
 
@@ -337,7 +436,8 @@ def vocab_shard(V: int, world: int, rank: int):
 
 
 def logprobs_shard_stats_f32(hidden, W_shard, v_begin: int, targets, alpha: float = 1.0,
-                             bias_shard=None, workspace=None, out=None, stream=None):
+                             bias_shard=None, workspace=None, out=None, stream=None,
+                             check: bool = False):
     """fp32 [rows, 3] per-row (max, sum of exp(z - max), target logit or NaN) over the logits of
     this GPU's vocab slice W_shard = W[v_begin : v_begin + V_shard] (targets are global ids)."""
     import torch
@@ -358,22 +458,22 @@ def logprobs_shard_stats_f32(hidden, W_shard, v_begin: int, targets, alpha: floa
                "bias_shard must be a contiguous [V_shard] tensor of the dtype")
     if out is None:
         out = torch.empty((rows, 3), dtype=torch.float32, device=hidden.device)
-    _check(out.dtype == torch.float32 and out.is_contiguous() and out.numel() == rows * 3,
-           "out must be a contiguous fp32 [rows, 3] tensor")
+    _check_out(out, torch.float32, (rows, 3), hidden.device, "out (stats)")
     need = logprobs_workspace_bytes(rows, V_shard)
     if workspace is None:
         workspace = torch.empty((max(need, 8),), dtype=torch.uint8, device=hidden.device)
+    _check(workspace.is_cuda and workspace.is_contiguous() and workspace.device == hidden.device,
+           "workspace must be a contiguous CUDA tensor on the inputs' device")
     st = lmhead_logprobs_shard_stats_f32(
         hidden.data_ptr(), dt, rows, H, W_shard.data_ptr(), V_shard, int(v_begin), float(alpha),
         0 if bias_shard is None else bias_shard.data_ptr(), targets.data_ptr(), out.data_ptr(),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
         _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logprobs_shard_stats_f32")
+    _finish(st, "lmhead_logprobs_shard_stats_f32", check, stream)
     return out
 
 
-def logprobs_merge_shards(stats, out=None, stream=None):
+def logprobs_merge_shards(stats, out=None, stream=None, check: bool = False):
     """(logprobs [rows], lse [rows]) fp32 from the gathered shard stats, fp32 [g, rows, 3] in
     shard order."""
     import torch
@@ -386,11 +486,13 @@ def logprobs_merge_shards(stats, out=None, stream=None):
         lse = torch.empty((rows,), dtype=torch.float32, device=stats.device)
     else:
         lp, lse = out
+        _check_out(lp, torch.float32, (rows,), stats.device, "out[0] (logprobs)")
+        if lse is not None:
+            _check_out(lse, torch.float32, (rows,), stats.device, "out[1] (lse)")
     st = lmhead_logprobs_merge_shards(stats.data_ptr(), g, rows, lp.data_ptr(),
                                       0 if lse is None else lse.data_ptr(),
                                       _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logprobs_merge_shards")
+    _finish(st, "lmhead_logprobs_merge_shards", check, stream)
     return lp, lse
 
 
@@ -411,7 +513,7 @@ def gather_shard_stats(stats, group=None):
 
 def logprobs_vocab_parallel(hidden, W_shard, v_begin: int, targets, alpha: float = 1.0,
                             bias_shard=None, group=None, workspace=None, stats=None, out=None,
-                            stream=None):
+                            stream=None, check: bool = False):
     """(logprobs [rows], lse [rows]) of the whole vocabulary on every rank of ``group``, each
     rank holding its slice W_shard = W[v_begin : v_begin + V_shard] (vocab_shard gives the
     split) and the same hidden rows and targets: shard stats, one all-gather, merge. Without a
@@ -424,11 +526,11 @@ def logprobs_vocab_parallel(hidden, W_shard, v_begin: int, targets, alpha: float
                                      workspace=workspace, out=stats, stream=stream)
     with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
         gathered = gather_shard_stats(stats, group)
-    return logprobs_merge_shards(gathered, out=out, stream=stream)
+    return logprobs_merge_shards(gathered, out=out, stream=stream, check=check)
 
 
 def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha: float = 1.0,
-                       out=None, stream=None):
+                       out=None, stream=None, check: bool = False):
     """bf16 logits[rows, V] for the NVFP4 head: w_packed uint8 [V, H/2], w_scales uint8
     (E4M3) [V, H/16], bf16 hidden [rows, H]."""
     import torch
@@ -442,11 +544,11 @@ def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha:
            "contiguous CUDA tensors required")
     if out is None:
         out = torch.empty((rows, V), dtype=torch.bfloat16, device=hidden.device)
-    _check(out.dtype == torch.bfloat16 and out.is_contiguous() and tuple(out.shape) == (rows, V),
-           "out must be a contiguous bf16 [rows, V] tensor")
+    _check_out(out, torch.bfloat16, (rows, V), hidden.device, "out")
+    _check(w_packed.device == hidden.device and w_scales.device == hidden.device,
+           "hidden, codes and scales must be on one device")
     st = lmhead_logits_w4a16_nvfp4(hidden.data_ptr(), rows, H, w_packed.data_ptr(),
                                    w_scales.data_ptr(), float(w_global_scale), V, float(alpha),
                                    out.data_ptr(), _stream_handle(stream))
-    if st != LMHEAD_OK:
-        raise LmheadError(st, "lmhead_logits_w4a16_nvfp4")
+    _finish(st, "lmhead_logits_w4a16_nvfp4", check, stream)
     return out

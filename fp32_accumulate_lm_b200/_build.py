@@ -1,4 +1,8 @@
-"""Build the CUDA library in-tree: fp32_accumulate_lm_b200/liblmhead.so, for sm_100a only.
+"""Build the CUDA library in-tree, for sm_100a only:
+
+    fp32_accumulate_lm_b200/liblmhead.so        the release library
+    fp32_accumulate_lm_b200/liblmhead_test.so   the same kernels plus two host-side test knobs
+                                                (LMHEAD_TEST_HOOKS=1), loaded only by the tests
 
     python -m fp32_accumulate_lm_b200._build [--force] [--verbose]
 
@@ -20,6 +24,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblmhead.so")
+TEST_LIB = os.path.join(PKG, "liblmhead_test.so")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -35,15 +40,15 @@ def sources() -> list[str]:
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def _compile(out: str, defines: list[str], force: bool, verbose: bool) -> str:
     newest = max(os.path.getmtime(s) for s in sources() + [os.path.abspath(__file__)])
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
            "-Xlinker", "--exclude-libs,ALL", "-Xlinker", "-Bsymbolic",
-           "-I", INCLUDE, "-I", CSRC, "-cudart", "static",
+           "-I", INCLUDE, "-I", CSRC, "-cudart", "static", *defines,
            "-o", tmp, os.path.join(CSRC, "lmhead.cu")]
     if verbose:
         cmd.insert(-3, "-Xptxas")
@@ -54,7 +59,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}): {' '.join(cmd)}")
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False, verbose: bool = False, test_hooks: bool = True) -> str:
+    """Build the release library (and, unless test_hooks is False, the test build); return the
+    release library's path."""
+    _compile(LIB, [], force, verbose)
+    if test_hooks:
+        _compile(TEST_LIB, ["-DLMHEAD_TEST_HOOKS=1"], force, False)
     return LIB
 
 

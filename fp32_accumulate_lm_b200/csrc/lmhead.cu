@@ -7,6 +7,10 @@
 // "muP is folded into the fp32 GEMM"; "FP32 LM head skip FP32 cast", implementation breakdown),
 // and the W4A16 NVFP4 head with bf16 logits (lm_head_nvfp4_rows.rs, lm_head_nvfp4_rows_run).
 // As on that page, a call that cannot run launches nothing and reports why.
+//
+// Built twice: liblmhead.so (the release library) and, with LMHEAD_TEST_HOOKS=1,
+// liblmhead_test.so, which adds the two host-side test knobs (load starvation for the timeout
+// path, a forced NVFP4 conversion). The kernels are the same in both.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,6 +22,10 @@
 #include "lmhead_bf16.cuh"
 #include "lmhead_nvfp4.cuh"
 #include "lmhead_quant.cuh"
+
+#ifndef LMHEAD_TEST_HOOKS
+#define LMHEAD_TEST_HOOKS 0
+#endif
 
 namespace {
 
@@ -50,11 +58,40 @@ struct DeviceInfo {
   bool probed = false;
   bool arch_ok = false;
   bool attrs_set = false;
+  unsigned long long ctx_id = 0;  // the context the kernel attributes were set in
   int num_sms = 0;
   int smem_optin = 0;        // per-block shared-memory opt-in limit (static + dynamic)
   int nvfp4_static_smem = 0;  // static shared memory of the NVFP4 kernels
   int smem_reserved = 0;      // shared memory the system reserves per block
 };
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The unique ID of the calling thread's current context (0 if it cannot be had). Per-context
+// set-up (kernel attributes, the scratch array's address) is redone when the ID changes, as it
+// does after cudaDeviceReset: context IDs are never reused within a process.
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
 
 // Let `kernel` use every byte of shared memory the device allows beside its static part.
 template <typename K>
@@ -106,6 +143,18 @@ int current_device(DeviceInfo* out) {
     d.probed = true;
   }
   if (!d.arch_ok) return LMHEAD_ERR_ARCH;
+  // Bind the device's primary context to this thread if nothing is bound yet (the runtime would
+  // do so at the first launch anyway), so that its ID can key the per-context set-up.
+  unsigned long long ctx = current_context_id();
+  if (ctx == 0) {
+    if (cudaSetDevice(dev) != cudaSuccess) return LMHEAD_ERR_LAUNCH;
+    ctx = current_context_id();
+    if (ctx == 0) return LMHEAD_ERR_LAUNCH;
+  }
+  if (d.ctx_id != ctx) {
+    d.attrs_set = false;
+    d.ctx_id = ctx;
+  }
   if (!d.attrs_set) {
     if (!raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2>, d.smem_optin, nullptr) ||
@@ -241,23 +290,79 @@ int pick_nsub(int32_t bn, int smem_budget) {
 static __device__ __align__(256) uint32_t g_quant_scratch[lmh::kQuantMaxPartials];
 
 std::mutex g_scratch_mu;
-uint32_t* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;
+  uint32_t* ptr = nullptr;
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// The scratch array's device address on the current device. Host code may not use the array's
-// name as a device address (it names a host-side stand-in), so the address is looked up once per
-// device, with that device current, and cached.
+// The scratch array's device address in the current device's context. Host code may not use the
+// array's name as a device address (it names a host-side stand-in), so the address is looked up
+// with cudaGetSymbolAddress once per device, with that device current, and cached for as long as
+// that context lives. The caller has already run current_device(), so a context is bound.
 int quant_scratch(uint32_t** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMHEAD_ERR_LAUNCH;
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return LMHEAD_ERR_LAUNCH;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchAddr& sa = g_scratch[dev];
+  if (sa.ptr == nullptr || sa.ctx_id != ctx) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_quant_scratch) != cudaSuccess || ptr == nullptr)
+    if (cudaGetSymbolAddress(&ptr, g_quant_scratch) != cudaSuccess || ptr == nullptr) {
+      (void)cudaGetLastError();  // leave no stale error for the next call's launch check
       return LMHEAD_ERR_LAUNCH;
-    g_scratch_ptr[dev] = static_cast<uint32_t*>(ptr);
+    }
+    sa.ptr = static_cast<uint32_t*>(ptr);
+    sa.ctx_id = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = sa.ptr;
   return LMHEAD_OK;
+}
+
+// Every host-side check of the quantiser's arguments except the workspace's: shapes, NULLs,
+// alignment and overlap of W and the three outputs. Touches no device state.
+int check_quantize_args(const void* w, int64_t V, int64_t H, const uint8_t* w_packed,
+                        const uint8_t* w_scales, const float* w_global_scale) {
+  if (V <= 0 || H <= 0) return LMHEAD_ERR_SHAPE;
+  if (H % 16 != 0) return LMHEAD_ERR_ALIGN;
+  if (V > kInt32Max || H > kInt32Max) return LMHEAD_ERR_SHAPE;
+  if (w == nullptr || w_packed == nullptr || w_scales == nullptr || w_global_scale == nullptr)
+    return LMHEAD_ERR_NULL;
+  if (!aligned(w, 16) || !aligned(w_packed, 8) || !aligned(w_global_scale, 4))
+    return LMHEAD_ERR_ALIGN;
+  const int64_t n = V * H;
+  const struct { const void* p; int64_t bytes; } regions[4] = {
+      {w, n * 2}, {w_packed, n / 2}, {w_scales, n / 16}, {w_global_scale, 4}};
+  for (int i = 0; i < 4; ++i)
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(regions[i].p, regions[i].bytes, regions[j].p, regions[j].bytes))
+        return LMHEAD_ERR_ALIAS;
+  return LMHEAD_OK;
+}
+
+// The two quantiser launches, after validation. `partial` holds at least `partial_words` words.
+int launch_quantize(const DeviceInfo& dev, const void* w, int64_t V, int64_t H,
+                    uint8_t* w_packed, uint8_t* w_scales, float* w_global_scale,
+                    uint32_t* partial, size_t partial_words, lmhead_stream_t stream) {
+  const int64_t n = V * H;
+  // Pass 1 grid: a few CTAs per SM, one partial word each, never past the scratch.
+  const int64_t n_chunks = n / 8;
+  int64_t grid = (int64_t)dev.num_sms * 6;
+  const int64_t by_work = (n_chunks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
+  if (grid > by_work) grid = by_work;
+  if (grid > lmh::kQuantMaxPartials) grid = lmh::kQuantMaxPartials;
+  if ((size_t)grid > partial_words) return LMHEAD_ERR_SHAPE;
+  const int64_t n_blocks = n / 16;
+  int64_t grid2 = (int64_t)dev.num_sms * 8;
+  const int64_t by_blocks = (n_blocks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
+  if (grid2 > by_blocks) grid2 = by_blocks;
+  lmh::nvfp4_absmax_kernel<<<(unsigned)grid, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(w), n_chunks, partial);
+  lmh::nvfp4_encode_kernel<<<(unsigned)grid2, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(w), n_blocks, partial, (int)grid,
+      reinterpret_cast<uint2*>(w_packed), w_scales, w_global_scale);
+  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
 }
 
 }  // namespace
@@ -280,6 +385,7 @@ const char* lmhead_status_string(int status) {
   }
 }
 
+#if LMHEAD_TEST_HOOKS
 void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) {
   g_starve_loads.store(starve_loads ? 1 : 0);
   g_wait_limit_ns.store(wait_limit_ns);
@@ -288,6 +394,7 @@ void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) 
 void lmhead_debug_set_nvfp4_conversion(int path) {
   g_nvfp4_path.store(path == 1 || path == 2 ? path : 0);
 }
+#endif
 
 size_t lmhead_nvfp4_quantize_workspace_bytes(void) {
   return (size_t)lmh::kQuantMaxPartials * sizeof(uint32_t);
@@ -296,64 +403,47 @@ size_t lmhead_nvfp4_quantize_workspace_bytes(void) {
 int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
                           uint8_t* w_scales, float* w_global_scale, void* workspace,
                           size_t workspace_bytes, lmhead_stream_t stream) {
-  if (V <= 0 || H <= 0) return LMHEAD_ERR_SHAPE;
-  if (H % 16 != 0) return LMHEAD_ERR_ALIGN;
-  if (V > kInt32Max || H > kInt32Max) return LMHEAD_ERR_SHAPE;
-  if (w == nullptr || w_packed == nullptr || w_scales == nullptr || w_global_scale == nullptr ||
-      workspace == nullptr) {
-    return LMHEAD_ERR_NULL;
-  }
-  if (!aligned(w, 16) || !aligned(w_packed, 8) || !aligned(w_global_scale, 4) ||
-      !aligned(workspace, 4)) {
-    return LMHEAD_ERR_ALIGN;
-  }
-  const int64_t n = V * H;
-  const struct { const void* p; int64_t bytes; } regions[5] = {
-      {w, n * 2}, {w_packed, n / 2}, {w_scales, n / 16}, {w_global_scale, 4},
-      {workspace, (int64_t)workspace_bytes}};
-  for (int i = 0; i < 5; ++i)
-    for (int j = i + 1; j < 5; ++j)
-      if (overlaps(regions[i].p, regions[i].bytes, regions[j].p, regions[j].bytes))
-        return LMHEAD_ERR_ALIAS;
-  DeviceInfo dev;
-  const int st = current_device(&dev);
+  int st = check_quantize_args(w, V, H, w_packed, w_scales, w_global_scale);
   if (st != LMHEAD_OK) return st;
-  // Pass 1 grid: a few CTAs per SM, one partial word each, never past the workspace.
-  const int64_t n_chunks = n / 8;
-  int64_t grid = (int64_t)dev.num_sms * 6;
-  const int64_t by_work = (n_chunks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
-  if (grid > by_work) grid = by_work;
-  if (grid > lmh::kQuantMaxPartials) grid = lmh::kQuantMaxPartials;
-  if (workspace_bytes < (size_t)grid * sizeof(uint32_t)) return LMHEAD_ERR_SHAPE;
-  const int64_t n_blocks = n / 16;
-  int64_t grid2 = (int64_t)dev.num_sms * 8;
-  const int64_t by_blocks = (n_blocks + lmh::kQuantThreads - 1) / lmh::kQuantThreads;
-  if (grid2 > by_blocks) grid2 = by_blocks;
-  uint32_t* partial = reinterpret_cast<uint32_t*>(workspace);
-  lmh::nvfp4_absmax_kernel<<<(unsigned)grid, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const uint4*>(w), n_chunks, partial);
-  lmh::nvfp4_encode_kernel<<<(unsigned)grid2, lmh::kQuantThreads, 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const uint4*>(w), n_blocks, partial, (int)grid,
-      reinterpret_cast<uint2*>(w_packed), w_scales, w_global_scale);
-  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+  if (workspace == nullptr) return LMHEAD_ERR_NULL;
+  if (!aligned(workspace, 4)) return LMHEAD_ERR_ALIGN;
+  const int64_t n = V * H;
+  const struct { const void* p; int64_t bytes; } regions[4] = {
+      {w, n * 2}, {w_packed, n / 2}, {w_scales, n / 16}, {w_global_scale, 4}};
+  for (const auto& r : regions)
+    if (overlaps(workspace, (int64_t)workspace_bytes, r.p, r.bytes)) return LMHEAD_ERR_ALIAS;
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+  return launch_quantize(dev, w, V, H, w_packed, w_scales, w_global_scale,
+                         reinterpret_cast<uint32_t*>(workspace), workspace_bytes / 4, stream);
 }
 
 int lmhead_nvfp4_quantize_noalloc(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
                                   uint8_t* w_scales, float* w_global_scale,
                                   lmhead_stream_t stream) {
-  // Validate first, as every entry does, so an invalid call touches no device state.
-  if (V <= 0 || H <= 0) return LMHEAD_ERR_SHAPE;
-  if (H % 16 != 0) return LMHEAD_ERR_ALIGN;
-  if (w == nullptr || w_packed == nullptr || w_scales == nullptr || w_global_scale == nullptr)
-    return LMHEAD_ERR_NULL;
-  uint32_t* scratch = nullptr;
-  const int st = quant_scratch(&scratch);
+  // Every argument check first, so an invalid call touches no device state; then the device
+  // check (ARCH before anything else), and only then the scratch lookup.
+  int st = check_quantize_args(w, V, H, w_packed, w_scales, w_global_scale);
   if (st != LMHEAD_OK) return st;
-  // The quantiser needs one word per CTA of its absmax pass; it sizes that grid to at most
-  // kQuantMaxPartials, so the 4 KB array always suffices, and the workspace entry rejects a
-  // call that would need more.
-  return lmhead_nvfp4_quantize(w, V, H, w_packed, w_scales, w_global_scale, scratch,
-                               sizeof(g_quant_scratch), stream);
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != LMHEAD_OK) return st;
+  uint32_t* scratch = nullptr;
+  st = quant_scratch(&scratch);
+  if (st != LMHEAD_OK) return st;
+  // The absmax grid is capped at kQuantMaxPartials words, the array's size, so a valid call
+  // always fits; launch_quantize still rejects one that would not (LMHEAD_ERR_SHAPE).
+  return launch_quantize(dev, w, V, H, w_packed, w_scales, w_global_scale, scratch,
+                         sizeof(g_quant_scratch) / sizeof(uint32_t), stream);
+}
+
+int lmhead_stream_status(lmhead_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return LMHEAD_ERR_LAUNCH;
+  }
+  return lmhead_device_status(1);
 }
 
 int lmhead_device_status(int clear) {
@@ -580,7 +670,7 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
                               const uint8_t* w_scales, float w_global_scale, int64_t V,
                               float alpha, void* logits, lmhead_stream_t stream) {
   if (rows < 0 || H <= 0 || V <= 0) return LMHEAD_ERR_SHAPE;
-  if (H % 64 != 0) return LMHEAD_ERR_ALIGN;
+  if (H % 32 != 0) return LMHEAD_ERR_ALIGN;
   if (rows > kInt32Max || H > kInt32Max || V > kInt32Max) return LMHEAD_ERR_SHAPE;
   if (rows == 0) return LMHEAD_OK;
   if (hidden == nullptr || w_packed == nullptr || w_scales == nullptr || logits == nullptr)
@@ -611,7 +701,9 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   int grid = 0;
   st = make_sched(rows, V, H, p.bn, dev.num_sms, &p.sched, &grid);
   if (st != LMHEAD_OK) return st;
-  p.num_kb = (int32_t)(H / lmh::kBK);
+  p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
+  p.half_tail = (H % lmh::kBK) != 0 ? 1 : 0;  // H % 64 == 32: the last K step is half a step
+  p.hid_2d = p.half_tail;
   // Hidden sub-tiles start on 1024-byte swizzle atoms: rows per K step rounded up to 8.
   p.hid_rows = rows < p.bn ? (int32_t)((rows + 7) / 8 * 8) : p.bn;
   p.max_stages = lmh::kMaxStages;
@@ -630,8 +722,11 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
                                    : path == 2 ? false : with_table.stages >= 3;
   if ((use_table ? with_table.stages : spread.stages) < 2) return LMHEAD_ERR_SHAPE;
   p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
-  // Block scales come by TMA when each scale row is a whole number of 16-byte units.
-  p.scale_tma = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? 1 : 0;
+  // Block scales come by TMA when each scale row is a whole number of 16-byte units, by 4-byte
+  // async copies when it is a whole number of words, else by the producer's 2-byte loads.
+  p.scale_mode = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? lmh::kScaleTma
+                 : (H / 16) % 4 == 0                             ? lmh::kScaleAsync4
+                                                                 : lmh::kScalePlain;
   p.wait = wait_cfg();
 
   // Packed codes as a [V, H/2] byte matrix, boxes of [128 rows x 128 bytes] (4 K steps) with the
@@ -640,14 +735,19 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   st = encode_rows(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_packed, H / 2, V,
                    lmh::kRawK * lmh::kBK / 2, lmh::kBM, CU_TENSOR_MAP_SWIZZLE_128B, kWeightPromo);
   if (st != LMHEAD_OK) return st;
-  if (p.scale_tma) {
+  if (p.scale_mode == lmh::kScaleTma) {
     st = encode_rows(&tmap_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_scales, H / 16, V,
                      lmh::kRawK * 4, lmh::kBM, CU_TENSOR_MAP_SWIZZLE_NONE, kWeightPromo);
     if (st != LMHEAD_OK) return st;
   } else {
     tmap_s = tmap_q;  // unused
   }
-  st = encode_hidden_ksteps(&tmap_h, hidden, rows, H, (uint32_t)p.hid_rows, lmh::kRawK);
+  if (p.hid_2d)  // [rows, H] with [hid_rows x 64] boxes: K past H is zero-filled
+    st = encode_rows(&tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, H * 2, rows,
+                     lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  else
+    st = encode_hidden_ksteps(&tmap_h, hidden, rows, H, (uint32_t)p.hid_rows, lmh::kRawK);
   if (st != LMHEAD_OK) return st;
 
   if (use_table)

@@ -80,12 +80,23 @@ struct Nvfp4HeadParams {
   int32_t hid_rows;       // hidden rows per K step in a stage: a multiple of 8, <= bn (MMA
                           // columns past the call's rows read neighbouring data, never stored)
   TileSched sched;
-  int32_t num_kb;         // K steps of 64 per tile (H / 64)
+  int32_t num_kb;         // K steps of 64 per tile: ceil(H / 64)
   int32_t max_stages;     // cap on the shared-memory ring; the kernel fits what room allows
   int32_t slots;          // TMEM weight slots: 3 when 2 * bn + 3 * 128 <= 512, else 2
-  int32_t scale_tma;      // 1: block scales by TMA (H % 256 == 0), 0: 4-byte async copies
+  int32_t scale_mode;     // block scales: kScaleTma, kScaleAsync4 or kScalePlain (see below)
+  int32_t half_tail;      // 1 when H % 64 == 32: the last K step holds 32 elements (2 MMAs)
+  int32_t hid_2d;         // 1: hidden rows by one 2-D box per K step (needed when H % 64 != 0)
   WaitCfg wait;
 };
+
+// How the producer brings a stage's block scales into shared memory:
+//   kScaleTma     one TMA box [128 rows x 16 bytes]; needs H % 256 == 0 and 16-byte aligned scales
+//   kScaleAsync4  4-byte async copies, one per row and K step; needs H % 64 == 0 (whole words)
+//   kScalePlain   2-byte loads and shared stores by the producer's lanes, for H % 64 == 32, where
+//                 a scale row is not a whole number of words (its K steps' 4 bytes straddle rows)
+constexpr int32_t kScaleAsync4 = 0;
+constexpr int32_t kScaleTma = 1;
+constexpr int32_t kScalePlain = 2;
 
 // Shared-memory stage (4 K steps): [hidden: 4 sub-tiles of hid_rows x 64 bf16, 128-byte swizzle,
 // from one 3-D box, plus room for the last sub-tile's MMA to read bn rows][codes: 128 rows x
@@ -149,6 +160,22 @@ __device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tm
       "setp.ne.b32 p, %4, 0;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Half a K step (32 elements) with A from TMEM: two K = 16 MMAs; only the first may start a fresh
+// accumulator. For the last K step of a head whose H is an odd multiple of 32.
+__device__ __forceinline__ void mma2_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 a1;\n\t.reg .b64 b1;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "add.s32 a1, %1, 8;\n\tadd.s64 b1, %2, 2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, 1;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -393,8 +420,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // expect_tx arrive (+ 32 scale-copy arrivals when the scales come by async copies)
-      mbar_init(full0 + 8 * s, p.scale_tma ? 1 : 1 + 32);
+      // expect_tx arrive (+ 32 producer-lane arrivals when the scales do not come by TMA)
+      mbar_init(full0 + 8 * s, p.scale_mode == kScaleTma ? 1 : 1 + 32);
       // the dequantisers have read the codes and the MMAs have read the hidden rows
       mbar_init(empty0 + 8 * s, kDequantThreads + 1);
     }
@@ -412,7 +439,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_q);
-    if (p.scale_tma) prefetch_tmap(&tmap_s);
+    if (p.scale_mode == kScaleTma) prefetch_tmap(&tmap_s);
     prefetch_tmap(&tmap_h);
   }
   if (warp == 1) {
@@ -457,17 +484,26 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           const uint32_t full = full0 + 8 * st;
           const uint32_t sbase = stage_addr(st);
           if (lane == 0) {
-            // Boxes are counted whole: K steps past H arrive zero-filled.
-            mbar_arrive_expect_tx(full,
-                                  kRawCodeBytes + (p.scale_tma ? kRawScaleBytes : 0u) + hid_tx);
+            // Boxes are counted whole: K steps past H arrive zero-filled. With 2-D hidden boxes
+            // only the stage's nk K steps are loaded.
+            const uint32_t h_tx = p.hid_2d ? (uint32_t)nk * hsub : hid_tx;
+            mbar_arrive_expect_tx(
+                full, kRawCodeBytes + (p.scale_mode == kScaleTma ? kRawScaleBytes : 0u) + h_tx);
             tma_load_2d(sbase + off_q, &tmap_q, full, tma_x(r * (kRawK * kBK / 2), 1),
                         (int32_t)tc.v0, pol_w);
-            if (p.scale_tma)
+            if (p.scale_mode == kScaleTma)
               tma_load_2d(sbase + off_s, &tmap_s, full, tma_x(r * (kRawK * 4), 1),
                           (int32_t)tc.v0, pol_w);
-            tma_load_3d(sbase, &tmap_h, full, 0, (int32_t)tc.r0, r * kRawK, pol_h);
+            if (p.hid_2d) {
+              // [hid_rows x 64] boxes of a [rows, H] map: elements past H are zero-filled
+              for (int j = 0; j < nk; ++j)
+                tma_load_2d(sbase + (uint32_t)j * hsub, &tmap_h, full,
+                            tma_x((int64_t)(r * kRawK + j) * kBK * 2, 2), (int32_t)tc.r0, pol_h);
+            } else {
+              tma_load_3d(sbase, &tmap_h, full, 0, (int32_t)tc.r0, r * kRawK, pol_h);
+            }
           }
-          if (!p.scale_tma) {
+          if (p.scale_mode == kScaleAsync4) {
             // 4 rows per lane, 4 K steps of 4 bytes each; rows past V and K steps past H copy
             // nothing (zero-filled).
 #pragma unroll
@@ -484,6 +520,33 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
               }
             }
             cp_async_arrive_noinc(full);
+          } else if (p.scale_mode == kScalePlain) {
+            // The scale row's pitch is 2 mod 4 bytes: read it in 2-byte pieces (every piece is
+            // 2-byte aligned), zeros past H and past V, so the dequantisers' words are whole.
+            uint32_t word[4][kRawK];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = lane * 4 + i;
+              const bool in_row = tc.v0 + row < p.V;
+              const uint16_t* srow = reinterpret_cast<const uint16_t*>(
+                  p.scales + (in_row ? (tc.v0 + row) * scale_pitch : 0));
+#pragma unroll
+              for (int j = 0; j < kRawK; ++j) {
+                const int64_t b0 = (int64_t)(r * kRawK + j) * 4;  // byte of the K step in a row
+                const uint32_t lo = (in_row && b0 < scale_pitch) ? srow[b0 >> 1] : 0u;
+                const uint32_t hi = (in_row && b0 + 2 < scale_pitch) ? srow[(b0 >> 1) + 1] : 0u;
+                word[i][j] = lo | (hi << 16);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int j = 0; j < kRawK; ++j)
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + off_s +
+                                                             (uint32_t)((lane * 4 + i) * 16 + j * 4)),
+                             "r"(word[i][j])
+                             : "memory");
+            mbar_arrive(full);  // release: the stores above are seen by whoever waits on `full`
           }
         }
         __syncwarp();
@@ -536,14 +599,21 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
           const uint64_t bdesc0 = sdesc_kmajor_sw128(stage_addr(st));
           const uint32_t a0 = tmem_base + slot_col0 + (uint32_t)sl * kSlotCols;
+          // The tile's last K step is half a step when H % 64 == 32: two MMAs, not four (the
+          // zero codes past H are never multiplied).
+          const bool half_last = p.half_tail && r == n_raw - 1;
           // descriptor start addresses are in 16-byte units
-          if (nk == kRawK) {
+          if (nk == kRawK && !half_last) {
             mma16_bf16_ts_elect(d_tmem, a0, bdesc0, hsub >> 4, idesc, r != 0);
           } else {
-            for (int j = 0; j < nk; ++j)
-              mma4_bf16_ts_elect(d_tmem, a0 + (uint32_t)(j * (kBK / 2)),
-                                 bdesc0 + (uint64_t)((j * hsub) >> 4), idesc,
-                                 (r | j) != 0);
+            for (int j = 0; j < nk; ++j) {
+              const uint32_t aj = a0 + (uint32_t)(j * (kBK / 2));
+              const uint64_t bj = bdesc0 + (uint64_t)((j * hsub) >> 4);
+              if (half_last && j == nk - 1)
+                mma2_bf16_ts_elect(d_tmem, aj, bj, idesc, (r | j) != 0);
+              else
+                mma4_bf16_ts_elect(d_tmem, aj, bj, idesc, (r | j) != 0);
+            }
           }
           mma_commit_elect(empty0 + 8 * st);
           mma_commit_elect(aempty0 + 8 * sl);

@@ -187,10 +187,11 @@ int lmhead_logprobs_merge_shards(const float* stats, int64_t shards, int64_t row
  * w_global_scale is the decode multiplier (w = code * scale * w_global_scale).
  *
  *   hidden    bf16 [rows, H], 16-byte aligned        rows >= 0
- *   w_packed  u8 [V, H/2],    16-byte aligned        H > 0, H % 64 == 0
+ *   w_packed  u8 [V, H/2],    16-byte aligned        H > 0, H % 32 == 0 (16-byte code rows)
  *   w_scales  u8 [V, H/16],   4-byte aligned
  *   logits    bf16 [rows, V], 2-byte aligned         V > 0
- * (H % 64 == 0 makes every scale row a whole number of 4-byte words.)
+ * The kernel works in K steps of 64; when H % 64 == 32 the last step is half a step (the codes
+ * past H read as zero and are not multiplied), with the same bits for every row count.
  * Returns an lmhead_status.
  */
 int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const uint8_t* w_packed,
@@ -228,17 +229,19 @@ int lmhead_nvfp4_quantize(const void* w, int64_t V, int64_t H, uint8_t* w_packed
  * lmhead_nvfp4_quantize without a workspace argument, for callers that cannot obtain device
  * memory of their own: code that is handed its weight and output buffers by another component
  * (a model loader or a serving engine's memory pool) and is not allowed to call cudaMalloc, which
- * can synchronise the whole device and bypasses the pool that owns the GPU's memory. The paper
- * has no counterpart to this entry point; it exists for those callers.
+ * can synchronise the whole device and bypasses the pool that owns the GPU's memory. The method's
+ * published description has no counterpart to this entry point; it exists for those callers.
  *
  * Same arguments, rules and results as lmhead_nvfp4_quantize. The absmax pass's scratch is a 4 KB
  * array that the library keeps on every GPU it is loaded on, until the process exits; the call
- * allocates nothing. Its first call on a device looks up that array's device address (a host-side
- * setup step, once per device, done while that device is current), so make that first call
- * before any stream capture. All calls on a device share the one array: calls whose work overlaps
- * on the GPU (on different streams without ordering between them) race and give undefined
- * results, so order them. The array needs no clearing; each call's absmax pass writes every word
- * its encode pass reads. A call that would need more than the 4 KB is rejected with
+ * allocates nothing. Every argument is checked before any device state is touched. The first
+ * call on a device (and the first after that device's context was replaced, e.g. by
+ * cudaDeviceReset) looks up the array's device address, a host-side set-up step done while that
+ * device is current, so make that first call before any stream capture. All calls on a device
+ * share the one array: calls whose work overlaps on the GPU (on different streams without
+ * ordering between them) race and give undefined results, so order them. The array needs no
+ * clearing: each call's absmax pass writes every word its encode pass reads, and the encode pass
+ * reads no other word. A call that would need more than the 4 KB is rejected with
  * LMHEAD_ERR_SHAPE (the quantiser's grid is sized to stay within it). Returns an lmhead_status.
  */
 int lmhead_nvfp4_quantize_noalloc(const void* w, int64_t V, int64_t H, uint8_t* w_packed,
@@ -251,32 +254,42 @@ const char* lmhead_status_string(int status);
 /*
  * Every wait inside the kernels is bounded. When one runs out (the default limit is 2 s of wall
  * time per wait) the kernel records LMHEAD_ERR_TIMEOUT, and where it gave up, in a per-device
- * status word, stops its work and exits cleanly, so the CUDA context stays usable; the logits
- * of that call are then undefined. Read the word after synchronising the stream:
- * returns the recorded status of the CURRENT device (LMHEAD_OK if none) and, when `clear` is
- * non-zero, resets it. The low byte is the lmhead_status; bits 8..15 name the waiting role.
+ * status word, stops its work and exits cleanly, so the CUDA context stays usable; the outputs
+ * of that call are then undefined. The call itself returned LMHEAD_OK before its kernels ran, so
+ * a caller that must not consume such outputs checks after synchronising:
+ *
+ * lmhead_device_status: the recorded status of the CURRENT device (LMHEAD_OK if none) and, when
+ * `clear` is non-zero, resets it. The low byte is the lmhead_status; bits 8..15 name the waiting
+ * role. It does not synchronise; read it after the work of interest has finished.
+ *
+ * lmhead_stream_status: synchronises `stream`, then returns and clears the current device's
+ * status word (LMHEAD_OK when no wait ran out; LMHEAD_ERR_LAUNCH when the synchronisation itself
+ * reported a CUDA error). The word is per device, not per stream: a timeout of work on another
+ * stream of the same device that finished before this call is reported here too.
  */
 int lmhead_device_status(int clear);
+int lmhead_stream_status(lmhead_stream_t stream);
 
 /* Library version as 10000 * major + 100 * minor + patch. */
 int lmhead_version(void);
 
+#if defined(LMHEAD_TEST_HOOKS) && LMHEAD_TEST_HOOKS
 /*
- * Fault-injection knob for tests of the timeout path (host side, per process). When
- * `starve_loads` is non-zero, subsequent launches issue no weight/activation loads, so their
- * consumers wait on barriers that never complete and must time out after `wait_limit_ns`
- * nanoseconds. wait_limit_ns == 0 restores the default limit. Not for production use.
- */
-void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
-
-/*
- * Test knob (host side, per process) for lmhead_logits_w4a16_nvfp4's two ways of turning codes
+ * Test build only (liblmhead_test.so, compiled with LMHEAD_TEST_HOOKS=1; the release
+ * liblmhead.so does not export these). Host-side, per process:
+ *
+ * lmhead_debug_set_fault_injection: when `starve_loads` is non-zero, subsequent launches issue
+ * no weight/activation loads, so their consumers wait on barriers that never complete and must
+ * time out after `wait_limit_ns` nanoseconds. wait_limit_ns == 0 restores the default limit.
+ *
+ * lmhead_debug_set_nvfp4_conversion: selects lmhead_logits_w4a16_nvfp4's way of turning codes
  * into bf16: 1 = the shared-memory pair table whenever it leaves room for two pipeline stages,
  * 2 = integer spreading only, anything else = automatic (the table when it leaves room for
- * three stages). Both give identical bits; the knob exists so tests can show that. Not for
- * production use.
+ * three stages). Both give identical bits; the knob lets tests show that.
  */
+void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
 void lmhead_debug_set_nvfp4_conversion(int path);
+#endif
 
 #ifdef __cplusplus
 }

@@ -4,7 +4,7 @@ import numpy as np
 import torch
 
 import fp32_accumulate_lm_b200 as lm
-from fp32_accumulate_lm_b200 import synth
+import synth
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:

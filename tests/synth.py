@@ -1,19 +1,16 @@
-"""Seeded synthetic inputs for the LM head (hidden rows, bf16 weights, NVFP4 weights).
+"""Seeded synthetic inputs for the LM head (hidden rows, bf16 and fp16 weights, biases, random
+NVFP4 codes for timing).
 
-This module makes data only; it holds none of the head's arithmetic (no products, sums, alpha or
-output rounding). Tests and the benchmark draw every input from here, so both sides of a parity
-check see the same bits.
+This module makes data only; it holds none of the head's arithmetic (no products, sums, alpha,
+output rounding or quantisation). Tests, the smoke run and the benchmark draw every input from
+here, so both sides of a parity check see the same bits. It is not part of the library.
 
 Recipe (the pages name no dataset; shapes and value distributions follow the workloads):
   * hidden[rows, H]  ~ N(0, 1) drawn in fp32 from a seeded ``torch.Generator``, rounded to bf16
     (round-to-nearest-even, ``Tensor.to(torch.bfloat16)``).
   * W[V, H]          ~ N(0, std) the same way (std 0.02, or 0.015 for the 4096-wide head).
-  * NVFP4 weights    come from quantising such a bf16 W: a per-tensor fp32 scale
-    g = amax|W| / (6 * 448), per-16-element E4M3 block scales s = RN_e4m3(amax_block / 6 / g)
-    (saturating at 448) and E2M1 codes q = RN_e2m1(w / (s * g)) (ties to even, saturating at
-    +-6; q = 0 where s = 0). lm_head_nvfp4_rows.rs and mtp_head/new_bf16_moe.rs name an NVFP4
-    quantiser (absmax, then encode) but print no rules, so these are this library's reading.
-    Packing: element 2j of a row is the low nibble of byte j, element 2j+1 the high nibble.
+  * NVFP4 test weights come from quantising such a bf16 W with the oracle's quantiser (the
+    tests do that, not this module); timing runs use uniformly random codes and scales instead.
 
 Arrays are returned as numpy (bf16 as uint16 bit patterns) unless a torch device is given.
 """
@@ -106,55 +103,6 @@ def bits_to_torch_bf16(bits: np.ndarray, device="cpu") -> torch.Tensor:
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns to float32 (exact)."""
     return (np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
-
-
-# ---------------------------------------------------------------- NVFP4 test-weight generator
-
-# Encoding tables, written from the formats' definitions (bias 7 / bias 1, subnormals below).
-_E4M3_POS_CODES = np.arange(0x00, 0x7F, dtype=np.uint8)  # 0x7F is NaN
-_E4M3_POS_VALUES = np.array(
-    [((c & 7) / 8.0) * 2.0 ** -6 if (c >> 3) == 0 else (1 + (c & 7) / 8.0) * 2.0 ** ((c >> 3) - 7)
-     for c in (int(x) for x in _E4M3_POS_CODES)], dtype=np.float64)
-_E2M1_MAGS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
-
-
-def _round_to_table(x: np.ndarray, values: np.ndarray) -> np.ndarray:
-    """Index of the nearest entry of the ascending table ``values`` (ties to the even index,
-    which is the even code); values beyond the ends saturate."""
-    x = np.clip(x, values[0], values[-1])
-    hi = np.clip(np.searchsorted(values, x, side="left"), 1, len(values) - 1)
-    lo = hi - 1
-    dlo = x - values[lo]
-    dhi = values[hi] - x
-    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
-    return np.where(pick_hi, hi, lo)
-
-
-def nvfp4_quantize(w_bits: np.ndarray):
-    """Quantise bf16 W[V, H] (uint16 bits, H % 16 == 0) to (packed [V, H/2] u8,
-    scales [V, H/16] u8, g float)."""
-    w = bf16_bits_to_f32(w_bits).astype(np.float64)
-    V, H = w.shape
-    if H % 16:
-        raise ValueError("H must be a multiple of 16")
-    amax = float(np.max(np.abs(w))) if w.size else 0.0
-    g = float(np.float32(amax / (6.0 * 448.0))) if amax > 0 else 1.0
-    blocks = np.abs(w).reshape(V, H // 16, 16).max(axis=2)
-    s_idx = _round_to_table(blocks / 6.0 / g, _E4M3_POS_VALUES)
-    scales = _E4M3_POS_CODES[s_idx].astype(np.uint8)
-    s_val = _E4M3_POS_VALUES[s_idx]
-    denom = np.repeat(s_val, 16, axis=1) * g
-    with np.errstate(divide="ignore", invalid="ignore"):
-        target = np.where(denom > 0, w / np.where(denom > 0, denom, 1.0), 0.0)
-    mag = _round_to_table(np.abs(target), _E2M1_MAGS).astype(np.uint8)
-    codes = mag | np.where((target < 0) & (mag > 0), 8, 0).astype(np.uint8)
-    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
-    return np.ascontiguousarray(packed), np.ascontiguousarray(scales), g
-
-
-def nvfp4_weights(V: int, H: int, std: float, seed: int):
-    """Seeded NVFP4 head: quantise a seeded N(0, std) bf16 W[V, H]."""
-    return nvfp4_quantize(weight(V, H, std, seed))
 
 
 def random_nvfp4_codes(V: int, H: int, seed: int, device=None):

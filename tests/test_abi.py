@@ -21,10 +21,31 @@ def lib():
     return lm.load_library()
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def _functions(text: str):
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(lmhead_[a-z0-9_]+)\s*\(", text)))
+
+
+def _test_block(text: str) -> str:
+    m = re.search(r"#if defined\(LMHEAD_TEST_HOOKS\) && LMHEAD_TEST_HOOKS(.*?)#endif", text, re.S)
+    return m.group(1) if m else ""
+
+
+def declared_functions():
+    """Functions of the release library: everything outside the test-build block."""
+    text = open(HEADER).read()
+    test_only = set(_functions(_test_block(text)))
+    return [f for f in _functions(text) if f not in test_only]
+
+
+def hook_functions():
+    return _functions(_test_block(open(HEADER).read()))
+
+
+def exported(path: str):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    return {line.split()[-1] for line in out.splitlines() if line.strip()}
 
 
 def test_header_declares_the_two_entry_points():
@@ -33,21 +54,36 @@ def test_header_declares_the_two_entry_points():
 
 
 def test_library_exports_every_declared_symbol(lib):
-    out = subprocess.run(["nm", "-D", "--defined-only", lm.library_path()], capture_output=True,
-                         text=True, check=True).stdout
-    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    syms = exported(lm.library_path())
     for name in declared_functions():
-        assert name in exported, name
+        assert name in syms, name
         assert getattr(lib, name) is not None
     # nothing from the statically linked CUDA runtime leaks out
-    assert not any(s.startswith("cuda") for s in exported)
+    assert not any(s.startswith("cuda") for s in syms)
+
+
+def test_test_knobs_exist_only_in_the_test_build(lib):
+    """The fault-injection and conversion knobs are declared for LMHEAD_TEST_HOOKS builds only:
+    the release library does not export them, the test build exports them and everything else."""
+    knobs = hook_functions()
+    assert set(knobs) == {"lmhead_debug_set_fault_injection", "lmhead_debug_set_nvfp4_conversion"}
+    release, test = exported(lm.library_path()), exported(_build.TEST_LIB)
+    assert not set(knobs) & release
+    assert set(knobs) | set(declared_functions()) <= test
+    assert not any(s.startswith("cuda") for s in test)
+    with pytest.raises(RuntimeError):
+        lm.set_fault_injection(True, 1)       # outside test_hooks(): refused, nothing changes
+    with lm.test_hooks() as tlib:
+        assert tlib is lm.load_test_library()
+        lm.set_nvfp4_conversion(0)           # reachable inside
 
 
 def test_header_compiles_as_c():
     src = f'#include "{HEADER}"\nint main(void) {{ return lmhead_version() < 0; }}\n'
-    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-x", "c", "-"],
-                         input=src, capture_output=True, text=True)
-    assert res.returncode == 0, res.stderr
+    for defs in ([], ["-DLMHEAD_TEST_HOOKS=1"]):
+        res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", *defs,
+                              "-x", "c", "-"], input=src, capture_output=True, text=True)
+        assert res.returncode == 0, res.stderr
 
 
 def test_status_strings_and_version(lib):
@@ -116,6 +152,32 @@ def test_quantiser_argument_errors(lib):
     assert f(A16, 4, 64, B16, C16, B16 + 8, WS, need, 0) == 7           # g inside packed
 
 
+def test_noalloc_quantiser_checks_everything_before_the_device(lib):
+    """lmhead_nvfp4_quantize_noalloc rejects every invalid call before it looks up its scratch
+    or touches any device state, so these codes come back the same on a host without a GPU."""
+    f = lm.lmhead_nvfp4_quantize_noalloc
+    G = 0x60000000
+    assert f(A16, 0, 64, B16, C16, G, 0) == 2                  # V = 0
+    assert f(A16, 4, 40, B16, C16, G, 0) == 3                  # H % 16 != 0
+    assert f(A16, 2 ** 31, 64, B16, C16, G, 0) == 2            # V past int32
+    assert f(A16, 4, 2 ** 31 + 16, B16, C16, G, 0) == 2        # H past int32
+    assert f(0, 4, 64, B16, C16, G, 0) == 1
+    assert f(A16, 4, 64, B16, C16, 0, 0) == 1
+    assert f(A16 + 8, 4, 64, B16, C16, G, 0) == 3              # W not 16-byte aligned
+    assert f(A16, 4, 64, B16 + 4, C16, G, 0) == 3              # codes not 8-byte aligned
+    assert f(A16, 4, 64, B16, C16, G + 2, 0) == 3              # g not 4-byte aligned
+    assert f(A16, 4, 64, B16, B16 + 64, G, 0) == 7             # scales over the codes
+    assert f(A16, 4, 64, A16 + 128, C16, G, 0) == 7            # codes over W
+    assert f(A16, 4, 64, B16, C16, C16 + 8, 0) == 7            # g inside the scales
+
+
+def test_stream_status_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lm.lmhead_stream_status(0) == 5                     # the synchronisation fails
+
+
 def test_logprobs_argument_errors(lib):
     f = lm.lmhead_logprobs_f32
     T, LP, LSE, WS = 0x60000000, 0x61000000, 0x62000000, 0x63000000
@@ -144,7 +206,8 @@ def test_nvfp4_argument_errors(lib):
     f = lm.lmhead_logits_w4a16_nvfp4
     assert f(A16, 4, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) != 2  # valid shape gets past
     assert f(A16, -1, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 2
-    assert f(A16, 4, 96, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 3   # H % 64 != 0
+    assert f(A16, 4, 80, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 3   # H % 32 != 0
+    assert f(A16, 4, 96, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) not in (1, 2, 3, 7)  # 32 mod 64
     assert f(A16, 4, 64, B16, C16, 1.0, 0, 1.0, 0x7000000, 0) == 2
     assert f(0, 4, 64, B16, C16, 1.0, 128, 1.0, 0x7000000, 0) == 1
     assert f(A16, 4, 64, 0, C16, 1.0, 128, 1.0, 0x7000000, 0) == 1

@@ -16,16 +16,40 @@ KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "
         "clocks"}
 
 
+RECORD_KEYS = {"value", "unit", "ms_per_step", "scaling", "dtype", "config", "per_rows",
+               "roofline", "e2e", "gpu_launches", "clocks"}
+
+
+def check_record(rec: dict):
+    assert rec["value"] > 0 and rec["gpu_launches"] >= 1
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(rec["roofline"])
+    assert {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"} <= set(rec["e2e"])
+    assert {"workload", "parallelism", "calls_per_step", "rows_per_call"} <= set(rec["config"])
+
+
 @pytest.mark.parametrize("workload", ["decode", "spec_verify", "nvfp4", "decode_f16_bias",
                                       "prefill", "prefill_logprobs", "nvfp4_quantize",
                                       "vocab_parallel_logprobs"])
 def test_bench_line(workload):
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", workload,
-                          "--steps", "1", "--warmup", "3", "--no-cpu-baseline"],
-                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    """Each workload alone (--only); the default decode run also measures every other workload
+    into the line's "workloads" map."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--workload", workload,
+           "--steps", "1", "--warmup", "3", "--no-cpu-baseline"]
+    if workload != "decode":
+        cmd.append("--only")
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert KEYS <= set(line), KEYS - set(line)
-    assert line["value"] > 0 and line["n_gpus"] == 1 and line["gpu_launches"] >= 1
-    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(line["roofline"])
-    assert {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"} <= set(line["e2e"])
+    assert line["n_gpus"] == 1
+    check_record(line)
+    if workload == "decode":
+        import bench
+        assert set(line["workloads"]) == set(bench.SECONDARY)
+        for name, rec in line["workloads"].items():
+            assert RECORD_KEYS <= set(rec), (name, RECORD_KEYS - set(rec))
+            check_record(rec)
+            assert rec["config"] == bench.config_of(name, 1)
+        assert line["workloads"]["prefill"]["roofline"]["bound"] == "tensor"
+    else:
+        assert "workloads" not in line

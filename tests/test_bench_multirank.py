@@ -70,3 +70,30 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     class Args:
         workload, steps, warmup, gpus = "decode", 3, 3, 2
     assert bench.run_reference(Args()) is None
+
+
+def test_reference_arm_line_and_config_match_the_repo_arm(monkeypatch):
+    """The reference arm (the CPU oracle) on a shrunken decode workload: the contract's keys,
+    impl "reference", and the same config dict as the repo arm's line for the same N, so the two
+    lines describe the same workload."""
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import bench
+    import synth
+    monkeypatch.setitem(synth.WORKLOADS, "decode", ([1, 2, 4], 256, 1024, 0.02, 1.0 / 8))
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+
+    class Args:
+        workload, steps, warmup, gpus = "decode", 3, 3, 1
+    line = bench.run_reference(Args())
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "us/call"
+    assert line["config"] == bench.config_of("decode", 1)
+    assert line["config"]["rows_per_call"] == [1, 2, 4]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "us/call", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    # the plan times the step's distinct rows (4 here) against the whole small vocabulary
+    n_rows, vslice, scale = bench._oracle_plan("decode", 1.0)
+    assert n_rows == 4 and vslice == 1024 and scale == pytest.approx((1 + 2 + 4) / 4 / 3)

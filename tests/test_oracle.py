@@ -16,7 +16,8 @@ import pytest
 import torch
 
 import oracle
-from fp32_accumulate_lm_b200 import synth
+import synth
+from oracle_inputs import nvfp4_weights
 
 
 def bf16_bits_of_f32(x: np.ndarray) -> np.ndarray:
@@ -279,7 +280,7 @@ def _dequant_with_torch(packed, scales, g):
 
 def test_nvfp4_weight_decode_matches_torch_dequant():
     V, H = 40, 64
-    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 123)
+    packed, scales, g = nvfp4_weights(V, H, 0.02, 123)
     ref = _dequant_with_torch(packed, scales, g)
     for v in range(V):
         for k in range(H):
@@ -288,7 +289,7 @@ def test_nvfp4_weight_decode_matches_torch_dequant():
 
 def test_nvfp4_head_one_hot_and_integer_cases():
     V, H = 48, 64
-    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 321)
+    packed, scales, g = nvfp4_weights(V, H, 0.02, 321)
     wq = _dequant_with_torch(packed, scales, g)
     ks = [0, 1, 15, 16, 63]
     h = np.zeros((len(ks), H), np.float32)
@@ -315,7 +316,7 @@ def test_nvfp4_head_one_hot_and_integer_cases():
 def test_nvfp4_head_matches_library_double_matmul():
     rows, H, V = 5, 256, 300
     h = synth.hidden(rows, H, 31)
-    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, 32)
+    packed, scales, g = nvfp4_weights(V, H, 0.02, 32)
     out, _ = oracle.logits_w4a16_nvfp4(h, packed, scales, g, 0.125)
     wq = _dequant_with_torch(packed, scales, g)
     ref = 0.125 * (synth.bf16_bits_to_f32(h).astype(np.float64) @ wq.T)
@@ -326,13 +327,14 @@ def test_nvfp4_head_matches_library_double_matmul():
 
 
 def test_nvfp4_quantiser_round_trip_bounds():
-    """The test-weight generator: decoded NVFP4 is within half an E2M1 step (relative to the block
-    scale) of the bf16 weights it came from, and block maxima land on +-6 * s * g within E4M3
-    rounding."""
+    """The oracle quantiser (which also makes the NVFP4 test weights): decoded NVFP4 is within one
+    E2M1 step (relative to the block scale) of the bf16 weights it came from, and no decoded
+    weight exceeds 6 * 448 * g."""
     V, H = 64, 256
     w_bits = synth.weight(V, H, 0.02, 44)
     wf = synth.bf16_bits_to_f32(w_bits).astype(np.float64)
-    packed, scales, g = synth.nvfp4_quantize(w_bits)
+    packed, scales, g = oracle.nvfp4_quantize(w_bits)
+    g = float(g)
     wq = _dequant_with_torch(packed, scales, g)
     s = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).double().numpy()
     step = np.repeat(s, 16, axis=1) * g  # the value of one E2M1 unit in this block
@@ -340,20 +342,6 @@ def test_nvfp4_quantiser_round_trip_bounds():
     assert np.all(np.abs(wq - wf) <= 1.0 * step + 1e-30)
     assert np.max(np.abs(wq)) <= 6 * 448 * g * (1 + 1e-12)
 
-
-def test_synth_e4m3_table_matches_torch():
-    """The generator's E4M3 encode table is ascending and equals torch's decode."""
-    vals = synth._E4M3_POS_VALUES
-    lib = torch.from_numpy(synth._E4M3_POS_CODES.copy()).view(torch.float8_e4m3fn).double().numpy()
-    assert np.array_equal(vals, lib)
-    assert np.all(np.diff(vals) > 0)
-
-
-# ---------------------------------------------------------------- fp16 inputs and the bias term
-# "FP32 LM head skip FP32 cast": the fused path's predicate admits float16 as well as bfloat16
-# hidden states of the weight's dtype. The first page's "Purpose" lists the embedding bias among
-# the cases handled as projection-with-bias followed by the multiply by 1/mup:
-#     logits = RN_fp32(alpha * (hidden @ W^T + bias)).
 
 def f16_bits(x: np.ndarray) -> np.ndarray:
     """float -> IEEE binary16 bits through numpy (round-to-nearest-even: a library routine)."""

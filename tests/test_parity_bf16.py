@@ -16,7 +16,7 @@ import torch
 
 import oracle
 import fp32_accumulate_lm_b200 as lm
-from fp32_accumulate_lm_b200 import synth
+import synth
 from gpu_helpers import bf16_bits_of_f32, check_status, dev_bf16, f32_bits, gpu_bf16_f32
 from tolerance import assert_fp32_close
 

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import fp32_accumulate_lm_b200 as lm
-from fp32_accumulate_lm_b200 import synth
+import synth
 from gpu_helpers import check_status
 from tolerance import assert_fp32_close
 

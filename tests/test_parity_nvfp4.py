@@ -11,7 +11,8 @@ import torch
 
 import oracle
 import fp32_accumulate_lm_b200 as lm
-from fp32_accumulate_lm_b200 import synth
+import synth
+from oracle_inputs import nvfp4_weights
 from gpu_helpers import bf16_bits_of_f32, check_status, dev_bf16, dev_u8, gpu_nvfp4
 from tolerance import assert_bf16_close
 
@@ -20,10 +21,14 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture(params=[1, 2], ids=["pair_table", "spread"])
 def conversion(request):
-    """Runs a test under each of the kernel's two code-to-bf16 conversions."""
-    lm.set_nvfp4_conversion(request.param)
-    yield request.param
-    lm.set_nvfp4_conversion(0)
+    """Runs a test under each of the kernel's two code-to-bf16 conversions (the knob lives in the
+    test build of the library, which has the same kernels)."""
+    with lm.test_hooks():
+        lm.set_nvfp4_conversion(request.param)
+        try:
+            yield request.param
+        finally:
+            lm.set_nvfp4_conversion(0)
 
 
 def pack(codes: np.ndarray) -> np.ndarray:
@@ -33,7 +38,7 @@ def pack(codes: np.ndarray) -> np.ndarray:
 def test_tiny_matches_oracle():
     H, V = 256, 1024
     h = synth.hidden(4, H, synth.SEED_TINY)
-    packed, scales, g = synth.nvfp4_weights(V, H, 0.02, synth.SEED_TINY)
+    packed, scales, g = nvfp4_weights(V, H, 0.02, synth.SEED_TINY)
     ref, absum = oracle.logits_w4a16_nvfp4(h, packed, scales, g, 0.25)
     got = gpu_nvfp4(h, packed, scales, g, 0.25)
     assert_bf16_close(got, ref, absum, "nvfp4 tiny")
@@ -82,7 +87,7 @@ def test_integer_valued_sums_are_exact(conversion):
 def test_ragged_shapes_and_global_scale(conversion):
     for rows, H, V, seed in [(1, 64, 1, 1), (17, 128, 129, 2), (65, 320, 300, 3), (300, 64, 200, 4)]:
         h = synth.hidden(rows, H, seed)
-        packed, scales, g = synth.nvfp4_weights(V, H, 0.02, seed)
+        packed, scales, g = nvfp4_weights(V, H, 0.02, seed)
         for alpha in (1.0 / 8, 0.7):
             ref, absum = oracle.logits_w4a16_nvfp4(h, packed, scales, g, alpha)
             got = gpu_nvfp4(h, packed, scales, g, alpha)
@@ -93,7 +98,7 @@ def test_ragged_shapes_and_global_scale(conversion):
 def nvfp4_inputs():
     rows_list, H, V, std, alpha = synth.WORKLOADS["nvfp4"]
     h = synth.hidden(max(rows_list), H, synth.SEED_NVFP4)
-    packed, scales, g = synth.nvfp4_weights(V, H, std, synth.SEED_NVFP4)
+    packed, scales, g = nvfp4_weights(V, H, std, synth.SEED_NVFP4)
     return h, packed, scales, g, dev_u8(packed), dev_u8(scales), rows_list, alpha
 
 
@@ -140,12 +145,52 @@ def test_pair_table_and_spread_give_identical_bits(nvfp4_inputs):
     """The two conversions are the same arithmetic (the table holds exactly the spread words), so
     every row count the table serves must match the spread path bit for bit."""
     h, packed, scales, g, pd, sd, rows_list, alpha = nvfp4_inputs
-    try:
-        for r in (1, 8, 9, 16, 17, 33, 64):
-            lm.set_nvfp4_conversion(1)
-            a = gpu_nvfp4(h[:r], pd, sd, g, alpha)
-            lm.set_nvfp4_conversion(2)
-            b = gpu_nvfp4(h[:r], pd, sd, g, alpha)
-            assert np.array_equal(a, b), r
-    finally:
-        lm.set_nvfp4_conversion(0)
+    with lm.test_hooks():
+        try:
+            for r in (1, 8, 9, 16, 17, 33, 64):
+                lm.set_nvfp4_conversion(1)
+                a = gpu_nvfp4(h[:r], pd, sd, g, alpha)
+                lm.set_nvfp4_conversion(2)
+                b = gpu_nvfp4(h[:r], pd, sd, g, alpha)
+                assert np.array_equal(a, b), r
+        finally:
+            lm.set_nvfp4_conversion(0)
+    # the release library (automatic choice) gives the same bits as well
+    for r in (1, 64):
+        assert np.array_equal(gpu_nvfp4(h[:r], pd, sd, g, alpha), gpu_nvfp4(h[:r], pd, sd, g, alpha))
+
+
+@pytest.mark.parametrize("H", [32, 96, 160, 224, 2080])
+def test_widths_that_are_odd_multiples_of_32(H, conversion):
+    """lm_head_nvfp4_rows_run checks only k = H and lda = H: a width that is a multiple of 32 but
+    not of 64 ends in half a K step of 64 (zero codes and zero scales past H, hidden zero-filled
+    past H, two MMAs of 16 instead of four). Against the oracle, and every row of the smaller
+    calls bit-identical to the same row of the 300-row call (two row tiles)."""
+    V = 517
+    h = synth.hidden(300, H, 50 + H)
+    packed, scales, g = nvfp4_weights(V, H, 0.02, 60 + H)
+    full = gpu_nvfp4(h, packed, scales, g, 0.125)
+    ref, absum = oracle.logits_w4a16_nvfp4(h[:70], packed, scales, g, 0.125)
+    assert_bf16_close(full[:70], ref, absum, f"nvfp4 H={H}")
+    for r in (1, 17, 65, 129):
+        assert np.array_equal(gpu_nvfp4(h[:r], packed, scales, g, 0.125), full[:r]), (H, r)
+
+
+def test_odd_width_integer_sums_are_exact():
+    """Integer-valued inputs at H = 2080 (32 mod 64): every fp32 order is exact, so the kernel
+    must equal the oracle bit for bit -- a dropped or doubled half K step would show."""
+    rng = np.random.default_rng(2080)
+    rows, H, V = 9, 2080, 300
+    codes = rng.integers(0, 16, (V, H)).astype(np.uint8)
+    scales = rng.choice(np.array([0x30, 0x38, 0x40], np.uint8), (V, H // 16))
+    hi = rng.integers(-2, 3, (rows, H)).astype(np.float32)
+    hb = bf16_bits_of_f32(hi)
+    ref, _ = oracle.logits_w4a16_nvfp4(hb, pack(codes), scales, 1.0, 1.0)
+    got = gpu_nvfp4(hb, pack(codes), scales, 1.0, 1.0)
+    assert np.array_equal(got, ref)
+    # the last 32 columns alone: hidden zero elsewhere
+    hz = np.zeros_like(hi)
+    hz[:, H - 32:] = hi[:, H - 32:]
+    hb = bf16_bits_of_f32(hz)
+    ref, _ = oracle.logits_w4a16_nvfp4(hb, pack(codes), scales, 1.0, 1.0)
+    assert np.array_equal(gpu_nvfp4(hb, pack(codes), scales, 1.0, 1.0), ref)

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import fp32_accumulate_lm_b200 as lm
-from fp32_accumulate_lm_b200 import synth
+import synth
 from gpu_helpers import check_status, dev_bf16, gpu_nvfp4
 from tolerance import assert_bf16_close
 
