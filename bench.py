@@ -55,6 +55,8 @@ WORKLOAD_TEXT = {
              "scale, bf16 hidden and logits, alpha=1/8",
     "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
                     "fp32 out, alpha=1/8",
+    "prefill_logprobs_2048": "log-prob mode of the prefill kernel on 2048 rows (profiling case): "
+                             "H=4096, V=151936, bf16 in, alpha=1/8, no logits written",
     "prefill_logprobs": "prefill LM head computing log-probabilities of one target token per row "
                         "(log-softmax in the epilogue, no logits written): rows=8192, H=4096, "
                         "V=151936, bf16 in, fp32 out, alpha=1/8",
@@ -181,6 +183,7 @@ class Workload:
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
                 "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16,
                 "nvfp4_quantize": synth.SEED_NVFP4, "prefill_logprobs": synth.SEED_PREFILL,
+                "prefill_logprobs_2048": synth.SEED_PREFILL,
                 "vocab_parallel_logprobs": synth.SEED_PREFILL}[name]
         rmax = max(rows_list)
         self.quantize = name == "nvfp4_quantize"
@@ -231,7 +234,8 @@ class Workload:
                          for r in rows_list}
         self.hid = {r: self.hidden[:r] for r in rows_list}
         self.general = self.bias is not None or self.dtype != torch.bfloat16  # lmhead_logits_f32
-        self.logprobs = name in ("prefill_logprobs", "vocab_parallel_logprobs")
+        self.logprobs = name in ("prefill_logprobs", "vocab_parallel_logprobs",
+                                 "prefill_logprobs_2048")
         if self.logprobs:
             import fp32_accumulate_lm_b200 as lm
             gen = torch.Generator(device="cpu")
@@ -580,7 +584,7 @@ def _oracle_inputs(name: str, n_rows: int, vslice: int, wl=None) -> dict:
     d["b"] = ((bits(wl.bias[:vslice]) if wl is not None else synth.bias(vslice, synth.SEED_BIAS,
                                                                         dtype=dt))
               if f16 else None)
-    if name in ("prefill_logprobs", "vocab_parallel_logprobs"):
+    if name in ("prefill_logprobs", "vocab_parallel_logprobs", "prefill_logprobs_2048"):
         gen = torch.Generator(device="cpu")
         gen.manual_seed(seed + 700_000)
         d["t"] = torch.randint(0, vslice, (n_rows,), generator=gen, dtype=torch.int32).numpy()

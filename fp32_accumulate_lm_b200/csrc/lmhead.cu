@@ -42,6 +42,10 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 #ifndef LMHEAD_FORCE_NSUB
 #define LMHEAD_FORCE_NSUB 0
 #endif
+// Hidden-row bytes of one row-tile group (build-time knob; see make_sched).
+#ifndef LMHEAD_RGROUP_MB
+#define LMHEAD_RGROUP_MB 32
+#endif
 constexpr CUtensorMapL2promotion kWeightPromo =
     (CUtensorMapL2promotion)(CU_TENSOR_MAP_L2_PROMOTION_NONE + LMHEAD_WEIGHT_L2_PROMOTION);
 
@@ -61,7 +65,7 @@ struct DeviceInfo {
   unsigned long long ctx_id = 0;  // the context the kernel attributes were set in
   int num_sms = 0;
   int smem_optin = 0;        // per-block shared-memory opt-in limit (static + dynamic)
-  int nvfp4_static_smem = 0;  // static shared memory of the NVFP4 kernels
+  int nvfp4_static_smem[2] = {0, 0};  // static shared memory of the NVFP4 kernel <false>, <true>
   int smem_reserved = 0;      // shared memory the system reserves per block
 };
 
@@ -160,8 +164,9 @@ int current_device(DeviceInfo* out) {
         !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<4>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<true>, d.smem_optin,
-                          &d.nvfp4_static_smem) ||
-        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<false>, d.smem_optin, nullptr)) {
+                          &d.nvfp4_static_smem[1]) ||
+        !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<false>, d.smem_optin,
+                          &d.nvfp4_static_smem[0])) {
       return LMHEAD_ERR_LAUNCH;
     }
     d.attrs_set = true;
@@ -265,9 +270,11 @@ int make_sched(int64_t rows, int64_t V, int64_t H, int32_t bn, int num_sms, lmh:
   if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
   s->num_tiles = (int32_t)tiles;
   s->n_vtiles = (int32_t)n_vtiles;
-  // Row tiles per group: their hidden rows within 16 MB (an eighth of L2).
+  // Row tiles per group: their hidden rows within LMHEAD_RGROUP_MB (32 MB, a quarter of L2;
+  // 16 MB read W twice as often at the prefill shape, 64 MB was slower on B200).
   const int64_t tile_hidden_bytes = (int64_t)bn * H * 2;
-  const int64_t rg = (16ll << 20) / (tile_hidden_bytes > 0 ? tile_hidden_bytes : 1);
+  const int64_t rg =
+      ((int64_t)LMHEAD_RGROUP_MB << 20) / (tile_hidden_bytes > 0 ? tile_hidden_bytes : 1);
   s->rgroup = (int32_t)(rg < 1 ? 1 : (rg > s->n_rtiles ? s->n_rtiles : rg));
   *grid = s->num_tiles < num_sms ? s->num_tiles : num_sms;
   return LMHEAD_OK;
@@ -708,19 +715,22 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.hid_rows = rows < p.bn ? (int32_t)((rows + 7) / 8 * 8) : p.bn;
   p.max_stages = lmh::kMaxStages;
   // Dynamic shared memory: all the opt-in room; the kernel lays its ring out in it. The window
-  // holds the reserved block, then the static variables, then the dynamic block.
-  const int dyn_bytes = dev.smem_optin - dev.nvfp4_static_smem;
+  // holds the reserved block, then the kernel's static variables, then the dynamic block.
   const uint32_t stage_bytes = lmh::nvfp4_stage_bytes(p.bn, p.hid_rows);
-  const uint32_t win_base = (uint32_t)(dev.smem_reserved + dev.nvfp4_static_smem);
-  const lmh::StageLayout with_table = lmh::nvfp4_stage_layout(
-      win_base, win_base + (uint32_t)dyn_bytes, stage_bytes, true, lmh::kMaxStages);
-  const lmh::StageLayout spread = lmh::nvfp4_stage_layout(
-      win_base, win_base + (uint32_t)dyn_bytes, stage_bytes, false, lmh::kMaxStages);
+  auto layout = [&](bool table) {
+    const int stat = dev.nvfp4_static_smem[table ? 1 : 0];
+    const uint32_t win_base = (uint32_t)(dev.smem_reserved + stat);
+    return lmh::nvfp4_stage_layout(win_base, win_base + (uint32_t)(dev.smem_optin - stat),
+                                   stage_bytes, table, lmh::kMaxStages);
+  };
+  const lmh::StageLayout with_table = layout(true);
+  const lmh::StageLayout spread = layout(false);
   const int path = g_nvfp4_path.load(std::memory_order_relaxed);
   // The pair table when it leaves room for 3 stages (both conversions give the same bits).
   const bool use_table = path == 1 ? with_table.stages >= 2
                                    : path == 2 ? false : with_table.stages >= 3;
   if ((use_table ? with_table.stages : spread.stages) < 2) return LMHEAD_ERR_SHAPE;
+  const int dyn_bytes = dev.smem_optin - dev.nvfp4_static_smem[use_table ? 1 : 0];
   p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
   // Block scales come by TMA when each scale row is a whole number of 16-byte units, by 4-byte
   // async copies when it is a whole number of words, else by the producer's 2-byte loads.

@@ -394,8 +394,11 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
             ps[0] = (lane & 1) ? __fadd_rn(got, ps[0]) : __fadd_rn(ps[0], got);
           }
           const int64_t row = r0 + c + ((lane >> 1) & 15);
+          // A streaming (evict-first) store, like the logits': with the default priority these
+          // pairs (0.3 GB at the prefill shape) would outrank the evict-first weight tiles in L2
+          // and push them out before the other row tiles of their group read them.
           if ((lane & 1) == 0 && row < p.rows)
-            p.partials[(int64_t)chunk * p.rows + row] = make_float2(pm[0], ps[0]);
+            __stcs(p.partials + (int64_t)chunk * p.rows + row, make_float2(pm[0], ps[0]));
           continue;
         }
         if (v_ok) {

@@ -35,15 +35,16 @@
 //   slot  (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; a ring of 3
 //         slots (2 when the row tile is 128), so refilling a slot never waits for the MMAs
 //         that were just issued.
-// Roles (192 + 128 * kDequantGroups threads):
+// Roles (192 + 128 * kWarpsPerQuarter * kDequantGroups threads):
 //   warp 0      producer: fills stages.
 //   warp 1      TMEM allocator and MMA issuer: per stage waits for its weight slot (filled only
 //               after the dequantisers saw the stage land, so the hidden rows are there too),
 //               16 x tcgen05.mma with A from TMEM, commits free the stage and the slot.
 //   warps 2-5   epilogue.
-//   warps 6-13  dequantisers: two groups of four warps (one per TMEM lane quarter); group g
-//               takes stages g, g + 2, ...; stage i goes to slot i mod slots. Each thread
-//               converts one weight row.
+//   warps 6-    dequantisers: two groups of 4 * kWarpsPerQuarter warps; group g takes stages
+//               g, g + 2, ...; stage i goes to slot i mod slots. In a group, each TMEM lane
+//               quarter has kWarpsPerQuarter warps, which split the stage's 4 K steps between
+//               them; each thread converts one weight row of its K steps.
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -52,13 +53,19 @@ namespace lmh {
 
 // Two dequantiser groups of four warps take stages in turn. The slot ring's phase waits assume
 // no more groups than TMEM weight slots (a group is never two uses of a slot ahead).
+#ifndef LMHEAD_NVFP4_WPQ
+#define LMHEAD_NVFP4_WPQ 2
+#endif
 constexpr int kDequantGroups = 2;
 constexpr int kDequantWarp0 = 6;
-constexpr int kDequantThreads = 128;                    // threads that fill one K step
+constexpr int kWarpsPerQuarter = LMHEAD_NVFP4_WPQ;       // warps per TMEM lane quarter and group
+constexpr int kDequantThreads = 128 * kWarpsPerQuarter;  // threads of one group (one stage)
 constexpr int kNvfp4Threads = 32 * kDequantWarp0 + kDequantThreads * kDequantGroups;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 3;         // dequantised weight slots at the top of TMEM
 static_assert(kDequantGroups <= 2, "the slot ring may have only 2 slots");
+static_assert(kWarpsPerQuarter == 1 || kWarpsPerQuarter == 2 || kWarpsPerQuarter == 4,
+              "the warps of a lane quarter split a stage's 4 K steps evenly");
 constexpr int kBnMax = 128;          // row tile cap: two accumulators of <= 128 columns
 
 constexpr int kRawK = 4;                                  // K steps per stage
@@ -69,6 +76,9 @@ constexpr uint32_t kSlotCols = kRawK * kBK / 2;            // TMEM columns of on
 constexpr int kMaxStages = 8;
 constexpr uint32_t kBarrierBytes = 1024;   // barrier block at the start of dynamic smem
 constexpr uint32_t kPairTableBytes = 65536;  // 256 entries x 256 bytes, on a 64 KB boundary
+// Entry e of the pair table: bytes [0, 128) hold the 32 lanes' copies of the code-pair word e,
+// bytes [128, 256) the 32 lanes' copies of E4M3 scale e as bf16x2 (value * 2^119).
+constexpr uint32_t kScaleTableOffset = 128;
 
 struct Nvfp4HeadParams {
   int64_t rows, H, V;
@@ -352,22 +362,37 @@ __device__ __forceinline__ void dequant8_any(uint32_t x, uint32_t s2, uint32_t l
     dequant8(x, s2, w);
 }
 
+// Block scale k (byte k of `sc`) as bf16x2. With the pair table: from this lane's own copy in
+// the table's second half, so a warp's 32 lookups never share a bank (one prmt builds the
+// address, as for the code pairs). Without it: from the one 256-word table `lut`.
+template <bool kTable>
+__device__ __forceinline__ uint32_t scale_of(uint32_t sc, int k, const uint32_t* lut,
+                                             uint32_t lane_base) {
+  if (kTable) {
+    const uint32_t a = prmt(sc, lane_base + kScaleTableOffset, 0x7604u | ((uint32_t)k << 4));
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+  }
+  return lut[(sc >> (8 * k)) & 0xFFu];
+}
+
 // One K step of one weight row: 64 codes (two 16-byte words) and their four block scales (one
 // byte each in `sc`, low byte first) to 32 bf16x2 words in K order.
 template <bool kTable>
 __device__ __forceinline__ void convert_kstep(const uint4& c0, const uint4& c1, uint32_t sc,
                                               const uint32_t* lut, uint32_t lane_base,
                                               uint32_t (&w)[32]) {
-  const uint32_t s0 = lut[sc & 0xFFu];
+  const uint32_t s0 = scale_of<kTable>(sc, 0, lut, lane_base);
   dequant8_any<kTable>(c0.x, s0, lane_base, w + 0);
   dequant8_any<kTable>(c0.y, s0, lane_base, w + 4);
-  const uint32_t s1 = lut[(sc >> 8) & 0xFFu];
+  const uint32_t s1 = scale_of<kTable>(sc, 1, lut, lane_base);
   dequant8_any<kTable>(c0.z, s1, lane_base, w + 8);
   dequant8_any<kTable>(c0.w, s1, lane_base, w + 12);
-  const uint32_t s2 = lut[(sc >> 16) & 0xFFu];
+  const uint32_t s2 = scale_of<kTable>(sc, 2, lut, lane_base);
   dequant8_any<kTable>(c1.x, s2, lane_base, w + 16);
   dequant8_any<kTable>(c1.y, s2, lane_base, w + 20);
-  const uint32_t s3 = lut[sc >> 24];
+  const uint32_t s3 = scale_of<kTable>(sc, 3, lut, lane_base);
   dequant8_any<kTable>(c1.z, s3, lane_base, w + 24);
   dequant8_any<kTable>(c1.w, s3, lane_base, w + 28);
 }
@@ -379,7 +404,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                               const __grid_constant__ CUtensorMap tmap_h,
                               const Nvfp4HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119
+  __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119 (no table)
   // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
   // counters and descriptors in uniform registers.
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
@@ -446,13 +471,17 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  for (int c = threadIdx.x; c < 256; c += blockDim.x) scale_lut[c] = scale_bf16x2((uint32_t)c);
+  if (!kTable)
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) scale_lut[c] = scale_bf16x2((uint32_t)c);
   if (kTable) {
-    // 256 entries x 32 lane copies; entry e of lane l at table + 256 e + 4 l.
+    // 256 entries x 32 lane copies: code pair e of lane l at table + 256 e + 4 l, scale e of
+    // lane l at table + 256 e + 128 + 4 l.
     uint8_t* table = smem_raw + (L.table - raw);
-    for (int c = threadIdx.x; c < 256 * 32; c += blockDim.x)
-      *reinterpret_cast<uint32_t*>(table + (c >> 5) * 256 + (c & 31) * 4) =
-          pair_entry((uint32_t)c >> 5);
+    for (int c = threadIdx.x; c < 256 * 32; c += blockDim.x) {
+      uint8_t* e = table + (c >> 5) * 256 + (c & 31) * 4;
+      *reinterpret_cast<uint32_t*>(e) = pair_entry((uint32_t)c >> 5);
+      *reinterpret_cast<uint32_t*>(e + kScaleTableOffset) = scale_bf16x2((uint32_t)c >> 5);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -675,12 +704,17 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------------- dequantisers
-    // Group g converts stages g, g + 2, ...; stage i goes to TMEM weight slot i mod slots. Each
-    // thread converts one weight row, 64 elements per K step; the stores of a stage are waited
-    // for once, at its end.
-    const int group = (warp - kDequantWarp0) >> 2;
+    // Group g converts stages g, g + 2, ...; stage i goes to TMEM weight slot i mod slots. In a
+    // group, warp w serves lane quarter w mod 4 and K steps [part * kPer, (part + 1) * kPer) of
+    // each stage, part = its index among the quarter's warps. Each thread converts one weight
+    // row, 64 elements per K step; the stores of a stage are waited for once, at its end.
+    constexpr int kPer = kRawK / kWarpsPerQuarter;  // K steps per warp and stage
+    const int gw = warp - kDequantWarp0;
+    const int group = gw / (4 * kWarpsPerQuarter);
+    const int part = (gw % (4 * kWarpsPerQuarter)) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int j0 = part * kPer;
     const uint32_t sw = (uint32_t)(row & 7);  // 128-byte swizzle of the codes box
     const uint32_t t_slots = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot_col0;
     const uint32_t lane_base = L.table + (uint32_t)lane * 4u;  // pair table only
@@ -700,28 +734,31 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       tc_fence_after_sync();
       const uint8_t* sbase = stage_ptr(st);
       const uint8_t* crow = sbase + off_q + row * 128;
-      const uint4 sc4 = *reinterpret_cast<const uint4*>(sbase + off_s + row * 16);
-      const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(sbase + off_s + row * 16);
+      uint32_t scw[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) scw[j] = srow[j0 + j];
       const uint32_t t_dst = t_slots + (uint32_t)sl * kSlotCols;
-      if (nk == kRawK) {
-        // Whole stage: all eight 16-byte code reads first, so their latency overlaps.
-        uint4 c[2 * kRawK];
+      if (j0 + kPer <= nk) {
+        // All of this warp's K steps: every 16-byte code read first, so their latency overlaps.
+        uint4 c[2 * kPer];
 #pragma unroll
-        for (int h = 0; h < 2 * kRawK; ++h)
-          c[h] = *reinterpret_cast<const uint4*>(crow + (((uint32_t)h ^ sw) << 4));
+        for (int h = 0; h < 2 * kPer; ++h)
+          c[h] = *reinterpret_cast<const uint4*>(crow + (((uint32_t)(2 * j0 + h) ^ sw) << 4));
 #pragma unroll
-        for (int j = 0; j < kRawK; ++j) {
+        for (int j = 0; j < kPer; ++j) {
           uint32_t w[32];
           convert_kstep<kTable>(c[2 * j], c[2 * j + 1], scw[j], scale_lut, lane_base, w);
-          tmem_st_32x32b_x32(t_dst + (uint32_t)j * (kBK / 2), w);
+          tmem_st_32x32b_x32(t_dst + (uint32_t)(j0 + j) * (kBK / 2), w);
         }
       } else {
-        for (int j = 0; j < nk; ++j) {
-          const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2u * j) ^ sw) << 4));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2u * j + 1u) ^ sw) << 4));
+        for (int j = 0; j < kPer && j0 + j < nk; ++j) {
+          const uint32_t h0 = 2u * (uint32_t)(j0 + j);
+          const uint4 c0 = *reinterpret_cast<const uint4*>(crow + ((h0 ^ sw) << 4));
+          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((h0 + 1u) ^ sw) << 4));
           uint32_t w[32];
           convert_kstep<kTable>(c0, c1, scw[j], scale_lut, lane_base, w);
-          tmem_st_32x32b_x32(t_dst + (uint32_t)j * (kBK / 2), w);
+          tmem_st_32x32b_x32(t_dst + (uint32_t)(j0 + j) * (kBK / 2), w);
         }
       }
       mbar_arrive(empty0 + 8 * st);  // this row's codes and scales are in registers
