@@ -56,7 +56,10 @@ namespace lmh {
 #ifndef LMHEAD_NVFP4_WPQ
 #define LMHEAD_NVFP4_WPQ 2
 #endif
-constexpr int kDequantGroups = 2;
+#ifndef LMHEAD_NVFP4_GROUPS
+#define LMHEAD_NVFP4_GROUPS 2
+#endif
+constexpr int kDequantGroups = LMHEAD_NVFP4_GROUPS;  // groups taking stages in turn
 constexpr int kDequantWarp0 = 6;
 constexpr int kWarpsPerQuarter = LMHEAD_NVFP4_WPQ;       // warps per TMEM lane quarter and group
 constexpr int kDequantThreads = 128 * kWarpsPerQuarter;  // threads of one group (one stage)
@@ -74,6 +77,14 @@ constexpr uint32_t kRawScaleBytes = kBM * kRawK * 4;       // 2 KB
 constexpr uint32_t kSlotCols = kRawK * kBK / 2;            // TMEM columns of one weight slot
 
 constexpr int kMaxStages = 8;
+
+// Suspend-time hint of the producer's, MMA issuer's and dequantisers' barrier waits (ns). Every
+// SM sub-partition holds converting dequantiser warps next to warps that wait (the producer, the
+// MMA issuer, the other group): a waiter that spins on try_wait takes issue slots from them.
+#ifndef LMHEAD_NVFP4_WAIT_SLEEP_NS
+#define LMHEAD_NVFP4_WAIT_SLEEP_NS 0
+#endif
+constexpr uint32_t kWaitSleepNs = LMHEAD_NVFP4_WAIT_SLEEP_NS;
 constexpr uint32_t kBarrierBytes = 1024;   // barrier block at the start of dynamic smem
 constexpr uint32_t kPairTableBytes = 65536;  // 256 entries x 256 bytes, on a 64 KB boundary
 // Entry e of the pair table: bytes [0, 128) hold the 32 lanes' copies of the code-pair word e,
@@ -377,24 +388,36 @@ __device__ __forceinline__ uint32_t scale_of(uint32_t sc, int k, const uint32_t*
   return lut[(sc >> (8 * k)) & 0xFFu];
 }
 
+// With the pair table, how many of a K step's eight 4-byte code words go through the table; the
+// others are spread with integer arithmetic. The table costs one shared-memory wavefront per
+// two weights of a warp, the spread none but five ALU instructions; shared-memory bandwidth is
+// what bounds the kernel at decode sizes, so the best split leaves both pipes about equally
+// busy. Both give identical bits.
+#ifndef LMHEAD_NVFP4_TABLE_WORDS
+#define LMHEAD_NVFP4_TABLE_WORDS 8
+#endif
+constexpr int kTableWords = LMHEAD_NVFP4_TABLE_WORDS;
+static_assert(kTableWords >= 0 && kTableWords <= 8, "a K step has 8 code words");
+
 // One K step of one weight row: 64 codes (two 16-byte words) and their four block scales (one
 // byte each in `sc`, low byte first) to 32 bf16x2 words in K order.
 template <bool kTable>
 __device__ __forceinline__ void convert_kstep(const uint4& c0, const uint4& c1, uint32_t sc,
                                               const uint32_t* lut, uint32_t lane_base,
                                               uint32_t (&w)[32]) {
-  const uint32_t s0 = scale_of<kTable>(sc, 0, lut, lane_base);
-  dequant8_any<kTable>(c0.x, s0, lane_base, w + 0);
-  dequant8_any<kTable>(c0.y, s0, lane_base, w + 4);
-  const uint32_t s1 = scale_of<kTable>(sc, 1, lut, lane_base);
-  dequant8_any<kTable>(c0.z, s1, lane_base, w + 8);
-  dequant8_any<kTable>(c0.w, s1, lane_base, w + 12);
-  const uint32_t s2 = scale_of<kTable>(sc, 2, lut, lane_base);
-  dequant8_any<kTable>(c1.x, s2, lane_base, w + 16);
-  dequant8_any<kTable>(c1.y, s2, lane_base, w + 20);
-  const uint32_t s3 = scale_of<kTable>(sc, 3, lut, lane_base);
-  dequant8_any<kTable>(c1.z, s3, lane_base, w + 24);
-  dequant8_any<kTable>(c1.w, s3, lane_base, w + 28);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {  // block scale q covers code words 2q, 2q + 1
+    const uint32_t sq = scale_of<kTable>(sc, q, lut, lane_base);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * q + h;
+      if (kTable && i < kTableWords)
+        dequant8_table(words[i], sq, lane_base, w + 4 * i);
+      else
+        dequant8(words[i], sq, w + 4 * i);
+    }
+  }
 }
 
 template <bool kTable>
@@ -503,7 +526,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     for (int t = 0; ok && t < my_tiles; ++t) {
       const TileCoord tc = sched_tile(p.sched, p.V, t);
       for (int r = 0; r < n_raw; ++r, ++gr) {
-        if (!wait_bounded(empty0 + 8 * st, ph ^ 1u, p.wait, abort_flag)) {
+        if (!wait_bounded(empty0 + 8 * st, ph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
           fail(kRoleProducer, abort_flag);
           ok = false;
           break;
@@ -618,7 +641,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       for (int r = 0; r < n_raw; ++r, ++gr) {
         // The slot is filled only after its dequantisers waited for this stage's loads, so the
         // hidden rows have landed too.
-        if (!wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag)) {
+        if (!wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag, kWaitSleepNs)) {
           fail(kRoleMma, abort_flag);
           ok = false;
           break;
@@ -726,8 +749,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     uint32_t sph = (uint32_t)(group / NA) & 1u;
     for (int gr = group; gr < total_raw; gr += kDequantGroups) {
       const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
-      if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag) ||
-          !wait_bounded(aempty0 + 8 * sl, sph ^ 1u, p.wait, abort_flag)) {
+      if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag, kWaitSleepNs) ||
+          !wait_bounded(aempty0 + 8 * sl, sph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
         fail(kRoleDequant, abort_flag);
         break;
       }
