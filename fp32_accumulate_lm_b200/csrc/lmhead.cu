@@ -713,23 +713,25 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.hid_2d = p.half_tail;
   // Hidden sub-tiles start on 1024-byte swizzle atoms: rows per K step rounded up to 8.
   p.hid_rows = rows < p.bn ? (int32_t)((rows + 7) / 8 * 8) : p.bn;
-  p.max_stages = lmh::kMaxStages;
-  // Dynamic shared memory: all the opt-in room; the kernel lays its ring out in it. The window
+  // Dynamic shared memory: all the opt-in room; the kernel lays its rings out in it. The window
   // holds the reserved block, then the kernel's static variables, then the dynamic block.
-  const uint32_t stage_bytes = lmh::nvfp4_stage_bytes(p.bn, p.hid_rows);
+  const uint32_t hid_bytes = lmh::nvfp4_hid_stage_bytes(p.bn, p.hid_rows);
   auto layout = [&](bool table) {
     const int stat = dev.nvfp4_static_smem[table ? 1 : 0];
     const uint32_t win_base = (uint32_t)(dev.smem_reserved + stat);
-    return lmh::nvfp4_stage_layout(win_base, win_base + (uint32_t)(dev.smem_optin - stat),
-                                   stage_bytes, table, lmh::kMaxStages);
+    uint32_t code[lmh::kMaxCodeStages], hid[lmh::kMaxHidStages];
+    return lmh::nvfp4_layout(win_base, win_base + (uint32_t)(dev.smem_optin - stat), hid_bytes,
+                             table, code, hid);
   };
-  const lmh::StageLayout with_table = layout(true);
-  const lmh::StageLayout spread = layout(false);
+  auto viable = [](const lmh::Nvfp4Layout& L) { return L.n_code >= 2 && L.n_hid >= 2; };
+  const lmh::Nvfp4Layout with_table = layout(true);
+  const lmh::Nvfp4Layout spread = layout(false);
   const int path = g_nvfp4_path.load(std::memory_order_relaxed);
-  // The pair table when it leaves room for 3 stages (both conversions give the same bits).
-  const bool use_table = path == 1 ? with_table.stages >= 2
-                                   : path == 2 ? false : with_table.stages >= 3;
-  if ((use_table ? with_table.stages : spread.stages) < 2) return LMHEAD_ERR_SHAPE;
+  // The pair table when it leaves room for 4 codes stages (both conversions give the same bits).
+  const bool use_table = path == 1   ? viable(with_table)
+                         : path == 2 ? false
+                                     : viable(with_table) && with_table.n_code >= 4;
+  if (!viable(use_table ? with_table : spread)) return LMHEAD_ERR_SHAPE;
   const int dyn_bytes = dev.smem_optin - dev.nvfp4_static_smem[use_table ? 1 : 0];
   p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
   // Block scales come by TMA when each scale row is a whole number of 16-byte units, by 4-byte

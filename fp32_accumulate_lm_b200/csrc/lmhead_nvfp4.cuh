@@ -25,26 +25,31 @@
 //               table, used when the table leaves room for fewer than two stages (large row
 //               tiles).
 //
-// Every hand-off covers 4 K steps (256 elements of K). The single-thread roles (TMA producer,
+// Every hand-off covers 4 K steps (256 elements of K). The single-thread roles (TMA producers,
 // MMA issuer) share their SM sub-partitions with busy dequantiser warps, so each of their
 // instructions is slow; paying one wait and one commit per K step of 64 made them the
-// bottleneck.
-//   stage (shared memory) 4 K steps of: the packed codes [128 rows x 128 bytes] in one box,
-//         their block scales [128 rows x 16 bytes] (TMA when the scale pitch allows, 4-byte
-//         async copies otherwise) and the hidden rows [BN x 64] x 4.
-//   slot  (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; a ring of 3
-//         slots (2 when the row tile is 128), so refilling a slot never waits for the MMAs
-//         that were just issued.
-// Roles (192 + 128 * kWarpsPerQuarter * kDequantGroups threads):
-//   warp 0      producer: fills stages.
-//   warp 1      TMEM allocator and MMA issuer: per stage waits for its weight slot (filled only
-//               after the dequantisers saw the stage land, so the hidden rows are there too),
-//               16 x tcgen05.mma with A from TMEM, commits free the stage and the slot.
+// bottleneck. A stage's two halves live in two shared-memory rings, because they are done with
+// at different times:
+//   codes stage  the packed codes [128 rows x 128 bytes] of 4 K steps in one box, and their
+//                block scales [128 rows x 16 bytes]; free once the dequantisers have read them,
+//                so this ring runs far ahead (up to 8 stages) and keeps the weight stream going.
+//   hidden stage the hidden rows [BN x 64] x 4; free only once the MMAs that read them are done.
+//                At 256 rows a hidden stage is 64 KB: when both halves shared one ring, only 2
+//                stages fitted, and each new stage waited for the MMAs two stages back.
+//   slot         (tensor memory) the dequantised weights of one stage, [128 x 256] bf16; a ring
+//                of 3 slots (2 when the row tile is 128), so refilling a slot never waits for the
+//                MMAs that were just issued.
+// Roles (224 + 128 * kWarpsPerQuarter * kDequantGroups threads):
+//   warp 0      codes producer: fills codes stages.
+//   warp 1      TMEM allocator and MMA issuer: per stage waits for its weight slot and its
+//               hidden stage, 16 x tcgen05.mma with A from TMEM, commits free the hidden stage
+//               and the slot.
 //   warps 2-5   epilogue.
 //   warps 6-    dequantisers: two groups of 4 * kWarpsPerQuarter warps; group g takes stages
 //               g, g + 2, ...; stage i goes to slot i mod slots. In a group, each TMEM lane
 //               quarter has kWarpsPerQuarter warps, which split the stage's 4 K steps between
 //               them; each thread converts one weight row of its K steps.
+//   last warp   hidden producer: fills hidden stages.
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -63,7 +68,8 @@ constexpr int kDequantGroups = LMHEAD_NVFP4_GROUPS;  // groups taking stages in 
 constexpr int kDequantWarp0 = 6;
 constexpr int kWarpsPerQuarter = LMHEAD_NVFP4_WPQ;       // warps per TMEM lane quarter and group
 constexpr int kDequantThreads = 128 * kWarpsPerQuarter;  // threads of one group (one stage)
-constexpr int kNvfp4Threads = 32 * kDequantWarp0 + kDequantThreads * kDequantGroups;
+constexpr int kHidProducerWarp = kDequantWarp0 + kDequantThreads * kDequantGroups / 32;
+constexpr int kNvfp4Threads = 32 * (kHidProducerWarp + 1);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 3;         // dequantised weight slots at the top of TMEM
 static_assert(kDequantGroups <= 2, "the slot ring may have only 2 slots");
@@ -76,7 +82,8 @@ constexpr uint32_t kRawCodeBytes = kBM * kRawK * kBK / 2;  // 16 KB
 constexpr uint32_t kRawScaleBytes = kBM * kRawK * 4;       // 2 KB
 constexpr uint32_t kSlotCols = kRawK * kBK / 2;            // TMEM columns of one weight slot
 
-constexpr int kMaxStages = 8;
+constexpr int kMaxCodeStages = 8;
+constexpr int kMaxHidStages = 4;
 
 // Suspend-time hint of the producer's, MMA issuer's and dequantisers' barrier waits (ns). Every
 // SM sub-partition holds converting dequantiser warps next to warps that wait (the producer, the
@@ -102,7 +109,6 @@ struct Nvfp4HeadParams {
                           // columns past the call's rows read neighbouring data, never stored)
   TileSched sched;
   int32_t num_kb;         // K steps of 64 per tile: ceil(H / 64)
-  int32_t max_stages;     // cap on the shared-memory ring; the kernel fits what room allows
   int32_t slots;          // TMEM weight slots: 3 when 2 * bn + 3 * 128 <= 512, else 2
   int32_t scale_mode;     // block scales: kScaleTma, kScaleAsync4 or kScalePlain (see below)
   int32_t half_tail;      // 1 when H % 64 == 32: the last K step holds 32 elements (2 MMAs)
@@ -119,45 +125,71 @@ constexpr int32_t kScaleAsync4 = 0;
 constexpr int32_t kScaleTma = 1;
 constexpr int32_t kScalePlain = 2;
 
-// Shared-memory stage (4 K steps): [hidden: 4 sub-tiles of hid_rows x 64 bf16, 128-byte swizzle,
-// from one 3-D box, plus room for the last sub-tile's MMA to read bn rows][codes: 128 rows x
-// 128 bytes, 128-byte swizzle][scales: 128 rows x 16 bytes]. Multiples of 1024 bytes.
-__host__ __device__ constexpr uint32_t nvfp4_hid_region_bytes(int bn, int hid_rows) {
+// Shared-memory stages. Codes stage (4 K steps): [codes: 128 rows x 128 bytes, 128-byte
+// swizzle][scales: 128 rows x 16 bytes] = 18 KB. Hidden stage: 4 sub-tiles of hid_rows x 64 bf16,
+// 128-byte swizzle, from one 3-D box, plus room for the last sub-tile's MMA to read bn rows.
+// Both are multiples of 1024 bytes.
+constexpr uint32_t kCodeStageBytes = kRawCodeBytes + kRawScaleBytes;
+__host__ __device__ constexpr uint32_t nvfp4_hid_stage_bytes(int bn, int hid_rows) {
   return (uint32_t)(((kRawK - 1) * hid_rows + bn) * kBK * 2);
 }
-__host__ __device__ constexpr uint32_t nvfp4_stage_bytes(int bn, int hid_rows) {
-  return nvfp4_hid_region_bytes(bn, hid_rows) + kRawCodeBytes + kRawScaleBytes;
-}
 
-// Where the stages go in dynamic shared memory [base, end) (shared-window addresses): after the
-// barrier block; with the pair table, around its 64 KB-aligned block. Host and device use the
-// same arithmetic, the host on the window layout it expects, the kernel on the real one.
-struct StageLayout {
-  uint32_t lo, n_lo;  // first region: start, stages
-  uint32_t hi;        // second region start (pair table only)
-  uint32_t table;     // pair table address (pair table only)
-  int stages;
+// Where everything goes in dynamic shared memory [base, end) (shared-window addresses): the
+// barrier block first; with the pair table, the table on the next 64 KB boundary, which splits
+// the rest into two regions. Hidden stages are placed first, the larger region first: 4, 3 or 2
+// of them, the most that still leaves room for 4 codes stages (else 2); then as many codes stages
+// as fit, at most 8. Host and device use the same arithmetic, the host on the window layout it
+// expects, the kernel on the real one.
+struct Nvfp4Layout {
+  uint32_t bars;   // barrier block (kBarrierBytes)
+  uint32_t table;  // pair table, or 0
+  int n_code, n_hid;
 };
-__host__ __device__ inline StageLayout nvfp4_stage_layout(uint32_t base, uint32_t end,
-                                                          uint32_t stage_bytes, bool pair_table,
-                                                          int max_stages) {
-  StageLayout L;
-  const uint32_t a0 = ((base + 1023u) & ~1023u) + kBarrierBytes;
-  L.lo = a0;
+// Writes the stage addresses to code[kMaxCodeStages] and hid[kMaxHidStages] (the kernel passes
+// its shared arrays, the host local ones).
+__host__ __device__ inline Nvfp4Layout nvfp4_layout(uint32_t base, uint32_t end,
+                                                    uint32_t hid_bytes, bool pair_table,
+                                                    uint32_t* code, uint32_t* hid) {
+  Nvfp4Layout L{};
+  L.bars = (base + 1023u) & ~1023u;
+  const uint32_t start = L.bars + kBarrierBytes;
+  uint32_t lo0 = start, hi0, lo1 = start, hi1 = start;
+  int nr = 1;
   if (pair_table) {
-    L.table = (a0 + 0xFFFFu) & ~0xFFFFu;
-    L.hi = L.table + kPairTableBytes;
-    L.n_lo = (L.table - a0) / stage_bytes;
-    const uint32_t n_hi = end > L.hi ? (end - L.hi) / stage_bytes : 0u;
-    L.stages = (int)(L.n_lo + n_hi);
+    L.table = (start + 0xFFFFu) & ~0xFFFFu;
+    hi0 = L.table;
+    lo1 = L.table + kPairTableBytes;
+    hi1 = end > lo1 ? end : lo1;
+    nr = 2;
   } else {
     L.table = 0;
-    L.hi = 0;
-    L.n_lo = end > a0 ? (end - a0) / stage_bytes : 0u;
-    L.stages = (int)L.n_lo;
+    hi0 = end > start ? end : start;
   }
-  if (L.stages > max_stages) L.stages = max_stages;
-  if ((int)L.n_lo > L.stages) L.n_lo = (uint32_t)L.stages;
+  const bool second_first = nr == 2 && hi1 - lo1 > hi0 - lo0;
+  for (int want = kMaxHidStages; want >= 2; --want) {
+    uint32_t cur0 = lo0, cur1 = lo1;
+    int nh = 0, nc = 0;
+    for (int pass = 0; pass < nr; ++pass) {
+      const bool use1 = (pass == 0) == second_first;
+      uint32_t& cur = use1 ? cur1 : cur0;
+      const uint32_t top = use1 ? hi1 : hi0;
+      while (nh < want && cur + hid_bytes <= top) {
+        hid[nh++] = cur;
+        cur += hid_bytes;
+      }
+    }
+    while (nc < kMaxCodeStages && cur0 + kCodeStageBytes <= hi0) {
+      code[nc++] = cur0;
+      cur0 += kCodeStageBytes;
+    }
+    while (nr == 2 && nc < kMaxCodeStages && cur1 + kCodeStageBytes <= hi1) {
+      code[nc++] = cur1;
+      cur1 += kCodeStageBytes;
+    }
+    L.n_hid = nh;
+    L.n_code = nc;
+    if ((nh == want && nc >= 4) || want == 2) break;
+  }
   return L;
 }
 
@@ -428,50 +460,62 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                               const Nvfp4HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119 (no table)
+  __shared__ uint32_t s_code[kMaxCodeStages];  // codes stage addresses (shared window)
+  __shared__ uint32_t s_hid[kMaxHidStages];    // hidden stage addresses
+  __shared__ uint32_t s_layout[4];             // barrier block, table, codes and hidden stages
   // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
   // counters and descriptors in uniform registers.
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const uint32_t hsub = (uint32_t)p.hid_rows * kBK * 2;  // hidden sub-tile stride in a stage
-  const uint32_t stage_bytes = nvfp4_stage_bytes(p.bn, p.hid_rows);
-  const uint32_t off_q = nvfp4_hid_region_bytes(p.bn, p.hid_rows);
-  const uint32_t off_s = off_q + kRawCodeBytes;
-  uint32_t dyn_bytes;
-  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
   const uint32_t raw = smem_u32(smem_raw);
-  const StageLayout L = nvfp4_stage_layout(raw, raw + dyn_bytes, stage_bytes, kTable,
-                                           p.max_stages);
-  const int S = L.stages;
-  if (S < 2) {  // the host sizes calls so this cannot happen; never run a one-stage ring
+  if (threadIdx.x == 0) {
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+    const Nvfp4Layout L = nvfp4_layout(raw, raw + dyn_bytes,
+                                       nvfp4_hid_stage_bytes(p.bn, p.hid_rows), kTable, s_code,
+                                       s_hid);
+    s_layout[0] = L.bars;
+    s_layout[1] = L.table;
+    s_layout[2] = (uint32_t)L.n_code;
+    s_layout[3] = (uint32_t)L.n_hid;
+  }
+  __syncthreads();
+  const int SC = (int)s_layout[2];
+  const int SH = (int)s_layout[3];
+  if (SC < 2 || SH < 2) {  // the host sizes calls so this cannot happen; never run a short ring
     if (threadIdx.x == 0) atomicCAS(&g_lmhead_status, 0u, kStatusNoRoom);
     return;
   }
-  // Stage s: shared-window address, and a generic pointer for the dequantisers' reads.
-  auto stage_addr = [&](int s) -> uint32_t {
-    return (uint32_t)s < L.n_lo ? L.lo + (uint32_t)s * stage_bytes
-                                : L.hi + ((uint32_t)s - L.n_lo) * stage_bytes;
-  };
-  auto stage_ptr = [&](int s) -> const uint8_t* { return smem_raw + (stage_addr(s) - raw); };
+  const uint32_t table_addr = s_layout[1];
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (L.lo - kBarrierBytes - raw));
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + S);
-  const uint32_t afull0 = smem_u32(bars + 2 * S);
-  const uint32_t aempty0 = smem_u32(bars + 2 * S + kMaxSlots);
-  const uint32_t tfull0 = smem_u32(bars + 2 * S + 2 * kMaxSlots);
-  const uint32_t tempty0 = smem_u32(bars + 2 * S + 2 * kMaxSlots + 2);
-  const uint32_t done_bar = smem_u32(bars + 2 * S + 2 * kMaxSlots + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kMaxSlots + 5);
+  // Barrier block: codes full / empty [8], hidden full / empty [4], slot full / empty [3],
+  // accumulator full / empty [2], done, then the TMEM address and the abort flag.
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (s_layout[0] - raw));
+  const uint32_t cfull0 = smem_u32(bars);
+  const uint32_t cempty0 = smem_u32(bars + kMaxCodeStages);
+  const uint32_t hfull0 = smem_u32(bars + 2 * kMaxCodeStages);
+  const uint32_t hempty0 = smem_u32(bars + 2 * kMaxCodeStages + kMaxHidStages);
+  const uint32_t afull0 = smem_u32(bars + 2 * kMaxCodeStages + 2 * kMaxHidStages);
+  const uint32_t aempty0 = afull0 + 8 * kMaxSlots;
+  const uint32_t tfull0 = aempty0 + 8 * kMaxSlots;
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t done_bar = tempty0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(
+      bars + 2 * kMaxCodeStages + 2 * kMaxHidStages + 2 * kMaxSlots + 5);
   const int NA = p.slots;
   const uint32_t slot_col0 = kTmemCols - (uint32_t)NA * kSlotCols;  // weight slots at the top
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SC; ++s) {
       // expect_tx arrive (+ 32 producer-lane arrivals when the scales do not come by TMA)
-      mbar_init(full0 + 8 * s, p.scale_mode == kScaleTma ? 1 : 1 + 32);
-      // the dequantisers have read the codes and the MMAs have read the hidden rows
-      mbar_init(empty0 + 8 * s, kDequantThreads + 1);
+      mbar_init(cfull0 + 8 * s, p.scale_mode == kScaleTma ? 1 : 1 + 32);
+      mbar_init(cempty0 + 8 * s, kDequantThreads);  // the group has read the codes and scales
+    }
+    for (int s = 0; s < SH; ++s) {
+      mbar_init(hfull0 + 8 * s, 1);
+      mbar_init(hempty0 + 8 * s, 1);  // the stage's MMAs are done
     }
     for (int a = 0; a < kMaxSlots; ++a) {
       mbar_init(afull0 + 8 * a, kDequantThreads);
@@ -488,8 +532,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_q);
     if (p.scale_mode == kScaleTma) prefetch_tmap(&tmap_s);
-    prefetch_tmap(&tmap_h);
   }
+  if (warp == kHidProducerWarp && lane == 0) prefetch_tmap(&tmap_h);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -499,7 +543,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   if (kTable) {
     // 256 entries x 32 lane copies: code pair e of lane l at table + 256 e + 4 l, scale e of
     // lane l at table + 256 e + 128 + 4 l.
-    uint8_t* table = smem_raw + (L.table - raw);
+    uint8_t* table = smem_raw + (table_addr - raw);
     for (int c = threadIdx.x; c < 256 * 32; c += blockDim.x) {
       uint8_t* e = table + (c >> 5) * 256 + (c & 31) * 4;
       *reinterpret_cast<uint32_t*>(e) = pair_entry((uint32_t)c >> 5);
@@ -515,10 +559,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   const int n_raw = (p.num_kb + kRawK - 1) / kRawK;  // stages per tile
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+    // ---------------------------------------------------------------- codes producer
     const uint64_t pol_w = l2_policy_weights();
-    const uint64_t pol_h = l2_policy_evict_last();
-    const uint32_t hid_tx = (uint32_t)kRawK * hsub;  // one box: 4 K steps of hid_rows rows
     int gr = 0;  // stages issued so far
     int st = 0;
     uint32_t ph = 0;
@@ -526,34 +568,24 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     for (int t = 0; ok && t < my_tiles; ++t) {
       const TileCoord tc = sched_tile(p.sched, p.V, t);
       for (int r = 0; r < n_raw; ++r, ++gr) {
-        if (!wait_bounded(empty0 + 8 * st, ph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
+        if (!wait_bounded(cempty0 + 8 * st, ph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
           fail(kRoleProducer, abort_flag);
           ok = false;
           break;
         }
         const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
         if (!p.wait.starve_loads) {
-          const uint32_t full = full0 + 8 * st;
-          const uint32_t sbase = stage_addr(st);
+          const uint32_t full = cfull0 + 8 * st;
+          const uint32_t cbase = s_code[st];
+          const uint32_t sbase = cbase + kRawCodeBytes;  // this stage's scales
           if (lane == 0) {
-            // Boxes are counted whole: K steps past H arrive zero-filled. With 2-D hidden boxes
-            // only the stage's nk K steps are loaded.
-            const uint32_t h_tx = p.hid_2d ? (uint32_t)nk * hsub : hid_tx;
+            // Boxes are counted whole: K steps past H arrive zero-filled.
             mbar_arrive_expect_tx(
-                full, kRawCodeBytes + (p.scale_mode == kScaleTma ? kRawScaleBytes : 0u) + h_tx);
-            tma_load_2d(sbase + off_q, &tmap_q, full, tma_x(r * (kRawK * kBK / 2), 1),
-                        (int32_t)tc.v0, pol_w);
+                full, kRawCodeBytes + (p.scale_mode == kScaleTma ? kRawScaleBytes : 0u));
+            tma_load_2d(cbase, &tmap_q, full, tma_x(r * (kRawK * kBK / 2), 1), (int32_t)tc.v0,
+                        pol_w);
             if (p.scale_mode == kScaleTma)
-              tma_load_2d(sbase + off_s, &tmap_s, full, tma_x(r * (kRawK * 4), 1),
-                          (int32_t)tc.v0, pol_w);
-            if (p.hid_2d) {
-              // [hid_rows x 64] boxes of a [rows, H] map: elements past H are zero-filled
-              for (int j = 0; j < nk; ++j)
-                tma_load_2d(sbase + (uint32_t)j * hsub, &tmap_h, full,
-                            tma_x((int64_t)(r * kRawK + j) * kBK * 2, 2), (int32_t)tc.r0, pol_h);
-            } else {
-              tma_load_3d(sbase, &tmap_h, full, 0, (int32_t)tc.r0, r * kRawK, pol_h);
-            }
+              tma_load_2d(sbase, &tmap_s, full, tma_x(r * (kRawK * 4), 1), (int32_t)tc.v0, pol_w);
           }
           if (p.scale_mode == kScaleAsync4) {
             // 4 rows per lane, 4 K steps of 4 bytes each; rows past V and K steps past H copy
@@ -568,7 +600,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                 const uint8_t* src =
                     p.scales +
                     (in ? (tc.v0 + row) * scale_pitch + (int64_t)(r * kRawK + j) * 4 : 0);
-                cp_async_4(sbase + off_s + (uint32_t)(row * 16 + j * 4), src, in ? 4u : 0u);
+                cp_async_4(sbase + (uint32_t)(row * 16 + j * 4), src, in ? 4u : 0u);
               }
             }
             cp_async_arrive_noinc(full);
@@ -594,7 +626,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
             for (int i = 0; i < 4; ++i)
 #pragma unroll
               for (int j = 0; j < kRawK; ++j)
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + off_s +
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase +
                                                              (uint32_t)((lane * 4 + i) * 16 + j * 4)),
                              "r"(word[i][j])
                              : "memory");
@@ -602,7 +634,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           }
         }
         __syncwarp();
-        if (++st == S) {
+        if (++st == SC) {
           st = 0;
           ph ^= 1u;
         }
@@ -610,12 +642,63 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     }
     // Drain: wait for the loads of the last stages issued.
     if (!p.wait.starve_loads) {
-      for (int i = 0; i < (gr < S ? gr : S); ++i) {
+      for (int i = 0; i < (gr < SC ? gr : SC); ++i) {
         if (--st < 0) {
-          st = S - 1;
+          st = SC - 1;
           ph ^= 1u;
         }
-        if (!wait_bounded(full0 + 8 * st, ph, p.wait, nullptr)) {
+        if (!wait_bounded(cfull0 + 8 * st, ph, p.wait, nullptr)) {
+          fail(kRoleDrain, abort_flag);
+          break;
+        }
+      }
+    }
+  } else if (warp == kHidProducerWarp) {
+    // ---------------------------------------------------------------- hidden producer
+    const uint64_t pol_h = l2_policy_evict_last();
+    const uint32_t hid_tx = (uint32_t)kRawK * hsub;  // one box: 4 K steps of hid_rows rows
+    int gr = 0;
+    int st = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int t = 0; ok && t < my_tiles; ++t) {
+      const TileCoord tc = sched_tile(p.sched, p.V, t);
+      for (int r = 0; r < n_raw; ++r, ++gr) {
+        if (!wait_bounded(hempty0 + 8 * st, ph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
+          fail(kRoleProducer, abort_flag);
+          ok = false;
+          break;
+        }
+        const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
+        if (!p.wait.starve_loads && lane == 0) {
+          const uint32_t full = hfull0 + 8 * st;
+          const uint32_t hbase = s_hid[st];
+          // With 2-D hidden boxes only the stage's nk K steps are loaded; the 3-D box is counted
+          // whole (K steps past H arrive zero-filled).
+          mbar_arrive_expect_tx(full, p.hid_2d ? (uint32_t)nk * hsub : hid_tx);
+          if (p.hid_2d) {
+            // [hid_rows x 64] boxes of a [rows, H] map: elements past H are zero-filled
+            for (int j = 0; j < nk; ++j)
+              tma_load_2d(hbase + (uint32_t)j * hsub, &tmap_h, full,
+                          tma_x((int64_t)(r * kRawK + j) * kBK * 2, 2), (int32_t)tc.r0, pol_h);
+          } else {
+            tma_load_3d(hbase, &tmap_h, full, 0, (int32_t)tc.r0, r * kRawK, pol_h);
+          }
+        }
+        __syncwarp();
+        if (++st == SH) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (!p.wait.starve_loads) {
+      for (int i = 0; i < (gr < SH ? gr : SH); ++i) {
+        if (--st < 0) {
+          st = SH - 1;
+          ph ^= 1u;
+        }
+        if (!wait_bounded(hfull0 + 8 * st, ph, p.wait, nullptr)) {
           fail(kRoleDrain, abort_flag);
           break;
         }
@@ -624,8 +707,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t idesc = idesc_bf16_f32(kBM, p.bn);
-    int gr = 0;
-    int st = 0;
+    int hs = 0;  // hidden stage of stage gr, and its phase
+    uint32_t hph = 0;
     int sl = 0;  // weight slot of stage gr, and its phase
     uint32_t sph = 0;
     int acc = 0;
@@ -638,10 +721,9 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn);
-      for (int r = 0; r < n_raw; ++r, ++gr) {
-        // The slot is filled only after its dequantisers waited for this stage's loads, so the
-        // hidden rows have landed too.
-        if (!wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag, kWaitSleepNs)) {
+      for (int r = 0; r < n_raw; ++r) {
+        if (!wait_bounded(afull0 + 8 * sl, sph, p.wait, abort_flag, kWaitSleepNs) ||
+            !wait_bounded(hfull0 + 8 * hs, hph, p.wait, abort_flag, kWaitSleepNs)) {
           fail(kRoleMma, abort_flag);
           ok = false;
           break;
@@ -649,7 +731,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         tc_fence_after_sync();
         {
           const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
-          const uint64_t bdesc0 = sdesc_kmajor_sw128(stage_addr(st));
+          const uint64_t bdesc0 = sdesc_kmajor_sw128(s_hid[hs]);
           const uint32_t a0 = tmem_base + slot_col0 + (uint32_t)sl * kSlotCols;
           // The tile's last K step is half a step when H % 64 == 32: two MMAs, not four (the
           // zero codes past H are never multiplied).
@@ -667,11 +749,14 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                 mma4_bf16_ts_elect(d_tmem, aj, bj, idesc, (r | j) != 0);
             }
           }
-          mma_commit_elect(empty0 + 8 * st);
+          mma_commit_elect(hempty0 + 8 * hs);
           mma_commit_elect(aempty0 + 8 * sl);
         }
         __syncwarp();
-        if (++st == S) st = 0;
+        if (++hs == SH) {
+          hs = 0;
+          hph ^= 1u;
+        }
         if (++sl == NA) {
           sl = 0;
           sph ^= 1u;
@@ -740,24 +825,24 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
     const int j0 = part * kPer;
     const uint32_t sw = (uint32_t)(row & 7);  // 128-byte swizzle of the codes box
     const uint32_t t_slots = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot_col0;
-    const uint32_t lane_base = L.table + (uint32_t)lane * 4u;  // pair table only
+    const uint32_t lane_base = table_addr + (uint32_t)lane * 4u;  // pair table only
     const int total_raw = my_tiles * n_raw;
-    int st = group % S;             // stage and phase of stage index gr, advanced by the group
-    uint32_t ph = (uint32_t)(group / S) & 1u;  // count each iteration (no divisions in the loop)
+    int st = group % SC;            // codes stage and phase of stage index gr, advanced by the
+    uint32_t ph = (uint32_t)(group / SC) & 1u;  // group each iteration (no divisions in the loop)
     int r = group % n_raw;          // stage within its tile
     int sl = group % NA;            // weight slot of stage gr, and its phase
     uint32_t sph = (uint32_t)(group / NA) & 1u;
     for (int gr = group; gr < total_raw; gr += kDequantGroups) {
       const int nk = p.num_kb - r * kRawK < kRawK ? p.num_kb - r * kRawK : kRawK;
-      if (!wait_bounded(full0 + 8 * st, ph, p.wait, abort_flag, kWaitSleepNs) ||
+      if (!wait_bounded(cfull0 + 8 * st, ph, p.wait, abort_flag, kWaitSleepNs) ||
           !wait_bounded(aempty0 + 8 * sl, sph ^ 1u, p.wait, abort_flag, kWaitSleepNs)) {
         fail(kRoleDequant, abort_flag);
         break;
       }
       tc_fence_after_sync();
-      const uint8_t* sbase = stage_ptr(st);
-      const uint8_t* crow = sbase + off_q + row * 128;
-      const uint32_t* srow = reinterpret_cast<const uint32_t*>(sbase + off_s + row * 16);
+      const uint8_t* sbase = smem_raw + (s_code[st] - raw);
+      const uint8_t* crow = sbase + row * 128;
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(sbase + kRawCodeBytes + row * 16);
       uint32_t scw[kPer];
 #pragma unroll
       for (int j = 0; j < kPer; ++j) scw[j] = srow[j0 + j];
@@ -784,7 +869,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
           tmem_st_32x32b_x32(t_dst + (uint32_t)(j0 + j) * (kBK / 2), w);
         }
       }
-      mbar_arrive(empty0 + 8 * st);  // this row's codes and scales are in registers
+      mbar_arrive(cempty0 + 8 * st);  // this row's codes and scales are in registers
       tmem_st_wait();
       tc_fence_before_sync();
       mbar_arrive(afull0 + 8 * sl);
@@ -794,8 +879,8 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
         sph ^= 1u;
       }
       st += kDequantGroups;
-      if (st >= S) {
-        st -= S;
+      if (st >= SC) {
+        st -= SC;
         ph ^= 1u;
       }
       r += kDequantGroups;
