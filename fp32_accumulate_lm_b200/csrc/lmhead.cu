@@ -733,7 +733,16 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
                                      : viable(with_table) && with_table.n_code >= 4;
   if (!viable(use_table ? with_table : spread)) return LMHEAD_ERR_SHAPE;
   const int dyn_bytes = dev.smem_optin - dev.nvfp4_static_smem[use_table ? 1 : 0];
-  p.slots = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols ? 3 : 2;
+  // TMEM: three weight slots at the top and two accumulators below them when they fit (row
+  // tiles <= 64), else two slots and two accumulators. (One accumulator and three slots for the
+  // wider tiles was measured slower on B200: the epilogue then no longer overlaps the next tile's
+  // MMAs, 153 -> 189 us at 256 rows; build-time knob LMHEAD_NVFP4_TWO_SLOTS=0.)
+#ifndef LMHEAD_NVFP4_TWO_SLOTS
+#define LMHEAD_NVFP4_TWO_SLOTS 1
+#endif
+  const bool two_acc = 2 * p.bn + 3 * (int)lmh::kSlotCols <= (int)lmh::kTmemCols;
+  p.slots = (LMHEAD_NVFP4_TWO_SLOTS && !two_acc) ? 2 : 3;
+  p.accs = (two_acc || p.slots == 2) ? 2 : 1;
   // Block scales come by TMA when each scale row is a whole number of 16-byte units, by 4-byte
   // async copies when it is a whole number of words, else by the producer's 2-byte loads.
   p.scale_mode = ((H / 16) % 16 == 0 && aligned(w_scales, 16)) ? lmh::kScaleTma

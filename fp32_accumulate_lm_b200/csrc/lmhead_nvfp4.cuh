@@ -109,7 +109,9 @@ struct Nvfp4HeadParams {
                           // columns past the call's rows read neighbouring data, never stored)
   TileSched sched;
   int32_t num_kb;         // K steps of 64 per tile: ceil(H / 64)
-  int32_t slots;          // TMEM weight slots: 3 when 2 * bn + 3 * 128 <= 512, else 2
+  int32_t slots;          // TMEM weight slots (3, or 2 when forced)
+  int32_t accs;           // TMEM accumulators: 2 when 2 * bn + 3 * 128 <= 512 (the epilogue of a
+                          // tile overlaps the next tile's MMAs), else 1
   int32_t scale_mode;     // block scales: kScaleTma, kScaleAsync4 or kScalePlain (see below)
   int32_t half_tail;      // 1 when H % 64 == 32: the last K step holds 32 elements (2 MMAs)
   int32_t hid_2d;         // 1: hidden rows by one 2-D box per K step (needed when H % 64 != 0)
@@ -765,8 +767,10 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       if (!ok) break;
       mma_commit_elect(tfull0 + 8 * acc);
       __syncwarp();
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == p.accs) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     mma_commit_elect(done_bar);
     __syncwarp();
@@ -807,8 +811,10 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
       }
       tc_fence_before_sync();
       mbar_arrive(tempty0 + 8 * acc);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == p.accs) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   } else {
     // ---------------------------------------------------------------- dequantisers
