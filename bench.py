@@ -393,40 +393,54 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     if lm.device_status(clear=True) != 0:
         raise RuntimeError(f"{name}: device status word set during warm-up")
 
+    # The timed region: exactly K steps, bracketed by barrier + synchronize, one CUDA event at
+    # each end on the launching stream (an event between every two calls would add about 3 us to
+    # each call on these GPUs).
     n_ev = args.steps * calls_per_step
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.current_device())
     barrier(world)
     sampler.start()
-    ev[0].record(stream)
-    i = 0
+    e_start.record(stream)
     for _ in range(args.steps):
         for r in rl:
             wl.call(r)
-            i += 1
-            ev[i].record(stream)
+    e_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier(world)
     if lm.device_status(clear=True) != 0:
         raise RuntimeError(f"{name}: device status word set during the timed region")
-    elapsed_ms = ev[0].elapsed_time(ev[n_ev])
-    per_call_ms = [ev[j].elapsed_time(ev[j + 1]) for j in range(n_ev)]
+    elapsed_ms = e_start.elapsed_time(e_end)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
+
+    # Per row count (the detail below the headline): each row count alone, as many calls as the
+    # timed region made of it, between two events.
+    per_row_ms = {}
+    for r in rl:
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            wl.call(r)
+        b.record(stream)
+        torch.cuda.synchronize()
+        per_row_ms[r] = a.elapsed_time(b) / args.steps
+    barrier(world)
 
     # per row count: mean launch duration, algorithmic bytes and flops
     detail = {}
-    tot_bytes = tot_flops = tot_ms = 0.0
-    for k, r in enumerate(rl):
-        ms = per_call_ms[k::calls_per_step]
-        mean_ms = sum(ms) / len(ms)
+    tot_bytes = tot_flops = 0.0
+    for r in rl:
+        mean_ms = per_row_ms[r]
         b, fl = wl.bytes_of(r), wl.flops_of(r)
-        detail[str(r)] = {"us": round(mean_ms * 1e3, 2), "us_min": round(min(ms) * 1e3, 2),
+        detail[str(r)] = {"us": round(mean_ms * 1e3, 2),
                           "GBps": round(b / (mean_ms * 1e-3) / 1e9, 1),
                           "TFLOPs": round(fl / (mean_ms * 1e-3) / 1e12, 1)}
         tot_bytes += b
         tot_flops += fl
-        tot_ms += mean_ms
+    # the timed region's mean launch duration (one step = one launch per row count)
+    tot_ms = elapsed_ms / args.steps
     # prefill, its profiling case, log-probs, vocab-parallel log-probs
     tensor_bound = name.startswith("prefill") or wl.vocab_parallel
     if tensor_bound:
