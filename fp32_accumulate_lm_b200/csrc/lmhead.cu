@@ -17,6 +17,7 @@
 #include <atomic>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "lmhead.h"
 #include "lmhead_bf16.cuh"
@@ -176,6 +177,30 @@ int current_device(DeviceInfo* out) {
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#ifndef LMHEAD_PDL
+#define LMHEAD_PDL 1
+#endif
+// Launch a head kernel with programmatic stream serialisation (see pdl_trigger / pdl_wait): the
+// kernel's set-up may overlap the tail of the previous kernel on the stream; its global-memory
+// work still follows it. Returns an lmhead_status.
+template <typename... KArgs, typename... Args>
+int launch_head(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                lmhead_stream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = LMHEAD_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+             ? LMHEAD_OK
+             : LMHEAD_ERR_LAUNCH;
+}
 
 bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
@@ -541,7 +566,11 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   auto kernel = nsub == 4 ? lmh::lmhead_bf16_f32_kernel<4>
                 : nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2>
                             : lmh::lmhead_bf16_f32_kernel<1>;
-  kernel<<<grid, lmh::kHeadThreads, smem, (cudaStream_t)stream>>>(tmap_w, tmap_h, p);
+  st = launch_head(kernel, (unsigned)grid, lmh::kHeadThreads, smem, stream, tmap_w, tmap_h, p);
+  if (st != LMHEAD_OK) {
+    (void)cudaGetLastError();
+    return st;
+  }
   if (lp != nullptr) {
     const int64_t blocks = (rows + lmh::kCombineRows - 1) / lmh::kCombineRows;
     lmh::lmhead_logprob_combine_kernel<<<(unsigned)blocks, 1024, 0, (cudaStream_t)stream>>>(
@@ -771,13 +800,12 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
     st = encode_hidden_ksteps(&tmap_h, hidden, rows, H, (uint32_t)p.hid_rows, lmh::kRawK);
   if (st != LMHEAD_OK) return st;
 
-  if (use_table)
-    lmh::lmhead_w4a16_nvfp4_kernel<true><<<grid, lmh::kNvfp4Threads, (size_t)dyn_bytes,
-                                            (cudaStream_t)stream>>>(tmap_q, tmap_s, tmap_h, p);
-  else
-    lmh::lmhead_w4a16_nvfp4_kernel<false><<<grid, lmh::kNvfp4Threads, (size_t)dyn_bytes,
-                                             (cudaStream_t)stream>>>(tmap_q, tmap_s, tmap_h, p);
-  return cudaGetLastError() == cudaSuccess ? LMHEAD_OK : LMHEAD_ERR_LAUNCH;
+  st = launch_head(use_table ? lmh::lmhead_w4a16_nvfp4_kernel<true>
+                             : lmh::lmhead_w4a16_nvfp4_kernel<false>,
+                   (unsigned)grid, lmh::kNvfp4Threads, (size_t)dyn_bytes, stream, tmap_q, tmap_s,
+                   tmap_h, p);
+  if (st != LMHEAD_OK) (void)cudaGetLastError();
+  return st;
 }
 
 }  // extern "C"

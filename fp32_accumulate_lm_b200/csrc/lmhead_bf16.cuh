@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     lmhead_bf16_f32_kernel(const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ CUtensorMap tmap_h, const Bf16HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
+  if (threadIdx.x == 0) pdl_trigger();
   uint8_t* smem = align_up_1024(smem_raw);
   // Broadcast from lane 0 so the compiler can prove role branches warp-uniform and keep their
   // counters and descriptors in uniform registers.
@@ -195,6 +196,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  pdl_wait();  // from here on global memory: earlier kernels of the stream are done
   const uint32_t tmem_base = *tmem_slot;
   const int my_tiles = sched_count(p.sched);
 

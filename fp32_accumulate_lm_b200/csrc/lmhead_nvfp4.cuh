@@ -461,6 +461,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
                               const __grid_constant__ CUtensorMap tmap_h,
                               const Nvfp4HeadParams p) {
   extern __shared__ uint8_t smem_raw[];
+  if (threadIdx.x == 0) pdl_trigger();
   __shared__ uint32_t scale_lut[256];  // E4M3 code -> bf16x2 of its value * 2^119 (no table)
   __shared__ uint32_t s_code[kMaxCodeStages];  // codes stage addresses (shared window)
   __shared__ uint32_t s_hid[kMaxHidStages];    // hidden stage addresses
@@ -555,6 +556,7 @@ __global__ void __launch_bounds__(kNvfp4Threads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  pdl_wait();  // from here on global memory: earlier kernels of the stream are done
   const uint32_t tmem_base = *tmem_slot;
   const int64_t scale_pitch = p.H / 16;
   const int my_tiles = sched_count(p.sched);

@@ -25,6 +25,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A head kernel launched with programmatic stream serialisation lets the next kernel of the
+// stream start its on-chip set-up on the SMs it has already left (pdl_trigger at entry), and
+// itself touches global memory only after every earlier kernel of the stream has finished and
+// its writes are visible (pdl_wait, by every thread, after the set-up).
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
