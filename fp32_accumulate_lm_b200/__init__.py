@@ -83,6 +83,9 @@ def _bind(lib, test: bool):
     lib.lmhead_logprobs_shard_stats_f32.restype = i32
     lib.lmhead_logprobs_merge_shards.argtypes = [vp, i64, i64, vp, vp, vp]
     lib.lmhead_logprobs_merge_shards.restype = i32
+    lib.lmhead_logits_vocab_slice_f32.argtypes = [vp, i32, i64, i64, vp, i64, i64, f32, vp,
+                                                  ctypes.POINTER(vp), i32, i64, vp]
+    lib.lmhead_logits_vocab_slice_f32.restype = i32
     lib.lmhead_logits_w4a16_nvfp4.argtypes = [vp, i64, i64, vp, vp, f32, i64, f32, vp, vp]
     lib.lmhead_logits_w4a16_nvfp4.restype = i32
     lib.lmhead_nvfp4_quantize_workspace_bytes.argtypes = []
@@ -104,6 +107,8 @@ def _bind(lib, test: bool):
         lib.lmhead_debug_set_fault_injection.restype = None
         lib.lmhead_debug_set_nvfp4_conversion.argtypes = [i32]
         lib.lmhead_debug_set_nvfp4_conversion.restype = None
+        lib.lmhead_debug_set_cta_pairs.argtypes = [i32]
+        lib.lmhead_debug_set_cta_pairs.restype = None
     return lib
 
 
@@ -193,6 +198,18 @@ def lmhead_logprobs_merge_shards(stats_ptr: int, shards: int, rows: int, logprob
                                  lse_ptr: int, stream: int = 0) -> int:
     return _active().lmhead_logprobs_merge_shards(stats_ptr, shards, rows, logprobs_ptr,
                                                        lse_ptr or None, stream)
+
+
+def lmhead_logits_vocab_slice_f32(hidden_ptr: int, dtype: int, rows: int, H: int,
+                                  w_slice_ptr: int, V_slice: int, v_begin: int, alpha: float,
+                                  bias_slice_ptr: int, logits_ptrs, ld_logits: int,
+                                  stream: int = 0) -> int:
+    """logits_ptrs: a sequence of device addresses (ints); passed as a host array."""
+    n = len(logits_ptrs)
+    arr = (ctypes.c_void_p * max(n, 1))(*[p or None for p in logits_ptrs])
+    return _active().lmhead_logits_vocab_slice_f32(
+        hidden_ptr, dtype, rows, H, w_slice_ptr, V_slice, v_begin, alpha, bias_slice_ptr or None,
+        arr if n else None, n, ld_logits, stream)
 
 
 def lmhead_logits_w4a16_nvfp4(hidden_ptr: int, rows: int, H: int, packed_ptr: int,
@@ -292,6 +309,13 @@ def set_nvfp4_conversion(path: int) -> None:
     (the same bits either way)."""
     _require_test_build("set_nvfp4_conversion")
     _active().lmhead_debug_set_nvfp4_conversion(int(path))
+
+
+def set_cta_pairs(enabled: bool) -> None:
+    """Test build only (inside ``test_hooks()``): whether the fp32 head may run full 256-row
+    tiles on CTA pairs (the default) or keeps every tile on one CTA (the same bits either way)."""
+    _require_test_build("set_cta_pairs")
+    _active().lmhead_debug_set_cta_pairs(1 if enabled else 0)
 
 
 def set_fault_injection(starve_loads: bool, wait_limit_ns: int = 0) -> None:
@@ -527,6 +551,91 @@ def logprobs_vocab_parallel(hidden, W_shard, v_begin: int, targets, alpha: float
     with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
         gathered = gather_shard_stats(stats, group)
     return logprobs_merge_shards(gathered, out=out, stream=stream, check=check)
+
+
+def logits_vocab_slice_f32(hidden, W_slice, v_begin: int, outs, alpha: float = 1.0,
+                           bias_slice=None, stream=None, check: bool = False):
+    """Write this GPU's slice of the fp32 logits, alpha * (hidden @ W_slice^T + bias_slice), into
+    columns [v_begin, v_begin + V_slice) of every fp32 [>= rows, ld] tensor in ``outs`` (at most
+    8; this GPU's own buffer and peers' buffers mapped for peer access alike). Nothing else of
+    them is written. Returns ``outs``."""
+    import torch
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}.get(hidden.dtype)
+    _check(dt is not None and W_slice.dtype == hidden.dtype,
+           "bf16 or fp16 operands of one dtype required")
+    _check(hidden.dim() == 2 and W_slice.dim() == 2 and hidden.shape[1] == W_slice.shape[1],
+           "shape mismatch")
+    _check(hidden.is_cuda and W_slice.is_cuda and hidden.is_contiguous()
+           and W_slice.is_contiguous(), "contiguous CUDA tensors required")
+    rows, H = hidden.shape
+    V_slice = W_slice.shape[0]
+    if bias_slice is not None:
+        _check(bias_slice.dtype == hidden.dtype and bias_slice.is_cuda
+               and bias_slice.is_contiguous() and tuple(bias_slice.shape) == (V_slice,),
+               "bias_slice must be a contiguous [V_slice] tensor of the dtype")
+    outs = list(outs)
+    _check(1 <= len(outs) <= 8, "between 1 and 8 output buffers")
+    ld = outs[0].shape[1] if outs[0].dim() == 2 else -1
+    for o in outs:
+        _check(o.dtype == torch.float32 and o.is_cuda and o.is_contiguous() and o.dim() == 2
+               and o.shape[1] == ld and o.shape[0] >= rows,
+               "outs must be contiguous fp32 CUDA tensors [>= rows, ld] of one width")
+    _check(v_begin >= 0 and v_begin + V_slice <= ld, "the slice's columns must fit the buffers")
+    st = lmhead_logits_vocab_slice_f32(
+        hidden.data_ptr(), dt, rows, H, W_slice.data_ptr(), V_slice, int(v_begin), float(alpha),
+        0 if bias_slice is None else bias_slice.data_ptr(), [o.data_ptr() for o in outs], ld,
+        _stream_handle(stream))
+    _finish(st, "lmhead_logits_vocab_slice_f32", check, stream)
+    return outs
+
+
+class VocabParallelLogits:
+    """fp32 logits [rows, V] of a vocab-parallel head on every rank of ``group``: rank r holds
+    W[v_begin, v_begin + V_shard) with (v_begin, V_shard) = vocab_shard(V, world, r), and the
+    same hidden rows. Each rank's head kernel stores its slice into every rank's logits buffer
+    (symmetric memory, peer stores over NVLink), between two barriers across the ranks; there is
+    no separate gather pass. The buffers hold ``max_rows`` rows; a call returns a view of this
+    rank's buffer, valid until the next call. Without a process group (or with one rank) the
+    call is lmhead_logits_f32 into a local buffer."""
+
+    def __init__(self, max_rows: int, V: int, group=None, device=None):
+        import torch
+        import torch.distributed as dist
+        multi = dist.is_initialized() and dist.get_world_size(group) > 1
+        self.world = dist.get_world_size(group) if multi else 1
+        self.rank = dist.get_rank(group) if multi else 0
+        self.V, self.max_rows = int(V), int(max_rows)
+        self.v_begin, self.V_shard = vocab_shard(self.V, self.world, self.rank)
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self._handle = None
+        if multi:
+            import torch.distributed._symmetric_memory as symm_mem
+            self.buffer = symm_mem.empty((self.max_rows, self.V), dtype=torch.float32,
+                                         device=device)
+            self._handle = symm_mem.rendezvous(self.buffer, group or dist.group.WORLD)
+            self._peers = [self._handle.get_buffer(r, (self.max_rows, self.V), torch.float32)
+                           for r in range(self.world)]
+        else:
+            self.buffer = torch.empty((self.max_rows, self.V), dtype=torch.float32,
+                                      device=device)
+            self._peers = [self.buffer]
+
+    def __call__(self, hidden, W_shard, alpha: float = 1.0, bias_shard=None, stream=None,
+                 check: bool = False):
+        import torch
+        rows = hidden.shape[0]
+        _check(rows <= self.max_rows, f"at most {self.max_rows} rows")
+        _check(W_shard.dim() == 2 and W_shard.shape[0] == self.V_shard,
+               f"rank {self.rank} holds {self.V_shard} vocab rows")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            if self._handle is not None:
+                self._handle.barrier(channel=0)   # every rank is done reading the last logits
+            logits_vocab_slice_f32(hidden, W_shard, self.v_begin, self._peers, alpha,
+                                   bias_slice=bias_shard, stream=s, check=check)
+            if self._handle is not None:
+                self._handle.barrier(channel=0)   # every slice has landed in every buffer
+        return self.buffer[:rows]
 
 
 def logits_w4a16_nvfp4(hidden, w_packed, w_scales, w_global_scale: float, alpha: float = 1.0,

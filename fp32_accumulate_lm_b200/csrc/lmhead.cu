@@ -43,6 +43,10 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 #ifndef LMHEAD_FORCE_NSUB
 #define LMHEAD_FORCE_NSUB 0
 #endif
+// 256-row tiles of the bf16 head on CTA pairs (cta_group::2 MMAs): 1 on, 0 off (build-time knob).
+#ifndef LMHEAD_PAIR
+#define LMHEAD_PAIR 1
+#endif
 // Hidden-row bytes of one row-tile group (build-time knob; see make_sched).
 #ifndef LMHEAD_RGROUP_MB
 #define LMHEAD_RGROUP_MB 32
@@ -52,6 +56,7 @@ constexpr CUtensorMapL2promotion kWeightPromo =
 
 std::atomic<int> g_starve_loads{0};
 std::atomic<int> g_nvfp4_path{0};  // 0: automatic, 1: pair table, 2: spread (test hook)
+std::atomic<int> g_no_cta_pairs{0};  // 1: the bf16 head runs 256-row tiles on lone CTAs (test hook)
 std::atomic<uint64_t> g_wait_limit_ns{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -68,6 +73,7 @@ struct DeviceInfo {
   int smem_optin = 0;        // per-block shared-memory opt-in limit (static + dynamic)
   int nvfp4_static_smem[2] = {0, 0};  // static shared memory of the NVFP4 kernel <false>, <true>
   int smem_reserved = 0;      // shared memory the system reserves per block
+  int pair_clusters = 0;      // CTA pairs of the bf16 head that fit the device at once (0: none)
 };
 
 using CtxGetCurrentFn = CUresult (*)(CUcontext*);
@@ -161,14 +167,38 @@ int current_device(DeviceInfo* out) {
     d.ctx_id = ctx;
   }
   if (!d.attrs_set) {
-    if (!raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1>, d.smem_optin, nullptr) ||
-        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2>, d.smem_optin, nullptr) ||
-        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<4>, d.smem_optin, nullptr) ||
+    if (!raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1, false>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2, false>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<4, false>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<1, true>, d.smem_optin, nullptr) ||
+        !raise_smem_limit(lmh::lmhead_bf16_f32_kernel<2, true>, d.smem_optin, nullptr) ||
         !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<true>, d.smem_optin,
                           &d.nvfp4_static_smem[1]) ||
         !raise_smem_limit(lmh::lmhead_w4a16_nvfp4_kernel<false>, d.smem_optin,
                           &d.nvfp4_static_smem[0])) {
       return LMHEAD_ERR_LAUNCH;
+    }
+    // How many CTA pairs fit at once with a whole SM's shared memory each: a pair must sit in
+    // one GPC, so this can be below half the SM count.
+    d.pair_clusters = 0;
+    if (LMHEAD_PAIR) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(d.num_sms & ~1));
+      cfg.blockDim = dim3(lmh::kHeadThreads);
+      cfg.dynamicSmemBytes = (size_t)d.smem_optin;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, lmh::lmhead_bf16_f32_kernel<2, true>, &cfg) ==
+          cudaSuccess)
+        d.pair_clusters = n;
+      else
+        (void)cudaGetLastError();
     }
     d.attrs_set = true;
   }
@@ -184,19 +214,24 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // Launch a head kernel with programmatic stream serialisation (see pdl_trigger / pdl_wait): the
 // kernel's set-up may overlap the tail of the previous kernel on the stream; its global-memory
 // work still follows it. Returns an lmhead_status.
+// `cluster` = 2 launches the grid as CTA pairs (clusters of two along x).
 template <typename... KArgs, typename... Args>
 int launch_head(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
-                lmhead_stream_t stream, Args&&... args) {
+                lmhead_stream_t stream, unsigned cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = (cudaStream_t)stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = LMHEAD_PDL;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
              ? LMHEAD_OK
              : LMHEAD_ERR_LAUNCH;
@@ -285,12 +320,15 @@ uint32_t tmem_cols_for(int32_t bn) {
 
 constexpr int kInt32Max = 0x7fffffff;
 
-// Tile ownership (see TileSched) and grid size: one persistent CTA per SM at most.
-int make_sched(int64_t rows, int64_t V, int64_t H, int32_t bn, int num_sms, lmh::TileSched* s,
-               int* grid) {
+// Tile ownership (see TileSched) and grid size: one persistent unit (a CTA, or with `pair` a
+// CTA pair) per slot, `units` slots at most.
+int make_sched(int64_t rows, int64_t V, int64_t H, int32_t bn, int pair, int units,
+               lmh::TileSched* s, int* grid) {
   s->bn = bn;
+  s->pair = pair;
   s->n_rtiles = (int32_t)((rows + bn - 1) / bn);
-  const int64_t n_vtiles = (V + lmh::kBM - 1) / lmh::kBM;
+  const int64_t vt_rows = (int64_t)lmh::kBM << pair;
+  const int64_t n_vtiles = (V + vt_rows - 1) / vt_rows;
   const int64_t tiles = (int64_t)s->n_rtiles * n_vtiles;
   if (tiles > kInt32Max) return LMHEAD_ERR_SHAPE;
   s->num_tiles = (int32_t)tiles;
@@ -301,7 +339,7 @@ int make_sched(int64_t rows, int64_t V, int64_t H, int32_t bn, int num_sms, lmh:
   const int64_t rg =
       ((int64_t)LMHEAD_RGROUP_MB << 20) / (tile_hidden_bytes > 0 ? tile_hidden_bytes : 1);
   s->rgroup = (int32_t)(rg < 1 ? 1 : (rg > s->n_rtiles ? s->n_rtiles : rg));
-  *grid = s->num_tiles < num_sms ? s->num_tiles : num_sms;
+  *grid = (s->num_tiles < units ? s->num_tiles : units) << pair;
   return LMHEAD_OK;
 }
 
@@ -426,6 +464,8 @@ void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns) 
 void lmhead_debug_set_nvfp4_conversion(int path) {
   g_nvfp4_path.store(path == 1 || path == 2 ? path : 0);
 }
+
+void lmhead_debug_set_cta_pairs(int enabled) { g_no_cta_pairs.store(enabled ? 0 : 1); }
 #endif
 
 size_t lmhead_nvfp4_quantize_workspace_bytes(void) {
@@ -511,9 +551,18 @@ struct LogprobArgs {
   float* stats;     // vocab-shard mode: per-row (max, sum, target logit) instead of logprobs
 };
 
+// Where the logits of a vocab slice go: columns [v_begin, v_begin + V) of each of n row-major
+// [rows, ld] buffers.
+struct LogitCopies {
+  float* const* bufs;
+  int n;
+  int64_t ld;
+  int64_t v_begin;
+};
+
 int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const void* W, int64_t V,
                  float alpha, const void* bias, float* logits, const LogprobArgs* lp,
-                 lmhead_stream_t stream) {
+                 lmhead_stream_t stream, const LogitCopies* copies = nullptr) {
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != LMHEAD_OK) return st;
@@ -522,7 +571,16 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   p.rows = rows;
   p.H = H;
   p.V = V;
-  p.out = logits;
+  for (int d = 0; d < lmh::kMaxLogitCopies; ++d) p.out[d] = nullptr;
+  if (copies != nullptr) {
+    for (int d = 0; d < copies->n; ++d) p.out[d] = copies->bufs[d] + copies->v_begin;
+    p.n_out = copies->n;
+    p.ld_out = copies->ld;
+  } else {
+    p.out[0] = logits;
+    p.n_out = 1;
+    p.ld_out = V;
+  }
   p.logprob = lp != nullptr ? 1 : 0;
   p.n_chunks = (int32_t)(4 * ((V + lmh::kBM - 1) / lmh::kBM));
   p.partials = lp != nullptr ? reinterpret_cast<float2*>(lp->workspace) : nullptr;
@@ -536,13 +594,26 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   p.alpha = alpha;
   p.fp16 = dtype == LMHEAD_DTYPE_F16 ? 1 : 0;
   p.bn = pick_bn(rows);
+  // Full 256-row tiles of the logits run on CTA pairs: M = 256 vocab rows per MMA, so each CTA
+  // loads its 128 W rows and half the hidden rows per K step (a third less shared-memory fill
+  // per flop). The log-prob modes keep lone CTAs: with pairs they measured slower at 8192 rows,
+  // moving twice the DRAM reads.
+  const int pair = (LMHEAD_PAIR && p.bn == 256 && lp == nullptr && dev.pair_clusters > 0 &&
+                    !g_no_cta_pairs.load(std::memory_order_relaxed))
+                       ? 1
+                       : 0;
+  const int32_t b_rows = p.bn >> pair;  // hidden rows in one CTA's tile
   int grid = 0;
-  st = make_sched(rows, V, H, p.bn, dev.num_sms, &p.sched, &grid);
+  st = make_sched(rows, V, H, p.bn, pair, pair ? dev.pair_clusters : dev.num_sms, &p.sched,
+                  &grid);
   if (st != LMHEAD_OK) return st;
   const int reserve = 1024 + 512;  // alignment slack + barriers
-  const int nsub = pick_nsub(p.bn, dev.smem_optin - reserve);
+  // (pairs: one K sub-tile per stage, six stages; two sub-tiles and three stages measured ~1 %
+  // slower at 2048 and 8192 rows)
+  int nsub = pair && !LMHEAD_FORCE_NSUB ? 1 : pick_nsub(b_rows, dev.smem_optin - reserve);
+  if (pair && nsub > 2) nsub = 2;  // the pair kernel is built for one or two
   p.num_ks = (int32_t)((H + nsub * lmh::kBK - 1) / (nsub * lmh::kBK));
-  p.stage_bytes = (uint32_t)(nsub * (lmh::kBM * lmh::kBK * 2 + p.bn * lmh::kBK * 2));
+  p.stage_bytes = (uint32_t)(nsub * (lmh::kBM * lmh::kBK * 2 + b_rows * lmh::kBK * 2));
   int stages = (dev.smem_optin - reserve) / (int)p.stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return LMHEAD_ERR_SHAPE;
@@ -556,17 +627,20 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   st = encode_rows(&tmap_w, tdt, 2, W, H * 2, V, lmh::kBK * 2,
                    lmh::kBM, CU_TENSOR_MAP_SWIZZLE_128B, kWeightPromo);
   if (st != LMHEAD_OK) return st;
-  p.hid_rows = hid_box_rows(rows, p.bn);
+  p.hid_rows = pair ? b_rows : hid_box_rows(rows, p.bn);
   st = encode_rows(&tmap_h, tdt, 2, hidden, H * 2, rows,
                    lmh::kBK * 2, (uint32_t)p.hid_rows, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (st != LMHEAD_OK) return st;
 
   const size_t smem = (size_t)reserve + (size_t)stages * p.stage_bytes;
-  auto kernel = nsub == 4 ? lmh::lmhead_bf16_f32_kernel<4>
-                : nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2>
-                            : lmh::lmhead_bf16_f32_kernel<1>;
-  st = launch_head(kernel, (unsigned)grid, lmh::kHeadThreads, smem, stream, tmap_w, tmap_h, p);
+  auto kernel = pair ? (nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2, true>
+                                  : lmh::lmhead_bf16_f32_kernel<1, true>)
+                : nsub == 4 ? lmh::lmhead_bf16_f32_kernel<4, false>
+                : nsub == 2 ? lmh::lmhead_bf16_f32_kernel<2, false>
+                            : lmh::lmhead_bf16_f32_kernel<1, false>;
+  st = launch_head(kernel, (unsigned)grid, lmh::kHeadThreads, smem, stream, pair ? 2u : 1u,
+                   tmap_w, tmap_h, p);
   if (st != LMHEAD_OK) {
     (void)cudaGetLastError();
     return st;
@@ -611,6 +685,34 @@ int lmhead_logits_f32(const void* hidden, int dtype, int64_t rows, int64_t H, co
     return LMHEAD_ERR_ALIAS;
   }
   return run_f32_head(hidden, dtype, rows, H, W, V, alpha, bias, logits, nullptr, stream);
+}
+
+int lmhead_logits_vocab_slice_f32(const void* hidden, int dtype, int64_t rows, int64_t H,
+                                  const void* W_slice, int64_t V_slice, int64_t v_begin,
+                                  float alpha, const void* bias_slice, float* const* logits,
+                                  int n_logits, int64_t ld_logits, lmhead_stream_t stream) {
+  int st = check_f32_head_args(hidden, dtype, rows, H, W_slice, V_slice, bias_slice);
+  if (st != LMHEAD_OK) return st;
+  if (n_logits < 1 || n_logits > lmh::kMaxLogitCopies) return LMHEAD_ERR_SHAPE;
+  if (v_begin < 0 || ld_logits < 1 || V_slice > ld_logits - v_begin) return LMHEAD_ERR_SHAPE;
+  // every buffer spans rows * ld_logits floats, which must fit an int64 byte count
+  if (rows > 0 && ld_logits > (INT64_MAX / 4) / rows) return LMHEAD_ERR_SHAPE;
+  if (rows == 0) return LMHEAD_OK;
+  if (logits == nullptr) return LMHEAD_ERR_NULL;
+  const int64_t span = ((rows - 1) * ld_logits + v_begin + V_slice) * 4;  // bytes touched
+  const struct { const void* p; int64_t bytes; } in[3] = {
+      {hidden, rows * H * 2}, {W_slice, V_slice * H * 2}, {bias_slice, bias_slice ? V_slice * 2 : 0}};
+  for (int d = 0; d < n_logits; ++d) {
+    if (logits[d] == nullptr) return LMHEAD_ERR_NULL;
+    if (!aligned(logits[d], 4)) return LMHEAD_ERR_ALIGN;
+    for (const auto& i : in)
+      if (i.p != nullptr && overlaps(logits[d], span, i.p, i.bytes)) return LMHEAD_ERR_ALIAS;
+    for (int e = 0; e < d; ++e)
+      if (overlaps(logits[d], span, logits[e], span)) return LMHEAD_ERR_ALIAS;
+  }
+  const LogitCopies copies{logits, n_logits, ld_logits, v_begin};
+  return run_f32_head(hidden, dtype, rows, H, W_slice, V_slice, alpha, bias_slice, nullptr,
+                      nullptr, stream, &copies);
 }
 
 size_t lmhead_logprobs_workspace_bytes(int64_t rows, int64_t V) {
@@ -735,7 +837,7 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
   p.gscale = w_global_scale;
   p.bn = pick_bn(rows) < lmh::kBnMax ? pick_bn(rows) : lmh::kBnMax;
   int grid = 0;
-  st = make_sched(rows, V, H, p.bn, dev.num_sms, &p.sched, &grid);
+  st = make_sched(rows, V, H, p.bn, 0, dev.num_sms, &p.sched, &grid);
   if (st != LMHEAD_OK) return st;
   p.num_kb = (int32_t)((H + lmh::kBK - 1) / lmh::kBK);
   p.half_tail = (H % lmh::kBK) != 0 ? 1 : 0;  // H % 64 == 32: the last K step is half a step
@@ -802,8 +904,8 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
 
   st = launch_head(use_table ? lmh::lmhead_w4a16_nvfp4_kernel<true>
                              : lmh::lmhead_w4a16_nvfp4_kernel<false>,
-                   (unsigned)grid, lmh::kNvfp4Threads, (size_t)dyn_bytes, stream, tmap_q, tmap_s,
-                   tmap_h, p);
+                   (unsigned)grid, lmh::kNvfp4Threads, (size_t)dyn_bytes, stream, 1u, tmap_q,
+                   tmap_s, tmap_h, p);
   if (st != LMHEAD_OK) (void)cudaGetLastError();
   return st;
 }

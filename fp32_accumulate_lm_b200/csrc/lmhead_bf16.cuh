@@ -34,9 +34,15 @@
 
 namespace lmh {
 
+// Copies of the logits one call can write (the vocab-slice entry: one per GPU of the group).
+constexpr int kMaxLogitCopies = 8;
+
 struct Bf16HeadParams {
   int64_t rows, H, V;
-  float* out;
+  // logits row r, vocab entry v at out[d][r * ld_out + v] for every d < n_out (n_out >= 1)
+  float* out[kMaxLogitCopies];
+  int32_t n_out;
+  int64_t ld_out;
   const uint16_t* bias;  // [V] in the operand type, or null
   float alpha;
   int32_t fp16;          // operands (and bias) are IEEE fp16, else bf16
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kMergeThreads)
   logprobs[row] = __fsub_rn(zt, l);
 }
 
-template <int NSUB>
+template <int NSUB, bool kPair>
 __global__ void __launch_bounds__(kHeadThreads, 1)
     lmhead_bf16_f32_kernel(const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ CUtensorMap tmap_h, const Bf16HeadParams p) {
@@ -157,10 +163,15 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
   const int lane = threadIdx.x & 31;
   const int S = p.stages;
+  // CTA pair: rank 0 (the leader) issues the MMAs and owns the full barriers; both CTAs load
+  // their halves, and both run an epilogue over their own TMEM rows.
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
-  // stage s: [A sub-tile 0 .. NSUB-1, 16 KB each][B sub-tile 0 .. NSUB-1, BN*128 bytes each]
+  // stage s: [A sub-tile 0 .. NSUB-1, 16 KB each][B sub-tile 0 .. NSUB-1, b_sub bytes each]
+  // (a CTA pair: this CTA's 128 W rows and its half of the bn hidden rows)
   constexpr uint32_t a_sub = kBM * kBK * 2;
-  const uint32_t b_sub = (uint32_t)p.bn * kBK * 2;
+  const uint32_t b_sub = (uint32_t)(kPair ? p.bn / 2 : p.bn) * kBK * 2;
   const uint32_t b_tx = (uint32_t)p.hid_rows * kBK * 2;
   uint8_t* stage_base = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
@@ -179,7 +190,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, kEpilogueThreads);
+      // a pair's accumulator is free once both CTAs' epilogues have read their rows
+      mbar_init(tempty0 + 8 * a, (kPair ? 2 : 1) * kEpilogueThreads);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -190,11 +202,20 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     prefetch_tmap(&tmap_h);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (kPair) {
+    cluster_sync_all();  // both CTAs' barriers are initialised before either signals the other's
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   pdl_wait();  // from here on global memory: earlier kernels of the stream are done
   const uint32_t tmem_base = *tmem_slot;
@@ -203,14 +224,16 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     const uint64_t pol_w = l2_policy_weights();
-    const uint64_t pol_h = l2_policy_evict_last();  // hidden rows are re-read per v-tile
+    const uint64_t pol_h = l2_policy_hidden();  // hidden rows are re-read per v-tile
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
     for (int t = 0; ok && t < my_tiles; ++t) {
       const TileCoord tc = sched_tile(p.sched, p.V, t);
-      const uint32_t tx = (uint32_t)NSUB * (a_sub + b_tx);
+      // a pair's full barrier (the leader's) counts both CTAs' bytes
+      const uint32_t tx = (uint32_t)NSUB * (a_sub + b_tx) * (kPair ? 2u : 1u);
+      const int32_t hid_y = (int32_t)(tc.r0 + (kPair ? (int64_t)rank * (p.bn / 2) : 0));
       for (int ks = 0; ks < p.num_ks; ++ks) {
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1u, p.wait, abort_flag)) {
           fail(kRoleProducer, abort_flag);
@@ -221,15 +244,18 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           const uint32_t full = full0 + 8 * stage;
           const uint32_t sa = smem_u32(stage_base + (size_t)stage * p.stage_bytes);
           const uint32_t sb = sa + NSUB * a_sub;
-          mbar_arrive_expect_tx(full, tx);
+          if (leader) mbar_arrive_expect_tx(full, tx);
 #pragma unroll
-          for (int j = 0; j < NSUB; ++j)
-            tma_load_2d(sa + j * a_sub, &tmap_w, full, tma_x((ks * NSUB + j) * kBK * 2, 2),
-                        (int32_t)tc.v0, pol_w);
-#pragma unroll
-          for (int j = 0; j < NSUB; ++j)
-            tma_load_2d(sb + j * b_sub, &tmap_h, full, tma_x((ks * NSUB + j) * kBK * 2, 2),
-                        (int32_t)tc.r0, pol_h);
+          for (int j = 0; j < NSUB; ++j) {
+            const int32_t x = tma_x((ks * NSUB + j) * kBK * 2, 2);
+            if constexpr (kPair) {
+              tma_load_2d_pair(sa + j * a_sub, &tmap_w, full, x, (int32_t)tc.v0, pol_w);
+              tma_load_2d_pair(sb + j * b_sub, &tmap_h, full, x, hid_y, pol_h);
+            } else {
+              tma_load_2d(sa + j * a_sub, &tmap_w, full, x, (int32_t)tc.v0, pol_w);
+              tma_load_2d(sb + j * b_sub, &tmap_h, full, x, hid_y, pol_h);
+            }
+          }
         }
         __syncwarp();
         ++issued;
@@ -239,7 +265,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         }
       }
     }
-    // Drain: wait until every load this CTA issued has landed before the CTA may exit.
+    // Drain: every load this CTA issued must land before the CTA may exit. A lone CTA sees that
+    // on its full barriers. A pair's loads are counted on the leader's full barriers, so both
+    // CTAs wait instead until the MMAs have released every stage they filled (which they do only
+    // after the stage's bytes arrived).
     if (!p.wait.starve_loads) {
       const int outstanding = issued < S ? issued : S;
       for (int i = 0; i < outstanding; ++i) {
@@ -247,7 +276,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           stage = S - 1;
           phase ^= 1u;
         }
-        if (!wait_bounded(full0 + 8 * stage, phase, p.wait, nullptr)) {
+        // the fill's round parity: its completion on full, its release on empty
+        if (!wait_bounded((kPair ? empty0 : full0) + 8 * stage, phase, p.wait, nullptr)) {
           fail(kRoleDrain, abort_flag);
           break;
         }
@@ -255,13 +285,15 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_f16kind_f32(kBM, p.bn, p.fp16 == 0);
+    // (a CTA pair: the leader's warp issues for both CTAs; the other CTA's warp only holds the
+    // pair's TMEM allocation)
+    const uint32_t idesc = idesc_f16kind_f32(kPair ? 2 * kBM : kBM, p.bn, p.fp16 == 0);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = 0; ok && t < my_tiles; ++t) {
+    for (int t = 0; ok && leader && t < my_tiles; ++t) {
       if (!wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, p.wait, abort_flag)) {
         fail(kRoleMma, abort_flag);
         break;
@@ -282,10 +314,20 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
 #pragma unroll
           for (int j = 0; j < NSUB; ++j) {
             // descriptor start addresses are in 16-byte units
-            mma4_bf16_ss_elect(d_tmem, adesc0 + (uint64_t)((j * a_sub) >> 4),
-                               bdesc0 + (uint64_t)((j * b_sub) >> 4), idesc, (ks | j) != 0);
+            const uint64_t ad = adesc0 + (uint64_t)((j * a_sub) >> 4);
+            const uint64_t bd = bdesc0 + (uint64_t)((j * b_sub) >> 4);
+            if constexpr (kPair) {
+              mma4_bf16_ss_pair_elect(d_tmem, ad, bd, idesc, (ks | j) != 0);
+            } else {
+              mma4_bf16_ss_elect(d_tmem, ad, bd, idesc, (ks | j) != 0);
+            }
           }
-          mma_commit_elect(empty0 + 8 * stage);
+          // frees the stage in both CTAs of a pair
+          if constexpr (kPair) {
+            mma_commit_pair_elect(empty0 + 8 * stage, 0x3);
+          } else {
+            mma_commit_elect(empty0 + 8 * stage);
+          }
         }
         __syncwarp();
         if (++stage == S) {
@@ -294,15 +336,26 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         }
       }
       if (!ok) break;
-      mma_commit_elect(tfull0 + 8 * acc);
+      if constexpr (kPair) {
+        mma_commit_pair_elect(tfull0 + 8 * acc, 0x3);
+      } else {
+        mma_commit_elect(tfull0 + 8 * acc);
+      }
       __syncwarp();
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    // Every MMA this warp issued must finish before TMEM is released.
-    mma_commit_elect(done_bar);
-    __syncwarp();
-    if (!wait_bounded(done_bar, 0, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
+    // Every MMA this warp issued must finish before TMEM is released (a pair's other CTA
+    // learns it at the closing cluster barrier).
+    if (leader) {
+      if constexpr (kPair) {
+        mma_commit_pair_elect(done_bar, 0x1);
+      } else {
+        mma_commit_elect(done_bar);
+      }
+      __syncwarp();
+      if (!wait_bounded(done_bar, 0, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
+    }
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -326,7 +379,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         const uint16_t bits = p.bias[v];
         b = p.fp16 ? __half2float(__ushort_as_half(bits)) : __uint_as_float((uint32_t)bits << 16);
       }
-      for (int c = 0; c < p.bn; c += 16) {
+      // (a pair's odd CTA holds no vocab rows of the last v-tile when V % 256 <= 128)
+      for (int c = 0; tc.vrows > 0 && c < p.bn; c += 16) {
         if (r0 + c >= p.rows) break;  // warp-uniform
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c, r);
@@ -404,35 +458,58 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           continue;
         }
         if (v_ok) {
-          float* dst = p.out + (r0 + c) * p.V + v;
-          if (p.bias == nullptr) {
+          float z[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (r0 + c + j < p.rows)
-                __stcs(dst + (int64_t)j * p.V, __fmul_rn(p.alpha, __uint_as_float(r[j])));
-            }
+          for (int j = 0; j < 16; ++j)
+            z[j] = p.bias == nullptr ? __fmul_rn(p.alpha, __uint_as_float(r[j]))
+                                     : __fmul_rn(p.alpha, __fadd_rn(__uint_as_float(r[j]), b));
+          const int64_t off = (r0 + c) * p.ld_out + v;
+          if (p.n_out == 1) {  // warp-uniform
+            float* dst = p.out[0] + off;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (r0 + c + j < p.rows) __stcs(dst + (int64_t)j * p.ld_out, z[j]);
           } else {
+            // every copy of the logits (a vocab slice's columns in each GPU's buffer); the
+            // index into the parameter array stays a constant
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (r0 + c + j < p.rows)
-                __stcs(dst + (int64_t)j * p.V,
-                       __fmul_rn(p.alpha, __fadd_rn(__uint_as_float(r[j]), b)));
+            for (int d = 0; d < kMaxLogitCopies; ++d) {
+              if (d < p.n_out) {  // warp-uniform
+                float* dst = p.out[d] + off;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (r0 + c + j < p.rows) __stcs(dst + (int64_t)j * p.ld_out, z[j]);
+              }
             }
           }
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(tempty0 + 8 * acc);
+      if constexpr (kPair) {
+        mbar_arrive_remote(tempty0 + 8 * acc, 0);  // the leader's barrier, counting both CTAs
+      } else {
+        mbar_arrive(tempty0 + 8 * acc);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (kPair) {
+    // Neither CTA releases the pair's TMEM or exits while the other may still signal its
+    // barriers or the leader's MMAs may still read its tiles.
+    cluster_sync_all();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (kPair) {
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    } else {
+      tmem_dealloc(tmem_base, p.tmem_cols);
+    }
   }
 }
 

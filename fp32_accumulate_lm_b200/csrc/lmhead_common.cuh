@@ -22,8 +22,11 @@
 #ifndef LMHEAD_HID_BOX_EXACT
 #define LMHEAD_HID_BOX_EXACT 1
 #endif
-// Elements per 128-byte row of a TMA box, and the x coordinate of byte offset b in a row.
-
+//   LMHEAD_HIDDEN_L2_POLICY  L2 hint for the fp32 head's hidden-row loads: 1 evict-first,
+//                            2 evict-normal, 3 evict-last
+#ifndef LMHEAD_HIDDEN_L2_POLICY
+#define LMHEAD_HIDDEN_L2_POLICY 3
+#endif
 
 namespace lmh {
 
@@ -88,40 +91,45 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-// Which output tiles a CTA owns. A tile is 128 vocab rows by bn hidden rows. Row tiles come in
-// groups of `rgroup` (whose hidden rows fit comfortably in L2); tiles run group by group, and
-// within a group v-major: t -> (v-tile, row-tile) = (local / rg, group * rgroup + local % rg),
-// rg = the group's row tiles. CTA i of G takes t = i, i + G, i + 2G, ... At any moment the G CTAs
-// work on neighbouring v-tiles of one group: the weight stream stays on few DRAM pages, CTAs
-// share each weight tile through L2, and the group's hidden rows stay in L2 instead of being
-// re-read for every v-tile (at 8192 x 4096 hidden rows, 64 MB, they did not survive the weight
-// and logits streams). With rgroup >= the row tiles there is one group: plain v-major order.
-// (Balanced per-CTA strips of W and splitting the last partial wave into 16-row pieces were both
-// measured slower on B200.) Every tile runs the same MMA chain over K, so the schedule changes no
-// output bit.
+// Which output tiles a CTA owns. A tile is 128 vocab rows by bn hidden rows, or, with `pair`
+// set, 256 vocab rows by bn hidden rows computed by the two CTAs of a cluster (CTA rank k of the
+// pair holds vocab rows [128 k, 128 k + 128) of it). Row tiles come in groups of `rgroup` (whose
+// hidden rows fit comfortably in L2); tiles run group by group, and within a group v-major:
+// t -> (v-tile, row-tile) = (local / rg, group * rgroup + local % rg), rg = the group's row
+// tiles. Unit i of G (a CTA, or a CTA pair) takes t = i, i + G, i + 2G, ... At any moment the G
+// units work on neighbouring v-tiles of one group: the weight stream stays on few DRAM pages,
+// units share each weight tile through L2, and the group's hidden rows stay in L2 instead of
+// being re-read for every v-tile (at 8192 x 4096 hidden rows, 64 MB, they did not survive the
+// weight and logits streams). With rgroup >= the row tiles there is one group: plain v-major
+// order. (Balanced per-CTA strips of W and splitting the last partial wave into 16-row pieces
+// were both measured slower on B200.) Every tile runs the same MMA chain over K, so the
+// schedule changes no output bit.
 struct TileSched {
   int32_t n_rtiles;
   int32_t num_tiles;
   int32_t bn;
   int32_t n_vtiles;
   int32_t rgroup;
+  int32_t pair;  // 1: units are CTA pairs (clusters of 2) and v-tiles 256 vocab rows
 };
 
 struct TileCoord {
-  int64_t v0;     // first vocab row
-  int32_t vrows;  // vocab rows that belong to this tile (<= 128; rows past V are zero-filled)
+  int64_t v0;     // first vocab row of this CTA's part
+  int32_t vrows;  // vocab rows that belong to it (0..128; rows past V are zero-filled)
   int64_t r0;     // first hidden row
 };
 
 __device__ __forceinline__ int sched_count(const TileSched& s) {
-  return blockIdx.x < (unsigned)s.num_tiles
-             ? (int)((s.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x) + 1
-             : 0;
+  const int unit = (int)blockIdx.x >> s.pair;
+  const int units = (int)gridDim.x >> s.pair;
+  return unit < s.num_tiles ? (s.num_tiles - 1 - unit) / units + 1 : 0;
 }
 
 __device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, int i) {
   TileCoord c;
-  const int t = (int)blockIdx.x + i * (int)gridDim.x;
+  const int unit = (int)blockIdx.x >> s.pair;
+  const int units = (int)gridDim.x >> s.pair;
+  const int t = unit + i * units;
   const int per_group = s.n_vtiles * s.rgroup;
   const int g = t / per_group;
   const int local = t - g * per_group;
@@ -129,9 +137,9 @@ __device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, i
   const int rg = left_rt < s.rgroup ? left_rt : s.rgroup;
   const int vt = local / rg;
   const int rt = g * s.rgroup + (local - vt * rg);
-  c.v0 = (int64_t)vt * kBM;
+  c.v0 = ((int64_t)vt << s.pair) * kBM + (int64_t)((int)blockIdx.x & s.pair) * kBM;
   const int64_t left = V - c.v0;
-  c.vrows = (int32_t)(left < kBM ? left : kBM);
+  c.vrows = (int32_t)(left < 0 ? 0 : left < kBM ? left : kBM);
   c.r0 = (int64_t)rt * s.bn;
   return c;
 }
@@ -143,6 +151,16 @@ __device__ __forceinline__ uint64_t l2_policy_weights() {
   return l2_policy_evict_normal();
 #else
   return 0;
+#endif
+}
+
+__device__ __forceinline__ uint64_t l2_policy_hidden() {
+#if LMHEAD_HIDDEN_L2_POLICY == 1
+  return l2_policy_evict_first();
+#elif LMHEAD_HIDDEN_L2_POLICY == 2
+  return l2_policy_evict_normal();
+#else
+  return l2_policy_evict_last();
 #endif
 }
 

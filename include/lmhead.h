@@ -176,6 +176,32 @@ int lmhead_logprobs_merge_shards(const float* stats, int64_t shards, int64_t row
                                  float* logprobs, float* lse, lmhead_stream_t stream);
 
 /*
+ * Vocab-parallel fp32 logits, gathered by the head itself. With the head split as above (each
+ * of g GPUs holds W_slice = W[v_begin, v_begin + V_slice)), the GPU's slice of the logits is
+ * written straight into columns [v_begin, v_begin + V_slice) of every buffer in `logits`:
+ *   logits[d][r * ld_logits + v_begin + v] = z[r, v]      for d < n_logits, v < V_slice,
+ * z the fp32 logits lmhead_logits_f32 would write for the slice (the same bits as those columns
+ * of the whole head's logits: no row's reduction order depends on the split). Nothing else of
+ * a buffer is written. Given every GPU's [rows, V] buffer (this GPU's own, and its peers'
+ * mapped for peer access: symmetric or IPC memory over NVLink), one call per GPU plus a barrier
+ * across the GPUs after it (and before the next call reuses the buffers) is the head and its
+ * all-gather in one pass: each element is stored once into each buffer, by the epilogue that
+ * produced it. The pages gather the sliced logits after the projection ("FP32 LM head skip FP32
+ * cast", `_compute_lm_head` with its VocabParallelEmbedding head); here no second pass exists.
+ *
+ *   hidden, W_slice, bias_slice, dtype, alpha: as lmhead_logits_f32 (V = V_slice)
+ *   logits     host array of n_logits device pointers, 1 <= n_logits <= 8, each 4-byte aligned,
+ *              to a row-major fp32 buffer of at least rows rows of ld_logits floats
+ *   v_begin    >= 0, with v_begin + V_slice <= ld_logits
+ * The buffers must not overlap each other or the inputs. One kernel is enqueued; the library
+ * synchronises nothing across GPUs. Returns an lmhead_status.
+ */
+int lmhead_logits_vocab_slice_f32(const void* hidden, int dtype, int64_t rows, int64_t H,
+                                  const void* W_slice, int64_t V_slice, int64_t v_begin,
+                                  float alpha, const void* bias_slice, float* const* logits,
+                                  int n_logits, int64_t ld_logits, lmhead_stream_t stream);
+
+/*
  * Entry 2: bf16 logits from the W4A16 NVFP4 head.
  *   W[v, k]      = e2m1(code[v, k]) * e4m3(w_scales[v, k / 16])      (exact in bf16)
  *   logits[r, v] = bf16_rn( fl32( fl32(acc[r, v] * w_global_scale) * alpha ) ),
@@ -286,9 +312,14 @@ int lmhead_version(void);
  * into bf16: 1 = the shared-memory pair table whenever it leaves room for two pipeline stages,
  * 2 = integer spreading only, anything else = automatic (the table when it leaves room for
  * three stages). Both give identical bits; the knob lets tests show that.
+ *
+ * lmhead_debug_set_cta_pairs: enabled != 0 (the default) lets the fp32 head run full 256-row
+ * tiles on CTA pairs (cta_group::2 MMAs, 256 vocab rows per tile); 0 keeps every tile on one
+ * CTA. Both give identical bits; the knob lets tests show that.
  */
 void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
 void lmhead_debug_set_nvfp4_conversion(int path);
+void lmhead_debug_set_cta_pairs(int enabled);
 #endif
 
 #ifdef __cplusplus

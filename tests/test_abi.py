@@ -66,7 +66,8 @@ def test_test_knobs_exist_only_in_the_test_build(lib):
     """The fault-injection and conversion knobs are declared for LMHEAD_TEST_HOOKS builds only:
     the release library does not export them, the test build exports them and everything else."""
     knobs = hook_functions()
-    assert set(knobs) == {"lmhead_debug_set_fault_injection", "lmhead_debug_set_nvfp4_conversion"}
+    assert set(knobs) == {"lmhead_debug_set_fault_injection", "lmhead_debug_set_nvfp4_conversion",
+                          "lmhead_debug_set_cta_pairs"}
     release, test = exported(lm.library_path()), exported(_build.TEST_LIB)
     assert not set(knobs) & release
     assert set(knobs) | set(declared_functions()) <= test
@@ -301,3 +302,41 @@ def test_vocab_parallel_wrappers_reject_bad_tensors():
         lm.logprobs_merge_shards(torch.zeros(2, 4, dtype=torch.float32))
     with pytest.raises(ValueError):
         lm.logprobs_merge_shards(torch.zeros(2, 4, 3, dtype=torch.float64))
+
+
+def test_vocab_slice_logits_argument_errors(lib):
+    """lmhead_logits_vocab_slice_f32: 1..8 buffers, the slice's columns inside the row stride,
+    every buffer aligned and apart from the inputs and from each other; all checked before any
+    CUDA call."""
+    f = lm.lmhead_logits_vocab_slice_f32
+    O1, O2 = 0x70000000, 0x78000000
+    args = lambda **kw: dict(dict(h=A16, dt=0, rows=4, H=64, w=B16, V=300, v0=100, alpha=1.0,
+                                  bias=0, outs=[O1, O2], ld=1000), **kw)
+    call = lambda a: f(a["h"], a["dt"], a["rows"], a["H"], a["w"], a["V"], a["v0"], a["alpha"],
+                       a["bias"], a["outs"], a["ld"], 0)
+    assert call(args()) not in (1, 2, 3, 7)                  # valid: reaches the device check
+    assert call(args(outs=[O1])) not in (1, 2, 3, 7)
+    assert call(args(v0=700)) not in (1, 2, 3, 7)            # last column ld - 1
+    assert call(args(v0=701)) == 2                           # one column past ld
+    assert call(args(v0=-1)) == 2
+    assert call(args(ld=0)) == 2
+    assert call(args(outs=[])) == 2                          # no buffer
+    assert call(args(outs=[O1 + 0x100000 * i for i in range(9)])) == 2   # more than 8
+    assert call(args(dt=2)) == 2
+    assert call(args(rows=2 ** 40, ld=2 ** 30)) == 2         # rows * ld * 4 bytes overflows
+    assert call(args(outs=[O1, 0])) == 1
+    assert call(args(outs=[O1, O2 + 2])) == 3
+    assert call(args(outs=[O1, O1 + 4 * 1000])) == 7         # second buffer inside the first
+    assert call(args(outs=[B16 - 64, O2])) == 7              # a buffer over W
+    assert call(args(rows=0, h=0, w=0, outs=[0])) == 0       # rows == 0 launches nothing
+
+
+def test_vocab_parallel_logits_wrappers_reject_bad_tensors():
+    import torch
+    h = torch.zeros(2, 64, dtype=torch.bfloat16)
+    w = torch.zeros(8, 64, dtype=torch.bfloat16)
+    o = torch.zeros(2, 16, dtype=torch.float32)
+    with pytest.raises(ValueError):                      # host tensors
+        lm.logits_vocab_slice_f32(h, w, 0, [o])
+    with pytest.raises(ValueError):                      # no buffer
+        lm.logits_vocab_slice_f32(h, w, 0, [])

@@ -182,3 +182,50 @@ def test_rows_past_the_first_row_tile():
     bound = 2 * merged_bound(lse1.cpu().numpy().astype(np.float64), 1667, 3)
     assert np.all(np.abs(lp - lp1.cpu().numpy()) <= bound)
     assert np.all(np.abs(lse - lse1.cpu().numpy()) <= bound)
+
+
+# ---------------------------------------------------------------- vocab-parallel logits
+
+@pytest.mark.parametrize("rows,g,dtype,with_bias", [(5, 1, "bf16", False), (5, 3, "bf16", True),
+                                                    (300, 4, "bf16", True), (37, 2, "f16", True),
+                                                    (513, 8, "bf16", False)])
+def test_slice_logits_written_into_every_buffer_make_the_whole_head(rows, g, dtype, with_bias):
+    """Each vocab slice's call (one per GPU of a g-way split, here run in turn on one device)
+    stores its columns into every buffer; the buffers, local here, stand for the g GPUs'
+    buffers, which the kernel addresses the same way. Afterwards every buffer holds the whole
+    head's logits bit for bit (lmhead_logits_f32 on all of W), and nothing outside its [rows, V]
+    block was written (NaN canaries in extra rows and in columns past V)."""
+    H, V = 192, 1111
+    (h, w, b, _), (hd, wd, bd, _) = make(rows, H, V, 60 + g, dtype, with_bias)
+    alpha = 0.3
+    ld = V + 13
+    bufs = [torch.full((rows + 3, ld), float("nan"), dtype=torch.float32, device="cuda")
+            for _ in range(min(g, 3))]
+    for b0, n in slices(V, g):
+        lm.logits_vocab_slice_f32(hd, wd[b0:b0 + n].contiguous(), b0, bufs, alpha,
+                                  bias_slice=None if bd is None else bd[b0:b0 + n].contiguous())
+    whole = lm.logits_f32(hd, wd, alpha, bias=bd)
+    check_status()
+    want = whole.cpu().numpy().view(np.uint32)
+    for buf in bufs:
+        got = buf.cpu().numpy()
+        assert np.array_equal(got[:rows, :V].view(np.uint32), want)
+        assert np.isnan(got[:rows, V:]).all() and np.isnan(got[rows:]).all()
+
+
+def test_vocab_parallel_logits_single_rank_and_oracle():
+    """VocabParallelLogits without a process group (one rank holds the whole vocabulary): the
+    one-GPU logits, and on sampled rows the CPU oracle within the fp32 bound."""
+    from tolerance import assert_fp32_close
+    rows, H, V = 260, 256, 3000
+    (h, w, b, _), (hd, wd, bd, _) = make(rows, H, V, 71, "bf16", True)
+    head = lm.VocabParallelLogits(max_rows=512, V=V)
+    assert (head.v_begin, head.V_shard) == (0, V)
+    got = head(hd, wd, 0.25, bias_shard=bd)
+    assert tuple(got.shape) == (rows, V)
+    whole = lm.logits_f32(hd, wd, 0.25, bias=bd)
+    check_status()
+    assert torch.equal(got.view(torch.int32), whole.view(torch.int32))
+    sample = np.array([0, 1, 128, 255, 256, 259])
+    ref, absum = oracle.logits_f32(h[sample], w, 0.25, bias_bits=b)
+    assert_fp32_close(got.cpu().numpy()[sample], ref, absum, "vocab-parallel logits")
