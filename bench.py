@@ -13,6 +13,7 @@ Workloads (seeded synthetic inputs from tests/synth.py; the pages use no dataset
   vocab_parallel_logprobs  the same with W's rows split over the GPUs (see below).
   nvfp4_quantize    the NVFP4 quantiser of a bf16 W [151936, 2048].
   prefill_2048      the prefill kernel on 2048 rows (a small case for profiling).
+  prefill_4608      the same on 4608 rows: two row-tile groups, as at 8192 (profiling).
 Metric: microseconds per LM-head call (lower is better) and the fraction of the roofline the
 kernel reaches. Every call reads a weight matrix larger than L2 (126 MB); two copies of it are
 alternated so no call starts with its weights cached by the previous one.
@@ -55,6 +56,8 @@ WORKLOAD_TEXT = {
              "scale, bf16 hidden and logits, alpha=1/8",
     "prefill_2048": "prefill kernel on 2048 rows (profiling case): H=4096, V=151936, bf16 in, "
                     "fp32 out, alpha=1/8",
+    "prefill_4608": "prefill kernel on 4608 rows (profiling case, two row-tile groups): H=4096, "
+                    "V=151936, bf16 in, fp32 out, alpha=1/8",
     "prefill_logprobs_2048": "log-prob mode of the prefill kernel on 2048 rows (profiling case): "
                              "H=4096, V=151936, bf16 in, alpha=1/8, no logits written",
     "prefill_logprobs": "prefill LM head computing log-probabilities of one target token per row "
@@ -181,7 +184,8 @@ class Workload:
         self.rows_list, self.H, self.V, self.alpha = rows_list, H, V, alpha
         seed = {"decode": synth.SEED_DECODE, "spec_verify": synth.SEED_SPEC,
                 "prefill": synth.SEED_PREFILL, "nvfp4": synth.SEED_NVFP4,
-                "prefill_2048": synth.SEED_PREFILL, "decode_f16_bias": synth.SEED_F16,
+                "prefill_2048": synth.SEED_PREFILL, "prefill_4608": synth.SEED_PREFILL,
+                "decode_f16_bias": synth.SEED_F16,
                 "nvfp4_quantize": synth.SEED_NVFP4, "prefill_logprobs": synth.SEED_PREFILL,
                 "prefill_logprobs_2048": synth.SEED_PREFILL,
                 "vocab_parallel_logprobs": synth.SEED_PREFILL}[name]
@@ -358,6 +362,7 @@ SECONDARY = ["spec_verify", "prefill", "nvfp4", "decode_f16_bias", "prefill_logp
              "vocab_parallel_logprobs", "nvfp4_quantize"]
 # A timed region at least this long is "a long step": the sustained bf16 peak applies.
 SUSTAINED_REGION_S = 1.0
+PER_ROW_IDLE_S = 1.0   # idle before each per-row-count loop (see measure)
 
 
 def config_of(name: str, world: int) -> dict:
@@ -415,9 +420,12 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     elapsed_ms = max_over_ranks(elapsed_ms, world)
 
     # Per row count (the detail below the headline): each row count alone, as many calls as the
-    # timed region made of it, between two events.
+    # timed region made of it, between two events. Each loop starts after PER_ROW_IDLE_S of idle,
+    # so that every row count starts from the same clock state: the loops follow the timed
+    # region, and after tensor-heavy calls the power cap holds the SM clock down for a while.
     per_row_ms = {}
     for r in rl:
+        time.sleep(PER_ROW_IDLE_S)
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)

@@ -48,6 +48,8 @@ WORKLOADS = {
     "decode_f16_bias": ([1, 2, 4, 8, 16, 32, 64], 2048, 151936, 0.02, 1.0 / 8),
     # profiling case: the prefill kernel and tile shape on 2048 rows (a few GB on the device)
     "prefill_2048": ([2048], 4096, 151936, 0.02, 1.0 / 8),
+    # profiling case with two row-tile groups (16 + 2 tiles of 256 rows), as at 8192 rows
+    "prefill_4608": ([4608], 4096, 151936, 0.02, 1.0 / 8),
     # profiling case of the log-prob mode: 2048 rows, one row-tile group
     "prefill_logprobs_2048": ([2048], 4096, 151936, 0.02, 1.0 / 8),
 }
