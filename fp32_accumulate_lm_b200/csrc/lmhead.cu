@@ -47,6 +47,10 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 #ifndef LMHEAD_PAIR
 #define LMHEAD_PAIR 1
 #endif
+// CTA pairs in the log-prob modes too: 1 on, 0 off (build-time knob).
+#ifndef LMHEAD_PAIR_LOGPROB
+#define LMHEAD_PAIR_LOGPROB 0
+#endif
 // Hidden-row bytes of one row-tile group (build-time knob; see make_sched).
 #ifndef LMHEAD_RGROUP_MB
 #define LMHEAD_RGROUP_MB 32
@@ -598,7 +602,8 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   // loads its 128 W rows and half the hidden rows per K step (a third less shared-memory fill
   // per flop). The log-prob modes keep lone CTAs: with pairs they measured slower at 8192 rows,
   // moving twice the DRAM reads.
-  const int pair = (LMHEAD_PAIR && p.bn == 256 && lp == nullptr && dev.pair_clusters > 0 &&
+  const int pair = (LMHEAD_PAIR && p.bn == 256 && (lp == nullptr || LMHEAD_PAIR_LOGPROB) &&
+                    dev.pair_clusters > 0 &&
                     !g_no_cta_pairs.load(std::memory_order_relaxed))
                        ? 1
                        : 0;

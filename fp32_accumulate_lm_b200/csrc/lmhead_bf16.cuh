@@ -14,13 +14,15 @@
 // a handful of decode rows pads N (16..256 in steps of 16), never M, and each TMEM lane holds one
 // vocab entry: the epilogue's 32 lanes of a warp write 32 consecutive logits of one row.
 //
-// Roles (192 threads):
+// Roles (64 + 32 * kBf16EpiWarps threads: 320 with the default 8 epilogue warps):
 //   warp 0     TMA producer: per pipeline stage, NSUB sub-tiles of 64 K-elements each of W
 //              [128 x 64] and of the hidden rows [BN x 64] (128-byte swizzle), landing on full[s].
 //   warp 1     TMEM allocator and MMA issuer: 4 * NSUB tcgen05.mma (K = 16 each) per stage into
 //              one of two TMEM accumulators; tcgen05.commit frees the stage (empty[s]) and, after
 //              the last K step, hands the accumulator to the epilogue (tmem_full[a]).
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, the bias (one IEEE fp32 add) if any, one
+//   warps 2-9  epilogue (two warps per TMEM lane quarter, warp w on quarter w % 4, each taking
+//              every other 16-column chunk; with 4 epilogue warps, warps 2-5 take all chunks):
+//              tcgen05.ld of the accumulator, the bias (one IEEE fp32 add) if any, one
 //              IEEE fp32 multiply by alpha, store. In log-prob mode the logits are not stored:
 //              each warp reduces its 32 vocab entries to (max, sum of exp(z - max)) per row
 //              and writes that pair to the workspace, and the lane holding a row's target token
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
       // a pair's accumulator is free once both CTAs' epilogues have read their rows
-      mbar_init(tempty0 + 8 * a, (kPair ? 2 : 1) * kEpilogueThreads);
+      mbar_init(tempty0 + 8 * a, (kPair ? 2 : 1) * 32 * kBf16EpiWarps);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -359,6 +361,9 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    // with two warps per lane quarter, each takes every other 16-column chunk of the tile
+    const int half = kBf16EpiWarps == 8 ? (warp - 2) >> 2 : 0;
+    constexpr int kChunkStep = kBf16EpiWarps == 8 ? 32 : 16;
     const int v_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
         b = p.fp16 ? __half2float(__ushort_as_half(bits)) : __uint_as_float((uint32_t)bits << 16);
       }
       // (a pair's odd CTA holds no vocab rows of the last v-tile when V % 256 <= 128)
-      for (int c = 0; tc.vrows > 0 && c < p.bn; c += 16) {
+      for (int c = 16 * half; tc.vrows > 0 && c < p.bn; c += kChunkStep) {
         if (r0 + c >= p.rows) break;  // warp-uniform
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c, r);

@@ -38,8 +38,14 @@ __host__ __device__ constexpr int32_t tma_x(int64_t bytes, int esize) {
 constexpr int kBM = 128;   // vocab rows per tile (MMA M)
 constexpr int kBK = 64;    // K elements per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kUK = 16;    // K per tcgen05.mma of kind::f16
-constexpr int kHeadThreads = 192;
-constexpr int kEpilogueThreads = 128;
+// Epilogue warps of the fp32 head (build-time knob): 4 (one per TMEM lane quarter) or 8 (two
+// per lane quarter, each taking every other 16-column chunk of a tile).
+#ifndef LMHEAD_EPI_WARPS
+#define LMHEAD_EPI_WARPS 8
+#endif
+constexpr int kBf16EpiWarps = LMHEAD_EPI_WARPS;
+constexpr int kHeadThreads = 64 + 32 * kBf16EpiWarps;
+constexpr int kEpilogueThreads = 128;  // the NVFP4 head's epilogue
 
 // Which role gave up waiting (bits 8..15 of the status word).
 enum : unsigned {
