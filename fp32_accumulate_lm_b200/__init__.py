@@ -596,19 +596,23 @@ class VocabParallelLogits:
     (symmetric memory, peer stores over NVLink), between two barriers across the ranks; there is
     no separate gather pass. The buffers hold ``max_rows`` rows; a call returns a view of this
     rank's buffer, valid until the next call. Without a process group (or with one rank) the
-    call is lmhead_logits_f32 into a local buffer."""
+    call is lmhead_logits_f32 into a local buffer, unless ``symmetric=True`` asks for the
+    symmetric-memory buffer and barriers anyway (a process group is needed then)."""
 
-    def __init__(self, max_rows: int, V: int, group=None, device=None):
+    def __init__(self, max_rows: int, V: int, group=None, device=None, symmetric=None):
         import torch
         import torch.distributed as dist
-        multi = dist.is_initialized() and dist.get_world_size(group) > 1
-        self.world = dist.get_world_size(group) if multi else 1
-        self.rank = dist.get_rank(group) if multi else 0
+        grouped = dist.is_initialized()
+        multi = grouped and dist.get_world_size(group) > 1
+        self.world = dist.get_world_size(group) if grouped else 1
+        self.rank = dist.get_rank(group) if grouped else 0
         self.V, self.max_rows = int(V), int(max_rows)
         self.v_begin, self.V_shard = vocab_shard(self.V, self.world, self.rank)
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self._handle = None
-        if multi:
+        use_symm = multi if symmetric is None else bool(symmetric)
+        _check(not use_symm or grouped, "symmetric memory needs an initialised process group")
+        if use_symm:
             import torch.distributed._symmetric_memory as symm_mem
             self.buffer = symm_mem.empty((self.max_rows, self.V), dtype=torch.float32,
                                          device=device)

@@ -229,3 +229,31 @@ def test_vocab_parallel_logits_single_rank_and_oracle():
     sample = np.array([0, 1, 128, 255, 256, 259])
     ref, absum = oracle.logits_f32(h[sample], w, 0.25, bias_bits=b)
     assert_fp32_close(got.cpu().numpy()[sample], ref, absum, "vocab-parallel logits")
+
+
+def test_vocab_parallel_logits_on_symmetric_memory_in_a_one_rank_group():
+    """VocabParallelLogits forced onto torch's symmetric memory in a one-rank NCCL group: the
+    rendezvous, the mapping of every rank's buffer and the two barriers around each call run for
+    real, and the buffer holds the one-GPU entry's bits for two calls of different row counts."""
+    import socket
+    from datetime import timedelta
+    import torch.distributed as dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        _, (hd, wd, bd, _) = make(300, 256, 3000, 72, "bf16", True)
+        head = lm.VocabParallelLogits(max_rows=512, V=3000, symmetric=True)
+        assert head._handle is not None and head.world == 1
+        for rows in (300, 5):
+            h = hd[:rows].contiguous()
+            got = head(h, wd, 0.25, bias_shard=bd).clone()
+            want = lm.logits_f32(h, wd, 0.25, bias=bd)
+            check_status()
+            assert torch.equal(got.view(torch.int32), want.view(torch.int32)), rows
+        del head
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
