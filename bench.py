@@ -530,35 +530,68 @@ def run_ours(args) -> dict | None:
 
 def run_e2e(args, wl, world: int) -> dict:
     """Same metric through the public call with host buffers: every call copies its hidden rows
-    from pinned host memory and its logits back to pinned host memory inside the timed region."""
+    from pinned host memory and its result back to pinned host memory inside the timed region,
+    pipelined as a caller would: the copies run on their own streams (host-to-device and
+    device-to-host, so PCIe carries both directions at once) and two sets of buffers alternate,
+    so call i's result travels back while call i + 1 computes. Events order each copy after the
+    work it depends on and keep a buffer from being overwritten before its copy has read it."""
     import torch
-    stream = torch.cuda.current_stream()
+    compute = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     rl = wl.rows_list
     h_host = {r: wl.hid[r].cpu().pin_memory() for r in rl}
-    h_dev = {r: torch.empty_like(wl.hid[r]) for r in rl}
+    h_dev = {r: [torch.empty_like(wl.hid[r]) for _ in range(2)] for r in rl}
+    o_dev = {r: [wl.outs[r], torch.empty_like(wl.outs[r])] for r in rl}
+    # one host buffer per row count: the downloads run in order on one stream
     o_host = {r: torch.empty(wl.outs[r].shape, dtype=wl.outs[r].dtype).pin_memory() for r in rl}
+    ev = lambda: torch.cuda.Event()
+    uploaded = [ev(), ev()]     # hidden rows of the slot are on the device
+    computed = [ev(), ev()]     # the slot's call is done (its hidden rows may be overwritten)
+    downloaded = [ev(), ev()]   # the slot's result is on the host (its buffer may be reused)
+    for e in computed + downloaded:
+        e.record(compute)
+    calls = [0]
+
+    def one_call(r):
+        s = calls[0] & 1
+        calls[0] += 1
+        up.wait_event(computed[s])
+        with torch.cuda.stream(up):
+            h_dev[r][s].copy_(h_host[r], non_blocking=True)
+        uploaded[s].record(up)
+        compute.wait_event(uploaded[s])
+        compute.wait_event(downloaded[s])
+        wl.call(r, hidden=h_dev[r][s], out=o_dev[r][s], stream=compute)
+        computed[s].record(compute)
+        down.wait_event(computed[s])
+        with torch.cuda.stream(down):
+            o_host[r].copy_(o_dev[r][s], non_blocking=True)
+        downloaded[s].record(down)
+
     steps = max(1, min(args.steps, 50))
     for _ in range(2):
         for r in rl:
-            h_dev[r].copy_(h_host[r], non_blocking=True)
-            wl.call(r, hidden=h_dev[r])
-            o_host[r].copy_(wl.outs[r], non_blocking=True)
+            one_call(r)
+    torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(compute)
+    up.wait_event(e0)
+    down.wait_event(e0)
     for _ in range(steps):
         for r in rl:
-            h_dev[r].copy_(h_host[r], non_blocking=True)
-            wl.call(r, hidden=h_dev[r])
-            o_host[r].copy_(wl.outs[r], non_blocking=True)
-    e1.record(stream)
+            one_call(r)
+    compute.wait_stream(up)
+    compute.wait_stream(down)
+    e1.record(compute)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = sum(h_host[r].numel() * h_host[r].element_size() for r in rl)
     d2h = sum(o_host[r].numel() * o_host[r].element_size() for r in rl)
     share = 1 if wl.vocab_parallel else world   # calls made together count once
     return {"value": round(ms * 1e3 / (steps * len(rl) * share), 3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelining": "copies on two streams, two buffer sets alternated"}
 
 
 # ---------------------------------------------------------------- CPU oracle (baseline arm)
