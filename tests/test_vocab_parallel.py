@@ -257,3 +257,24 @@ def test_vocab_parallel_logits_on_symmetric_memory_in_a_one_rank_group():
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("rows,H", [(64, 2048), (300, 4096)])
+def test_slice_logits_at_the_bench_shapes(rows, H):
+    """The decode shape (64 rows, H = 2048) and a CTA-pair shape (300 rows, H = 4096) at
+    V = 151936, split 8 ways into two buffers: every buffer is the whole head's logits bit for
+    bit, and sampled rows agree with the CPU oracle."""
+    from tolerance import assert_fp32_close
+    V, g = 151936, 8
+    (h, w, _, _), (hd, wd, _, _) = make(rows, H, V, 80 + rows, "bf16", False, std=0.02)
+    alpha = 0.125
+    bufs = [torch.empty((rows, V), dtype=torch.float32, device="cuda") for _ in range(2)]
+    for b0, n in slices(V, g):
+        lm.logits_vocab_slice_f32(hd, wd[b0:b0 + n], b0, bufs, alpha)
+    whole = lm.logits_f32(hd, wd, alpha)
+    check_status()
+    for buf in bufs:
+        assert torch.equal(buf.view(torch.int32), whole.view(torch.int32))
+    sample = np.array([0, rows // 2, rows - 1])
+    ref, absum = oracle.logits_bf16_f32(h[sample], w, alpha)
+    assert_fp32_close(bufs[1].cpu().numpy()[sample], ref, absum, "slice logits, bench shape")
