@@ -55,6 +55,8 @@ SHAPES = [
     (300, 200, 1000),    # V mod 256 = 232: odd CTA of the last pair partly filled
     (513, 72, 129),      # one pair v-tile, odd CTA holds one row; H not a multiple of 64
     (600, 320, 2048 + 128),  # V mod 256 = 128: the odd CTA of the last pair empty
+    (256, 64, 1),        # one vocab row: the only pair's odd CTA holds nothing
+    (241, 136, 128),     # the fewest rows that make a 256-row tile; V = 128: odd CTA empty
 ]
 
 
