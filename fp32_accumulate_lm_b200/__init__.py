@@ -109,6 +109,8 @@ def _bind(lib, test: bool):
         lib.lmhead_debug_set_nvfp4_conversion.restype = None
         lib.lmhead_debug_set_cta_pairs.argtypes = [i32]
         lib.lmhead_debug_set_cta_pairs.restype = None
+        lib.lmhead_debug_set_dynamic_tiles.argtypes = [i32]
+        lib.lmhead_debug_set_dynamic_tiles.restype = None
     return lib
 
 
@@ -316,6 +318,14 @@ def set_cta_pairs(enabled: bool) -> None:
     tiles on CTA pairs (the default) or keeps every tile on one CTA (the same bits either way)."""
     _require_test_build("set_cta_pairs")
     _active().lmhead_debug_set_cta_pairs(1 if enabled else 0)
+
+
+def set_dynamic_tiles(enabled: bool) -> None:
+    """Test build only (inside ``test_hooks()``): whether the fp32 head's units take their later
+    tiles by cluster launch control (the default) or follow the static schedule (the same bits
+    either way)."""
+    _require_test_build("set_dynamic_tiles")
+    _active().lmhead_debug_set_dynamic_tiles(1 if enabled else 0)
 
 
 def set_fault_injection(starve_loads: bool, wait_limit_ns: int = 0) -> None:

@@ -47,6 +47,11 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
 #ifndef LMHEAD_PAIR
 #define LMHEAD_PAIR 1
 #endif
+// Tiles after a unit's first taken by cluster launch control (one unit launched per tile, the
+// running units cancel the launches of the rest in order): 1 on, 0 static (build-time knob).
+#ifndef LMHEAD_CLC
+#define LMHEAD_CLC 1
+#endif
 // CTA pairs in the log-prob modes too: 1 on, 0 off (build-time knob).
 #ifndef LMHEAD_PAIR_LOGPROB
 #define LMHEAD_PAIR_LOGPROB 0
@@ -61,6 +66,7 @@ constexpr CUtensorMapL2promotion kWeightPromo =
 std::atomic<int> g_starve_loads{0};
 std::atomic<int> g_nvfp4_path{0};  // 0: automatic, 1: pair table, 2: spread (test hook)
 std::atomic<int> g_no_cta_pairs{0};  // 1: the bf16 head runs 256-row tiles on lone CTAs (test hook)
+std::atomic<int> g_static_tiles{0};  // 1: the bf16 head's static schedule only (test hook)
 std::atomic<uint64_t> g_wait_limit_ns{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -470,6 +476,8 @@ void lmhead_debug_set_nvfp4_conversion(int path) {
 }
 
 void lmhead_debug_set_cta_pairs(int enabled) { g_no_cta_pairs.store(enabled ? 0 : 1); }
+
+void lmhead_debug_set_dynamic_tiles(int enabled) { g_static_tiles.store(enabled ? 0 : 1); }
 #endif
 
 size_t lmhead_nvfp4_quantize_workspace_bytes(void) {
@@ -612,6 +620,8 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   st = make_sched(rows, V, H, p.bn, pair, pair ? dev.pair_clusters : dev.num_sms, &p.sched,
                   &grid);
   if (st != LMHEAD_OK) return st;
+  p.clc = LMHEAD_CLC && !g_static_tiles.load(std::memory_order_relaxed);
+  if (p.clc) grid = p.sched.num_tiles << pair;  // every tile a unit of its own at launch
   const int reserve = 1024 + 512;  // alignment slack + barriers
   // (pairs: one K sub-tile per stage, six stages; two sub-tiles and three stages measured ~1 %
   // slower at 2048 and 8192 rows)

@@ -51,6 +51,7 @@ struct Bf16HeadParams {
   int32_t bn;        // rows per tile: multiple of 16 in [16, 256]
   int32_t hid_rows;  // rows of hidden one TMA box brings (<= bn; MMA columns past it unused)
   TileSched sched;
+  int32_t clc;       // 1: units take their tiles after the first by cluster launch control
   int32_t num_ks;    // pipeline stages per tile: ceil(H / (64 * NSUB))
   int32_t stages;
   uint32_t tmem_cols;
@@ -153,6 +154,64 @@ __global__ void __launch_bounds__(kMergeThreads)
   logprobs[row] = __fsub_rn(zt, l);
 }
 
+// Tile streams. Every role walks the same tiles of its unit in the same order: under the static
+// schedule tile j is unit + j * units while j < the unit's count; under cluster launch control
+// (one unit launched per tile) tile 0 is the unit's own and tile j >= 1 comes from the j-th
+// answer, which the leader's producer asks for when it starts tile j - 1. The answers live in a
+// ring of kClcSlots 16-byte slots: full[k] counts the answer's 16 bytes, empty[k] the reads of
+// every role that takes tile ids (the leader's MMA warp, both CTAs' producers and epilogue
+// warps), so a slot is asked again only after all of them have read it.
+constexpr int kClcSlots = 4;
+
+struct ClcRing {
+  uint32_t resp0, full0, empty0;
+};
+
+// Tile j (j >= 1) of this unit from the cluster launch control answers, or -1 when none is left
+// (or the wait gave up; `ok` is then false). The whole warp reads the answer; lane 0 releases
+// the slot on the pair leader's empty barrier.
+template <bool kPair>
+__device__ __forceinline__ int clc_take(const ClcRing& r, int j, const WaitCfg& w,
+                                        volatile int* abort_flag, bool& ok) {
+  const int slot = (j - 1) % kClcSlots;
+  const uint32_t phase = (uint32_t)((j - 1) / kClcSlots) & 1u;
+  if (!wait_bounded(r.full0 + 8 * slot, phase, w, abort_flag)) {
+    ok = false;
+    return -1;
+  }
+  const int x = clc_first_ctaid_x(r.resp0 + 16 * slot);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    if constexpr (kPair) {
+      mbar_arrive_remote(r.empty0 + 8 * slot, 0);
+    } else {
+      mbar_arrive(r.empty0 + 8 * slot);
+    }
+  }
+  return x < 0 ? -1 : (x >> (kPair ? 1 : 0));
+}
+
+// The leader's producer asks for tile j (j >= 1) of its unit. Both CTAs' full barriers are
+// armed for the 16-byte answer before the request goes out.
+template <bool kPair>
+__device__ __forceinline__ bool clc_ask(const ClcRing& r, int j, const WaitCfg& w,
+                                        volatile int* abort_flag) {
+  const int slot = (j - 1) % kClcSlots;
+  const uint32_t phase = ((uint32_t)((j - 1) / kClcSlots) & 1u) ^ 1u;
+  if (!wait_bounded(r.empty0 + 8 * slot, phase, w, abort_flag)) return false;
+  if ((threadIdx.x & 31) == 0) {
+    mbar_arrive_expect_tx(r.full0 + 8 * slot, 16);
+    if constexpr (kPair) {
+      mbar_arrive_expect_tx_remote(r.full0 + 8 * slot, 1, 16);
+      clc_try_cancel_all(r.resp0 + 16 * slot, r.full0 + 8 * slot);
+    } else {
+      clc_try_cancel(r.resp0 + 16 * slot, r.full0 + 8 * slot);
+    }
+  }
+  __syncwarp();
+  return true;
+}
+
 template <int NSUB, bool kPair>
 __global__ void __launch_bounds__(kHeadThreads, 1)
     lmhead_bf16_f32_kernel(const __grid_constant__ CUtensorMap tmap_w,
@@ -184,11 +243,20 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   const uint32_t done_bar = smem_u32(bars + 2 * S + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // cluster launch control: 4 answer slots (16-byte aligned), then their full and empty barriers
+  const ClcRing clc{smem_u32(bars + 2 * S + 6), smem_u32(bars + 2 * S + 14),
+                    smem_u32(bars + 2 * S + 18)};
+  // readers of an answer: both CTAs' producers and epilogue warps, the leader's MMA warp
+  constexpr uint32_t kClcReaders = (kPair ? 2u : 1u) * (1u + kBf16EpiWarps) + 1u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int k = 0; k < kClcSlots; ++k) {
+      mbar_init(clc.full0 + 8 * k, 1);
+      mbar_init(clc.empty0 + 8 * k, kClcReaders);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
@@ -222,6 +290,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
   pdl_wait();  // from here on global memory: earlier kernels of the stream are done
   const uint32_t tmem_base = *tmem_slot;
   const int my_tiles = sched_count(p.sched);
+  const int unit = (int)blockIdx.x >> (kPair ? 1 : 0);
+  const int units = (int)gridDim.x >> (kPair ? 1 : 0);
+  // this unit's first tile; -1 when the static schedule gives it none
+  const int first_tile = my_tiles > 0 ? unit : -1;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -231,8 +303,18 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    for (int t = 0; ok && t < my_tiles; ++t) {
-      const TileCoord tc = sched_tile(p.sched, p.V, t);
+    int asked = 0;  // cluster launch control requests issued (answers read: j below)
+    int tile = first_tile;
+    for (int j = 0; ok && tile >= 0; ++j) {
+      // ask for the next tile as this one starts, so the answer is in before it is needed
+      if (p.clc && leader) {
+        if (!clc_ask<kPair>(clc, j + 1, p.wait, abort_flag)) {
+          fail(kRoleProducer, abort_flag);
+          break;
+        }
+        asked = j + 1;
+      }
+      const TileCoord tc = sched_tile_at(p.sched, p.V, tile);
       // a pair's full barrier (the leader's) counts both CTAs' bytes
       const uint32_t tx = (uint32_t)NSUB * (a_sub + b_tx) * (kPair ? 2u : 1u);
       const int32_t hid_y = (int32_t)(tc.r0 + (kPair ? (int64_t)rank * (p.bn / 2) : 0));
@@ -266,6 +348,19 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
           phase ^= 1u;
         }
       }
+      if (!ok) break;
+      if (p.clc) {
+        tile = clc_take<kPair>(clc, j + 1, p.wait, abort_flag, ok);
+        if (!ok) fail(kRoleProducer, abort_flag);
+      } else {
+        tile = j + 1 < my_tiles ? unit + (j + 1) * units : -1;
+      }
+    }
+    // An answer asked for but not read (an error path) must still land before the CTA exits.
+    if (p.clc && leader && asked > 0) {
+      const int slot = (asked - 1) % kClcSlots;
+      const uint32_t ph = (uint32_t)((asked - 1) / kClcSlots) & 1u;
+      if (!wait_bounded(clc.full0 + 8 * slot, ph, p.wait, nullptr)) fail(kRoleDrain, abort_flag);
     }
     // Drain: every load this CTA issued must land before the CTA may exit. A lone CTA sees that
     // on its full barriers. A pair's loads are counted on the leader's full barriers, so both
@@ -295,7 +390,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = 0; ok && leader && t < my_tiles; ++t) {
+    int tile = leader ? first_tile : -1;
+    for (int tj = 0; ok && tile >= 0; ++tj) {
       if (!wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, p.wait, abort_flag)) {
         fail(kRoleMma, abort_flag);
         break;
@@ -346,6 +442,12 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
       __syncwarp();
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+      if (p.clc) {
+        tile = clc_take<kPair>(clc, tj + 1, p.wait, abort_flag, ok);
+        if (!ok) fail(kRoleMma, abort_flag);
+      } else {
+        tile = tj + 1 < my_tiles ? unit + (tj + 1) * units : -1;
+      }
     }
     // Every MMA this warp issued must finish before TMEM is released (a pair's other CTA
     // learns it at the closing cluster barrier).
@@ -367,8 +469,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
     const int v_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = 0; t < my_tiles; ++t) {
-      const TileCoord tc = sched_tile(p.sched, p.V, t);
+    bool ok = true;
+    int tile = first_tile;
+    for (int tj = 0; ok && tile >= 0; ++tj) {
+      const TileCoord tc = sched_tile_at(p.sched, p.V, tile);
       if (!wait_bounded(tfull0 + 8 * acc, acc_phase, p.wait, abort_flag, kSleepHintNs)) {
         fail(kRoleEpilogue, abort_flag);
         break;
@@ -497,6 +601,12 @@ __global__ void __launch_bounds__(kHeadThreads, 1)
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+      if (p.clc) {
+        tile = clc_take<kPair>(clc, tj + 1, p.wait, abort_flag, ok);
+        if (!ok) fail(kRoleEpilogue, abort_flag);
+      } else {
+        tile = tj + 1 < my_tiles ? unit + (tj + 1) * units : -1;
+      }
     }
   }
 

@@ -131,11 +131,9 @@ __device__ __forceinline__ int sched_count(const TileSched& s) {
   return unit < s.num_tiles ? (s.num_tiles - 1 - unit) / units + 1 : 0;
 }
 
-__device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, int i) {
+// The coordinates of tile t (this CTA's part of it, for a pair).
+__device__ __forceinline__ TileCoord sched_tile_at(const TileSched& s, int64_t V, int t) {
   TileCoord c;
-  const int unit = (int)blockIdx.x >> s.pair;
-  const int units = (int)gridDim.x >> s.pair;
-  const int t = unit + i * units;
   const int per_group = s.n_vtiles * s.rgroup;
   const int g = t / per_group;
   const int local = t - g * per_group;
@@ -148,6 +146,11 @@ __device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, i
   c.vrows = (int32_t)(left < 0 ? 0 : left < kBM ? left : kBM);
   c.r0 = (int64_t)rt * s.bn;
   return c;
+}
+
+// The coordinates of this unit's i-th tile under the static schedule.
+__device__ __forceinline__ TileCoord sched_tile(const TileSched& s, int64_t V, int i) {
+  return sched_tile_at(s, V, ((int)blockIdx.x >> s.pair) + i * ((int)gridDim.x >> s.pair));
 }
 
 __device__ __forceinline__ uint64_t l2_policy_weights() {

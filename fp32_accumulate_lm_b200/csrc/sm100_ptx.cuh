@@ -228,6 +228,62 @@ __device__ __forceinline__ void mma_commit_pair_elect(uint32_t bar, uint16_t cta
       : "memory");
 }
 
+// ------------------------------------------------------------------ cluster launch control
+// A persistent CTA (or CTA pair) takes its next tile by cancelling the launch of a cluster of
+// the same grid that has not started yet: the hardware answers with that cluster's first CTA
+// id (16 bytes written to shared memory, counted on an mbarrier as 16 transaction bytes) or
+// with "nothing left". Clusters are handed out in launch order, so the tiles are taken in
+// order by whichever units are free first.
+
+// Ask for the next cluster; the answer lands in this CTA's `resp` (16-byte aligned).
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+
+// The same for a cluster of CTAs: the answer lands at the same offset in every CTA of the
+// cluster and is counted on each CTA's mbarrier at the same offset as `bar`.
+__device__ __forceinline__ void clc_try_cancel_all(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes"
+      ".multicast::cluster::all.b128 [%0], [%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+
+// The x of the cancelled cluster's first CTA, or -1 when there was nothing left to cancel.
+__device__ __forceinline__ int clc_first_ctaid_x(uint32_t resp) {
+  uint32_t valid, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "mov.u32 %1, 0;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, _, _, _}, r;\n\t}"
+      : "=r"(valid), "=r"(x)
+      : "r"(resp)
+      : "memory");
+  // the answer's buffer is rewritten by the asynchronous proxy: order this read before that
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  return valid ? (int)x : -1;
+}
+
+// Arm the mbarrier at local offset `bar` of cluster CTA `rank` for `bytes` more transaction
+// bytes, with one arrival (release, cluster scope).
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t rank,
+                                                             uint32_t bytes) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(bar), "r"(rank));
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   remote),
+               "r"(bytes)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05 / TMEM
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {

@@ -316,10 +316,15 @@ int lmhead_version(void);
  * lmhead_debug_set_cta_pairs: enabled != 0 (the default) lets the fp32 head run full 256-row
  * tiles on CTA pairs (cta_group::2 MMAs, 256 vocab rows per tile); 0 keeps every tile on one
  * CTA. Both give identical bits; the knob lets tests show that.
+ *
+ * lmhead_debug_set_dynamic_tiles: enabled != 0 (the default) lets the fp32 head's persistent
+ * units take their tiles after the first by cluster launch control, in launch order; 0 keeps
+ * the static round-robin schedule. Both give identical bits; the knob lets tests show that.
  */
 void lmhead_debug_set_fault_injection(int starve_loads, uint64_t wait_limit_ns);
 void lmhead_debug_set_nvfp4_conversion(int path);
 void lmhead_debug_set_cta_pairs(int enabled);
+void lmhead_debug_set_dynamic_tiles(int enabled);
 #endif
 
 #ifdef __cplusplus

@@ -67,7 +67,7 @@ def test_test_knobs_exist_only_in_the_test_build(lib):
     the release library does not export them, the test build exports them and everything else."""
     knobs = hook_functions()
     assert set(knobs) == {"lmhead_debug_set_fault_injection", "lmhead_debug_set_nvfp4_conversion",
-                          "lmhead_debug_set_cta_pairs"}
+                          "lmhead_debug_set_cta_pairs", "lmhead_debug_set_dynamic_tiles"}
     release, test = exported(lm.library_path()), exported(_build.TEST_LIB)
     assert not set(knobs) & release
     assert set(knobs) | set(declared_functions()) <= test
