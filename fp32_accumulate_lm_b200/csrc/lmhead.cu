@@ -620,8 +620,10 @@ int run_f32_head(const void* hidden, int dtype, int64_t rows, int64_t H, const v
   st = make_sched(rows, V, H, p.bn, pair, pair ? dev.pair_clusters : dev.num_sms, &p.sched,
                   &grid);
   if (st != LMHEAD_OK) return st;
-  p.clc = LMHEAD_CLC && !g_static_tiles.load(std::memory_order_relaxed);
-  if (p.clc) grid = p.sched.num_tiles << pair;  // every tile a unit of its own at launch
+  // every tile a unit of its own at launch (the static schedule when that grid would not fit)
+  p.clc = LMHEAD_CLC && !g_static_tiles.load(std::memory_order_relaxed) &&
+          ((int64_t)p.sched.num_tiles << pair) <= kInt32Max;
+  if (p.clc) grid = p.sched.num_tiles << pair;
   const int reserve = 1024 + 512;  // alignment slack + barriers
   // (pairs: one K sub-tile per stage, six stages; two sub-tiles and three stages measured ~1 %
   // slower at 2048 and 8192 rows)
