@@ -363,6 +363,8 @@ SECONDARY = ["spec_verify", "prefill", "nvfp4", "decode_f16_bias", "prefill_logp
 # A timed region at least this long is "a long step": the sustained bf16 peak applies.
 SUSTAINED_REGION_S = 1.0
 PER_ROW_IDLE_S = 1.0   # idle before each per-row-count loop (see measure)
+PER_ROW_WARMUP = 20    # untimed calls of the row count before its loop
+PER_ROW_MIN_CALLS = 100  # timed calls per row count at least
 
 
 def config_of(name: str, world: int) -> dict:
@@ -419,21 +421,26 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     elapsed_ms = e_start.elapsed_time(e_end)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
 
-    # Per row count (the detail below the headline): each row count alone, as many calls as the
-    # timed region made of it, between two events. Each loop starts after PER_ROW_IDLE_S of idle,
-    # so that every row count starts from the same clock state: the loops follow the timed
-    # region, and after tensor-heavy calls the power cap holds the SM clock down for a while.
+    # Per row count (the detail below the headline): each row count alone, between two events.
+    # Each loop starts after PER_ROW_IDLE_S of idle, so that every row count starts from the same
+    # power state (the loops follow the timed region, and after tensor-heavy calls the power cap
+    # holds the SM clock down for a while), then runs PER_ROW_WARMUP untimed calls of its row
+    # count so the clock is back up from idle, then times max(steps, PER_ROW_MIN_CALLS) calls.
     per_row_ms = {}
+    per_row_calls = max(args.steps, PER_ROW_MIN_CALLS)
     for r in rl:
         time.sleep(PER_ROW_IDLE_S)
+        for _ in range(max(args.warmup, PER_ROW_WARMUP)):
+            wl.call(r)
+        torch.cuda.synchronize()
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.steps):
+        for _ in range(per_row_calls):
             wl.call(r)
         b.record(stream)
         torch.cuda.synchronize()
-        per_row_ms[r] = a.elapsed_time(b) / args.steps
+        per_row_ms[r] = a.elapsed_time(b) / per_row_calls
     barrier(world)
 
     # per row count: mean launch duration, algorithmic bytes and flops
@@ -442,7 +449,7 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     for r in rl:
         mean_ms = per_row_ms[r]
         b, fl = wl.bytes_of(r), wl.flops_of(r)
-        detail[str(r)] = {"us": round(mean_ms * 1e3, 2),
+        detail[str(r)] = {"us": round(mean_ms * 1e3, 2), "calls": per_row_calls,
                           "GBps": round(b / (mean_ms * 1e-3) / 1e9, 1),
                           "TFLOPs": round(fl / (mean_ms * 1e-3) / 1e12, 1)}
         tot_bytes += b
