@@ -15,9 +15,17 @@ from oracle_inputs import nvfp4_weights
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("entry", ["bf16", "nvfp4"])
-def test_starved_loads_time_out_cleanly(entry):
-    rows, H, V = 8, 128, 512
+@pytest.mark.parametrize("entry,rows,V", [
+    ("bf16", 8, 512),
+    # many more tiles than SMs: units that gave up leave launches pending, which then start,
+    # take no tile answers of their own and give up as well
+    ("bf16", 8, 151936),
+    # CTA pairs (256-row tiles) with their dynamic tiles: both CTAs of a pair give up
+    ("bf16", 300, 2048),
+    ("nvfp4", 8, 512),
+])
+def test_starved_loads_time_out_cleanly(entry, rows, V):
+    H = 128
     h = dev_bf16(synth.hidden(rows, H, 1))
     w = dev_bf16(synth.weight(V, H, 0.02, 1))
     packed, scales, g = nvfp4_weights(V, H, 0.02, 1)
