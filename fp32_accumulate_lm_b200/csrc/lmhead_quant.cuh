@@ -8,7 +8,10 @@
 //                          only on a non-zero magnitude
 // RN is round to nearest, ties to the even code (the conversions' .rn mode).
 //
-// Both passes stream W once (HBM-bound); the encode pass's divisions are IEEE (div.rn).
+// Both passes stream W once. The absmax pass is HBM-bound; the encode pass is held by its
+// instruction issue (about 8 instructions an element), so its per-block work is trimmed: the
+// block maximum on the bf16x2 max, the divisor and reciprocals of every scale code from a
+// per-CTA table, the codes packed by byte permutes. Its divisions are IEEE (div.rn).
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -23,6 +26,21 @@ constexpr int kQuantMaxPartials = 1024;  // absmax partials: one 32-bit word per
 __device__ __forceinline__ uint32_t chunk_absmax_bits(const uint4& c) {
   const uint32_t m = __vmaxu2(__vmaxu2(c.x & 0x7FFF7FFFu, c.y & 0x7FFF7FFFu),
                               __vmaxu2(c.z & 0x7FFF7FFFu, c.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Largest |bf16| of a 32-byte block of finite values as magnitude bits, on the bf16x2 max
+// (each lane's result has magnitude max(|a|, |b|); the sign bits are cleared at the end).
+__device__ __forceinline__ uint32_t block_absmax_bits(const uint4& c0, const uint4& c1) {
+  uint32_t a, b, c, d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(c0.x), "r"(c0.y));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(c0.z), "r"(c0.w));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(c1.x), "r"(c1.y));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(c1.z), "r"(c1.w));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(b));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(c), "r"(d));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(c));
+  const uint32_t m = a & 0x7FFF7FFFu;
   return max(m & 0xFFFFu, m >> 16);
 }
 
@@ -89,6 +107,20 @@ __device__ __forceinline__ uint32_t e2m1_pair_code(float lo, float hi) {
   return two & 0xFFu;
 }
 
+// The byte of e2m1_pair_code in the low byte of a word whose other bytes are not specified.
+__device__ __forceinline__ uint32_t e2m1_pair_byte(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The low bytes of a, b, c, d as one word, a in the low byte.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
 // Eight E2M1 codes in a word: clear the sign bit of every nibble whose magnitude is zero. Adding
 // 7 to a 3-bit magnitude carries into the nibble's bit 3 exactly when the magnitude is non-zero,
 // and never out of the nibble.
@@ -110,24 +142,47 @@ constexpr float kQuotientBand = 0x1p-16f;
 // magnitude, so when both products give the same code, x has that code as well. Only a pair with
 // a quotient within about 2^-16 of a boundary (0.25, 0.75, ..., 5) is divided exactly. d outside
 // [2^-120, 2^120], where r could leave the normal range, is always divided exactly.
-__device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, float g,
-                                             float six_g, uint2* packed, uint8_t* scale) {
-  const float bmax = __uint_as_float(max(chunk_absmax_bits(c0), chunk_absmax_bits(c1)) << 16);
+//
+// The divisor d = fl(e4m3(s) g) and the two bracketing reciprocals depend only on the scale
+// code s, so each CTA computes them once for all 128 codes (make_scale_entry) into a shared
+// table; the conversion saturates at 448 (code 0x7E), so code 0x7F (NaN) is never looked up.
+struct ScaleEntry {
+  float d, r_lo, r_hi;
+  uint32_t shortcut;  // 1 when d is in [2^-120, 2^120]
+};
+
+__device__ __forceinline__ ScaleEntry make_scale_entry(uint32_t s, float g) {
+  ScaleEntry e;
+  e.d = __fmul_rn(e4m3_value(s), g);
+  e.shortcut = (e.d >= 0x1p-120f && e.d <= 0x1p120f) ? 1u : 0u;
+  const float r = __frcp_rn(e.d);
+  e.r_lo = __fmul_rn(r, 1.0f - kQuotientBand);
+  e.r_hi = __fmul_rn(r, 1.0f + kQuotientBand);
+  return e;
+}
+
+__device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, float six_g,
+                                             const float4* scale_table, uint2* packed,
+                                             uint8_t* scale) {
+  const float bmax = __uint_as_float(block_absmax_bits(c0, c1) << 16);
   const uint32_t s = rn_e4m3_code(__fdiv_rn(bmax, six_g));
-  const float d = __fmul_rn(e4m3_value(s), g);
-  const bool shortcut = d >= 0x1p-120f && d <= 0x1p120f;
-  const float r = __frcp_rn(d);
-  const float r_lo = __fmul_rn(r, 1.0f - kQuotientBand);
-  const float r_hi = __fmul_rn(r, 1.0f + kQuotientBand);
+  const float4 te = scale_table[s & 0x7Fu];  // s <= 0x7E: the conversion saturates at 448
+  const float d = te.x, r_lo = te.y, r_hi = te.z;
+  const bool shortcut = __float_as_uint(te.w) != 0u;
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
+  uint32_t bl[8], bh[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
     const float w0 = __uint_as_float(words[i] << 16);
     const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
-    lo[i >> 2] |= e2m1_pair_code(__fmul_rn(w0, r_lo), __fmul_rn(w1, r_lo)) << (8 * (i & 3));
-    hi[i >> 2] |= e2m1_pair_code(__fmul_rn(w0, r_hi), __fmul_rn(w1, r_hi)) << (8 * (i & 3));
+    bl[i] = e2m1_pair_byte(__fmul_rn(w0, r_lo), __fmul_rn(w1, r_lo));
+    bh[i] = e2m1_pair_byte(__fmul_rn(w0, r_hi), __fmul_rn(w1, r_hi));
   }
+  lo[0] = pack_low_bytes(bl[0], bl[1], bl[2], bl[3]);
+  lo[1] = pack_low_bytes(bl[4], bl[5], bl[6], bl[7]);
+  hi[0] = pack_low_bytes(bh[0], bh[1], bh[2], bh[3]);
+  hi[1] = pack_low_bytes(bh[4], bh[5], bh[6], bh[7]);
   if (!shortcut || lo[0] != hi[0] || lo[1] != hi[1]) {
     // Some quotient of the block sits near a code boundary (or r is unusable): divide those
     // pairs exactly.
@@ -151,11 +206,13 @@ __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, f
 
 // Pass 2: every CTA reduces the partials to amax (the same value everywhere), then each thread
 // encodes 16-element blocks: 32 bytes of W in, 8 bytes of codes and one scale byte out.
-__global__ void __launch_bounds__(kQuantThreads)
+// Four CTAs per SM (64 registers a thread): two full waves of the 8-per-SM grid.
+__global__ void __launch_bounds__(kQuantThreads, 4)
     nvfp4_encode_kernel(const uint4* __restrict__ w, int64_t n_blocks,
                         const uint32_t* __restrict__ partial, int n_partial, uint2* packed,
                         uint8_t* scales, float* g_out) {
   __shared__ uint32_t red[32];
+  __shared__ float4 scale_table[128];
   uint32_t m = 0;
   for (int i = threadIdx.x; i < n_partial; i += blockDim.x) m = max(m, partial[i]);
   m = block_max_u32(m, red);
@@ -163,19 +220,25 @@ __global__ void __launch_bounds__(kQuantThreads)
   const float g = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
   const float six_g = __fmul_rn(6.0f, g);
   if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  static_assert(kQuantThreads >= 128, "one thread per scale code");
+  if (threadIdx.x < 128) {
+    const ScaleEntry e = make_scale_entry(threadIdx.x, g);
+    scale_table[threadIdx.x] = make_float4(e.d, e.r_lo, e.r_hi, __uint_as_float(e.shortcut));
+  }
+  __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   // Two blocks per iteration, their four loads issued together.
   for (; b + stride < n_blocks; b += 2 * stride) {
     const uint4 a0 = __ldcs(w + 2 * b), a1 = __ldcs(w + 2 * b + 1);
     const uint4 b0 = __ldcs(w + 2 * (b + stride)), b1 = __ldcs(w + 2 * (b + stride) + 1);
-    encode_block(a0, a1, g, six_g, packed + b, scales + b);
-    encode_block(b0, b1, g, six_g, packed + b + stride, scales + b + stride);
+    encode_block(a0, a1, six_g, scale_table, packed + b, scales + b);
+    encode_block(b0, b1, six_g, scale_table, packed + b + stride, scales + b + stride);
   }
   for (; b < n_blocks; b += stride) {
     const uint4 c0 = __ldcs(w + 2 * b);
     const uint4 c1 = __ldcs(w + 2 * b + 1);
-    encode_block(c0, c1, g, six_g, packed + b, scales + b);
+    encode_block(c0, c1, six_g, scale_table, packed + b, scales + b);
   }
 }
 
