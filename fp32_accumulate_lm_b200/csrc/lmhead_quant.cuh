@@ -11,7 +11,7 @@
 // Both passes stream W once. The absmax pass is HBM-bound; the encode pass is held by its
 // instruction issue (about 8 instructions an element), so its per-block work is trimmed: the
 // block maximum on the bf16x2 max, the divisor and reciprocals of every scale code from a
-// per-CTA table, the codes packed by byte permutes. Its divisions are IEEE (div.rn).
+// per-CTA table, four codes bytes packed by one vector move. Its divisions are IEEE (div.rn).
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -67,13 +67,14 @@ __global__ void __launch_bounds__(kQuantThreads)
   uint32_t m = 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  // Four independent 16-byte loads in flight per thread: enough bytes in flight per SM to cover
-  // the DRAM latency at the HBM rate.
-  for (; i + 3 * stride < n_chunks; i += 4 * stride) {
-    const uint4 a = __ldcs(w + i), b = __ldcs(w + i + stride), c = __ldcs(w + i + 2 * stride),
-                d = __ldcs(w + i + 3 * stride);
-    m = max(max(m, chunk_absmax_bits(a)), max(chunk_absmax_bits(b),
-                                              max(chunk_absmax_bits(c), chunk_absmax_bits(d))));
+  // Eight independent 16-byte loads in flight per thread (128 B; the grid's 6 CTAs per SM are
+  // all resident at 32 registers a thread), to cover the DRAM latency at the HBM rate.
+  for (; i + 7 * stride < n_chunks; i += 8 * stride) {
+    uint4 c[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) c[k] = __ldcs(w + i + k * stride);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = max(m, chunk_absmax_bits(c[k]));
   }
   for (; i < n_chunks; i += stride) m = max(m, chunk_absmax_bits(__ldcs(w + i)));
   m = block_max_u32(m, red);
@@ -107,18 +108,20 @@ __device__ __forceinline__ uint32_t e2m1_pair_code(float lo, float hi) {
   return two & 0xFFu;
 }
 
-// The byte of e2m1_pair_code in the low byte of a word whose other bytes are not specified.
-__device__ __forceinline__ uint32_t e2m1_pair_byte(float lo, float hi) {
+// E2M1 codes of four pairs (x0, x1) .. (x6, x7) as one word: pair j in byte j, its first value in
+// the low nibble (the codes of e2m1_pair_code, packed by one vector move).
+__device__ __forceinline__ uint32_t e2m1_quad(float x0, float x1, float x2, float x3, float x4,
+                                              float x5, float x6, float x7) {
   uint32_t r;
-  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
       : "=r"(r)
-      : "f"(hi), "f"(lo));
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
   return r;
-}
-
-// The low bytes of a, b, c, d as one word, a in the low byte.
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
 
 // Eight E2M1 codes in a word: clear the sign bit of every nibble whose magnitude is zero. Adding
@@ -171,18 +174,20 @@ __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, f
   const bool shortcut = __float_as_uint(te.w) != 0u;
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
-  uint32_t bl[8], bh[8];
+  float pl[16], ph[16];  // the products by r_lo and by r_hi, in element order
 #pragma unroll
   for (int i = 0; i < 8; ++i) {  // word i holds elements 2i (low half) and 2i + 1
     const float w0 = __uint_as_float(words[i] << 16);
     const float w1 = __uint_as_float(words[i] & 0xFFFF0000u);
-    bl[i] = e2m1_pair_byte(__fmul_rn(w0, r_lo), __fmul_rn(w1, r_lo));
-    bh[i] = e2m1_pair_byte(__fmul_rn(w0, r_hi), __fmul_rn(w1, r_hi));
+    pl[2 * i] = __fmul_rn(w0, r_lo);
+    pl[2 * i + 1] = __fmul_rn(w1, r_lo);
+    ph[2 * i] = __fmul_rn(w0, r_hi);
+    ph[2 * i + 1] = __fmul_rn(w1, r_hi);
   }
-  lo[0] = pack_low_bytes(bl[0], bl[1], bl[2], bl[3]);
-  lo[1] = pack_low_bytes(bl[4], bl[5], bl[6], bl[7]);
-  hi[0] = pack_low_bytes(bh[0], bh[1], bh[2], bh[3]);
-  hi[1] = pack_low_bytes(bh[4], bh[5], bh[6], bh[7]);
+  lo[0] = e2m1_quad(pl[0], pl[1], pl[2], pl[3], pl[4], pl[5], pl[6], pl[7]);
+  lo[1] = e2m1_quad(pl[8], pl[9], pl[10], pl[11], pl[12], pl[13], pl[14], pl[15]);
+  hi[0] = e2m1_quad(ph[0], ph[1], ph[2], ph[3], ph[4], ph[5], ph[6], ph[7]);
+  hi[1] = e2m1_quad(ph[8], ph[9], ph[10], ph[11], ph[12], ph[13], ph[14], ph[15]);
   if (!shortcut || lo[0] != hi[0] || lo[1] != hi[1]) {
     // Some quotient of the block sits near a code boundary (or r is unusable): divide those
     // pairs exactly.
@@ -206,7 +211,7 @@ __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, f
 
 // Pass 2: every CTA reduces the partials to amax (the same value everywhere), then each thread
 // encodes 16-element blocks: 32 bytes of W in, 8 bytes of codes and one scale byte out.
-// Four CTAs per SM (64 registers a thread): two full waves of the 8-per-SM grid.
+// Four CTAs per SM (at most 64 registers a thread): two full waves of the 8-per-SM grid.
 __global__ void __launch_bounds__(kQuantThreads, 4)
     nvfp4_encode_kernel(const uint4* __restrict__ w, int64_t n_blocks,
                         const uint32_t* __restrict__ partial, int n_partial, uint2* packed,
