@@ -77,6 +77,26 @@ def test_all_zero_and_single_spike():
     assert_same_as_oracle(bf16_bits(w), "spike")
 
 
+def test_subnormal_weights_divide_every_block():
+    """W wholly in bf16's subnormal range: amax < 2^-126 makes g, and every divisor e4m3(s)·g, an
+    fp32 subnormal, outside the reciprocal shortcut's range, so every block's codes come from the
+    exact quotients, and the block scale's quotient has a subnormal divisor."""
+    rng = np.random.default_rng(83)
+    w = rng.normal(0, 1, (32, 256)) * 2.0 ** -130
+    p, s, g = assert_same_as_oracle(bf16_bits(w), "subnormal")
+    assert 0 < g < np.float32(2.0 ** -126)
+    assert s.any() and p.any()
+
+
+def test_rows_scaled_over_120_binades():
+    """Rows scaled by 2^-60 .. 2^60: g near 2^50, the small rows' blocks round to scale code 0
+    (every code 0), the large rows' span the E4M3 range."""
+    rng = np.random.default_rng(84)
+    w = rng.normal(0, 1, (96, 256)) * 2.0 ** rng.integers(-60, 61, (96, 1))
+    p, s, g = assert_same_as_oracle(bf16_bits(w), "scaled")
+    assert (s == 0).any() and (s > 0).any()
+
+
 def test_quantised_head_runs_through_the_nvfp4_entry():
     """quantise on the GPU, then the W4A16 head on the GPU against the oracle head on the same
     codes."""
