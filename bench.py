@@ -365,6 +365,7 @@ SUSTAINED_REGION_S = 1.0
 PER_ROW_IDLE_S = 1.0   # idle before each per-row-count loop (see measure)
 PER_ROW_WARMUP = 20    # untimed calls of the row count before its loop
 PER_ROW_MIN_CALLS = 100  # timed calls per row count at least
+PER_ROW_BLOCKS = 5     # blocks of each per-row-count loop (median and minimum of their means)
 
 
 def config_of(name: str, world: int) -> dict:
@@ -426,21 +427,28 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     # power state (the loops follow the timed region, and after tensor-heavy calls the power cap
     # holds the SM clock down for a while), then runs PER_ROW_WARMUP untimed calls of its row
     # count so the clock is back up from idle, then times max(steps, PER_ROW_MIN_CALLS) calls.
-    per_row_ms = {}
+    # The loop is cut into PER_ROW_BLOCKS blocks with an event at each boundary, so the median and
+    # the minimum of the block means come with the mean.
+    per_row_ms, per_row_blocks = {}, {}
     per_row_calls = max(args.steps, PER_ROW_MIN_CALLS)
+    per_block = -(-per_row_calls // PER_ROW_BLOCKS)
+    per_row_calls = per_block * PER_ROW_BLOCKS
     for r in rl:
         time.sleep(PER_ROW_IDLE_S)
         for _ in range(max(args.warmup, PER_ROW_WARMUP)):
             wl.call(r)
         torch.cuda.synchronize()
         barrier(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(per_row_calls):
-            wl.call(r)
-        b.record(stream)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(PER_ROW_BLOCKS + 1)]
+        evs[0].record(stream)
+        for blk in range(PER_ROW_BLOCKS):
+            for _ in range(per_block):
+                wl.call(r)
+            evs[blk + 1].record(stream)
         torch.cuda.synchronize()
-        per_row_ms[r] = a.elapsed_time(b) / per_row_calls
+        per_row_ms[r] = evs[0].elapsed_time(evs[-1]) / per_row_calls
+        per_row_blocks[r] = [evs[i].elapsed_time(evs[i + 1]) / per_block
+                             for i in range(PER_ROW_BLOCKS)]
     barrier(world)
 
     # per row count: mean launch duration, algorithmic bytes and flops
@@ -449,7 +457,10 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     for r in rl:
         mean_ms = per_row_ms[r]
         b, fl = wl.bytes_of(r), wl.flops_of(r)
+        blocks = per_row_blocks[r]
         detail[str(r)] = {"us": round(mean_ms * 1e3, 2), "calls": per_row_calls,
+                          "us_median_block": round(statistics.median(blocks) * 1e3, 2),
+                          "us_min_block": round(min(blocks) * 1e3, 2),
                           "GBps": round(b / (mean_ms * 1e-3) / 1e9, 1),
                           "TFLOPs": round(fl / (mean_ms * 1e-3) / 1e12, 1)}
         tot_bytes += b
@@ -477,6 +488,10 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
     roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
     roof["source_hash"] = kernel_source_hash()
 
+    # the same step replayed from a CUDA graph, and the pages' PyTorch call for context
+    graph = run_graph(args, wl, world)
+    torch_mm = run_torch_mm(args, wl, tot_ms / calls_per_step)
+
     # end to end through the C ABI: pinned host hidden -> device, call, outputs -> pinned host
     e2e = run_e2e(args, wl, world)
 
@@ -492,6 +507,8 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
         "per_rows": detail,
         "roofline": roof,
         "e2e": e2e,
+        "graph": graph,
+        "torch_mm": torch_mm,
         "gpu_launches": n_ev * (3 if wl.vocab_parallel else
                                 2 if (wl.quantize or wl.logprobs) else 1),
         "clocks": clocks,
@@ -519,6 +536,8 @@ def run_ours(args) -> dict | None:
         "per_rows": main["per_rows"],
         "roofline": main["roofline"],
         "e2e": main["e2e"],
+        "graph": main["graph"],
+        "torch_mm": main["torch_mm"],
         "gpu_launches": main["gpu_launches"],
         "clocks": main["clocks"],
     }
@@ -533,6 +552,90 @@ def run_ours(args) -> dict | None:
         dist.barrier()
         dist.destroy_process_group()
     return line if rank == 0 else None
+
+
+def run_graph(args, wl, world: int) -> dict:
+    """The timed region's calls replayed from a CUDA graph: two steps (an even number of calls,
+    so the two weight copies keep alternating across replays) captured once through the same
+    Python calls, then max(1, steps // 2) replays between two events on the launching stream.
+    This leaves out the host's launch work that the main figure includes. The vocab-parallel
+    workload is left out: its step holds a collective."""
+    import torch
+    if wl.vocab_parallel:
+        return {"skipped": "the step holds an all-gather across the ranks"}
+    stream = torch.cuda.current_stream()
+    steps_per_graph = 2
+    calls = steps_per_graph * len(wl.rows_list)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps_per_graph):
+            for r in wl.rows_list:
+                wl.call(r)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // steps_per_graph)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(a.elapsed_time(b), world)
+    del g
+    import fp32_accumulate_lm_b200 as lm
+    if lm.device_status(clear=True) != 0:
+        raise RuntimeError(f"{wl.name}: device status word set during the graph replays")
+    return {"value": round(job_us_per_call(elapsed_ms, reps, calls, world), 3), "unit": UNIT,
+            "replays": reps, "calls_per_replay": calls}
+
+
+def run_torch_mm(args, wl, ours_ms_per_call: float) -> dict:
+    """Context only: the pages' own call, torch.mm(hidden, W.T, out_dtype=float32) (cuBLAS
+    through PyTorch), then the multiply by alpha (after adding the bias, where the workload has
+    one), on the same inputs, the same weight alternation and the same timed-region shape.
+    Only the workloads whose product is the fp32 logits have it."""
+    import torch
+    if wl.quantize or wl.nvfp4 or wl.logprobs or wl.vocab_parallel:
+        return {"skipped": "no fp32-logits call to compare with"}
+    stream = torch.cuda.current_stream()
+    k = [0]
+    into = [True]  # the out= form, unless this torch refuses it with out_dtype
+
+    def one(r):
+        w = wl.weights[k[0] & 1]
+        k[0] += 1
+        if into[0]:
+            try:
+                o = torch.mm(wl.hid[r], w.t(), out_dtype=torch.float32, out=wl.outs[r])
+            except (RuntimeError, TypeError):
+                into[0] = False
+        if not into[0]:
+            o = torch.mm(wl.hid[r], w.t(), out_dtype=torch.float32)
+        if wl.bias is not None:
+            o.add_(wl.bias)
+        o.mul_(wl.alpha)
+
+    for _ in range(args.warmup):
+        for r in wl.rows_list:
+            one(r)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        for r in wl.rows_list:
+            one(r)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_per_call = a.elapsed_time(b) / (args.steps * len(wl.rows_list))
+    return {"value": round(ms_per_call * 1e3, 3), "unit": UNIT,
+            "ours_speedup": round(ms_per_call / ours_ms_per_call, 3),
+            "how": ("torch.mm(hidden, W.T, out_dtype=float32, out=logits)" if into[0] else
+                    "logits = torch.mm(hidden, W.T, out_dtype=float32)") +
+                   (", logits.add_(bias)" if wl.bias is not None else "") +
+                   ", logits.mul_(alpha); per rank, context only"}
 
 
 def run_e2e(args, wl, world: int) -> dict:
