@@ -801,6 +801,20 @@ def _oracle_sample_text(name: str, n_rows: int, vslice: int, secs: float) -> str
             "sample), scaled by V and by rows, per call")
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count, for the CPU-baseline records."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 def cpu_baseline(name: str, wl, budget_s: float = 10.0) -> dict:
     """The oracle as it stands, on the host cores, on the bench's own inputs (rank 0, N = 1)."""
     import oracle
@@ -809,7 +823,7 @@ def cpu_baseline(name: str, wl, budget_s: float = 10.0) -> dict:
     secs = _oracle_run(d)
     cores = 1 if name == "nvfp4_quantize" else oracle.default_threads()
     return {"value": round(1e6 * secs * scale, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": _oracle_sample_text(name, n_rows, vslice, secs)}
+            "sample": _oracle_sample_text(name, n_rows, vslice, secs), **host_cpu()}
 
 
 def run_reference(args) -> dict | None:
@@ -840,7 +854,7 @@ def run_reference(args) -> dict | None:
         "config": config_of(name, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(us_per_call, 1), "unit": UNIT, "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, **host_cpu()},
         "e2e": {"value": round(us_per_call, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
