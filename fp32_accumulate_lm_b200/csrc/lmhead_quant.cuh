@@ -4,14 +4,14 @@
 // operation, so a CPU re-implementation can match it bit for bit:
 //   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
 //   per 16-element block:  s = RN_e4m3(bmax / (6 * g)), saturating at 448
-//   per element:           q = RN_e2m1(w / (e4m3(s) * g)), saturating at 6; the sign is kept
-//                          only on a non-zero magnitude
+//   per element:           q = RN_e2m1(w / d), d = e4m3(s) * g, saturating at 6, and 0 where
+//                          d is 0; the sign is kept only on a non-zero magnitude
 // RN is round to nearest, ties to the even code (the conversions' .rn mode).
 //
 // Both passes stream W once. The absmax pass is HBM-bound; the encode pass is held by its
 // instruction issue (about 8 instructions an element), so its per-block work is trimmed: the
 // block maximum on the bf16x2 max, the divisor and reciprocals of every scale code from a
-// per-CTA table, four codes bytes packed by one vector move. Its divisions are IEEE (div.rn).
+// per-CTA table, four code bytes packed by one vector move. Its divisions are IEEE (div.rn).
 #pragma once
 
 #include "lmhead_common.cuh"
@@ -202,7 +202,8 @@ __device__ __forceinline__ void encode_block(const uint4& c0, const uint4& c1, f
       lo[i >> 2] = (lo[i >> 2] & ~(0xFFu << sh)) | (q << sh);
     }
   }
-  // d = 0 only when the block's scale code is 0 (a block far below amax): every code is 0.
+  // d = 0 when the block's scale code is 0 (a block far below amax), or when e4m3(s) * g
+  // underflows (g subnormal): every code is 0.
   const bool zero = !(d > 0.0f);
   *packed = make_uint2(zero ? 0u : drop_negative_zeros(lo[0]),
                        zero ? 0u : drop_negative_zeros(lo[1]));

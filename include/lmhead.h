@@ -231,8 +231,9 @@ int lmhead_logits_w4a16_nvfp4(const void* hidden, int64_t rows, int64_t H, const
  * two kernels and a stream), but print no rules. This library's rules take every decision as one IEEE binary32 operation:
  *   amax = max |w|;  g = amax / 2688 (= 6 * 448), or 1 when amax = 0
  *   w_scales[v, j]  = RN_e4m3(max_{k in block j} |w[v, k]| / (6 * g)), saturating at 448
- *   code[v, k]      = RN_e2m1(w[v, k] / (e4m3(w_scales[v, k/16]) * g)), saturating at +-6,
- *                     with no negative zero; RN = nearest, ties to the even code
+ *   code[v, k]      = RN_e2m1(w[v, k] / d), d = e4m3(w_scales[v, k/16]) * g, saturating at
+ *                     +-6, with no negative zero; 0 where d is 0 (a block whose scale code is
+ *                     0, or a product that underflows); RN = nearest, ties to the even code
  * Packing as lmhead_logits_w4a16_nvfp4 reads it (element 2j in the low nibble of byte j).
  *
  *   w               bf16 [V, H], 16-byte aligned, finite    H > 0, H % 16 == 0, V > 0
