@@ -544,6 +544,21 @@ def test_quantiser_closed_forms():
     assert codes[0, 0] == 7 and not codes[0, 1:].any()
 
 
+def test_quantiser_block_below_the_smallest_scale_gets_zero_codes():
+    """A block whose maximum is far below amax rounds to scale code 0, so its divisor e4m3(0)·g
+    is 0; the reading makes every code of that block 0 (not the +-6 that w / 0 would saturate
+    to), signs included."""
+    H = 32
+    w = np.zeros((1, H))
+    w[0, 0] = 2688.0                       # g = 1
+    w[0, 16:32] = [1e-4, -1e-4, 3e-5, -2e-5] * 4   # t = bmax / 6 < 2^-10: scale code 0
+    p, s, g = oracle.nvfp4_quantize(bf16_bits_of_f32(w))
+    assert g == np.float32(1.0)
+    assert s[0, 1] == 0
+    codes = np.stack([p & 0x0F, p >> 4], axis=2).reshape(1, H)
+    assert not codes[0, 16:].any()
+
+
 def test_quantiser_all_zero_weights():
     p, s, g = oracle.nvfp4_quantize(np.zeros((3, 48), np.uint16))
     assert g == np.float32(1.0) and not p.any() and not s.any()
