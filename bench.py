@@ -567,7 +567,9 @@ def run_graph(args, wl, world: int) -> dict:
     steps_per_graph = 2
     calls = steps_per_graph * len(wl.rows_list)
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    # thread_local: other threads' CUDA calls (the NCCL watchdog's under torchrun) may go on
+    # during the capture; only this thread's calls are checked
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
         for _ in range(steps_per_graph):
             for r in wl.rows_list:
                 wl.call(r)
