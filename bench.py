@@ -103,6 +103,92 @@ def recorded_traffic(kernel: str, workload: str):
     return ent.get("bytes_per_launch")
 
 
+def roofline_kernel(name: str) -> str:
+    """The kernel (or kernel pair) a workload's roofline and traffic figures belong to."""
+    return ("nvfp4_encode_kernel + nvfp4_absmax_kernel" if name == "nvfp4_quantize" else
+            "lmhead_w4a16_nvfp4_kernel" if name == "nvfp4" else "lmhead_bf16_f32_kernel")
+
+
+def kernels_per_call(name: str) -> int:
+    """Launches of this library's kernels per call of a workload."""
+    if name == "vocab_parallel_logprobs":
+        return 3            # slice stats, combine, merge
+    if name in ("nvfp4_quantize", "prefill_logprobs", "prefill_logprobs_2048"):
+        return 2            # absmax + encode; log-prob epilogue + combine
+    return 1
+
+
+TRAFFIC_ABOUT = (
+    "DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum, summed over the call's "
+    "kernels), mean over the calls of one timed bench step, from one ncu capture per workload "
+    "(1 pass, --clock-control none): python bench.py --workload W --only --steps 1 --warmup 3 "
+    "--no-cpu-baseline under ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,"
+    "dram__bytes_write.sum -k 'regex:(lmhead|nvfp4)' -s <warm-up launches> -c <one step's "
+    "launches> --csv --log-file DIR/W.csv; written by python bench.py --traffic-from DIR; valid "
+    "only while source_hash matches bench.kernel_source_hash().")
+
+_NCU_UNITS = {"byte": 1, "B": 1, "Kbyte": 1e3, "KB": 1e3, "Mbyte": 1e6, "MB": 1e6, "Gbyte": 1e9,
+              "GB": 1e9, "nsecond": 1, "ns": 1, "usecond": 1e3, "us": 1e3, "msecond": 1e6,
+              "ms": 1e6}
+
+
+def read_ncu_launches(path: str) -> list:
+    """An ncu --csv launch list as one dict per launch, in launch order: the kernel name, "ns"
+    (gpu__time_duration.sum) and the dram__bytes_* counters in bytes, when captured."""
+    import csv
+    launches, hdr = {}, None
+    with open(path, newline="") as f:
+        for row in csv.reader(f):
+            if row and row[0] == "ID":
+                hdr = row
+                continue
+            if hdr is None or len(row) != len(hdr):
+                continue              # ncu's own messages before the table
+            d = dict(zip(hdr, row))
+            e = launches.setdefault(int(d["ID"]), {"name": d["Kernel Name"]})
+            v = float(d["Metric Value"].replace(",", "")) * _NCU_UNITS[d["Metric Unit"]]
+            if d["Metric Name"] == "gpu__time_duration.sum":
+                e["ns"] = v
+            elif d["Metric Name"].startswith("dram__bytes"):
+                e[d["Metric Name"]] = v
+    return [launches[k] for k in sorted(launches)]
+
+
+def write_traffic(csv_dir: str, out_path: str | None = None) -> dict:
+    """profiles/traffic.json from the launch lists DIR/<workload>.csv (one timed step of each
+    workload, captured as TRAFFIC_ABOUT says), tied to the current kernel sources."""
+    h = kernel_source_hash()
+    res = {"_about": TRAFFIC_ABOUT}
+    for name in sorted(WORKLOAD_TEXT):
+        path = os.path.join(csv_dir, name + ".csv")
+        if not os.path.exists(path):
+            continue
+        launches = read_ncu_launches(path)
+        kpc = kernels_per_call(name)
+        calls = len(launches) // kpc
+        if calls == 0:
+            raise ValueError(f"{path}: {len(launches)} launches, fewer than one call's {kpc}")
+        groups = [launches[c * kpc:(c + 1) * kpc] for c in range(calls)]
+        ent = {"calls": calls, "kernels_per_call": kpc,
+               "per_call_ns_under_ncu": [sum(k["ns"] for k in g) for g in groups],
+               "source_hash": h}
+        if all("dram__bytes_read.sum" in k and "dram__bytes_write.sum" in k for k in launches):
+            per_call = [int(sum(k["dram__bytes_read.sum"] + k["dram__bytes_write.sum"] for k in g))
+                        for g in groups]
+            ent["bytes_per_launch"] = int(sum(per_call) / calls)
+            ent["per_call_bytes"] = per_call
+        else:
+            ent["bytes_per_launch"] = None
+            ent["note"] = ("launch list only (gpu__time_duration.sum); DRAM bytes not captured "
+                           "at this size")
+        res.setdefault(roofline_kernel(name), {})[name] = ent
+    out_path = out_path or os.path.join(_ROOT, "profiles", "traffic.json")
+    with open(out_path, "w") as f:
+        json.dump(res, f, indent=1)
+        f.write("\n")
+    return res
+
+
 def load_peaks() -> dict:
     path = os.path.join(_ROOT, "MEASURED_PEAKS.json")
     try:
@@ -482,8 +568,7 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": f"HBM copy ({peaks['source']})"}
-    roof["kernel"] = ("nvfp4_encode_kernel + nvfp4_absmax_kernel" if wl.quantize else
-                      "lmhead_w4a16_nvfp4_kernel" if wl.nvfp4 else "lmhead_bf16_f32_kernel")
+    roof["kernel"] = roofline_kernel(name)
     roof["traffic"] = recorded_traffic(roof["kernel"], name)
     roof["algorithmic_bytes_per_launch"] = int(tot_bytes / calls_per_step)
     roof["source_hash"] = kernel_source_hash()
@@ -509,8 +594,7 @@ def measure(name: str, args, world: int, rank: int, peaks: dict, cpu_budget_s: f
         "e2e": e2e,
         "graph": graph,
         "torch_mm": torch_mm,
-        "gpu_launches": n_ev * (3 if wl.vocab_parallel else
-                                2 if (wl.quantize or wl.logprobs) else 1),
+        "gpu_launches": n_ev * kernels_per_call(name),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and cpu_budget_s > 0:
@@ -872,7 +956,19 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true",
                     help="measure only --workload (the default run adds every other workload)")
+    ap.add_argument("--traffic-from", metavar="DIR",
+                    help="write profiles/traffic.json from the ncu launch lists DIR/<workload>.csv "
+                         "and exit (no GPU needed)")
     args = ap.parse_args()
+    if args.traffic_from:
+        res = write_traffic(args.traffic_from)
+        for kern, ents in res.items():
+            if kern != "_about":
+                for name, e in ents.items():
+                    print(f"{name}: {kern}, {e['calls']} calls, bytes per call "
+                          f"{e['bytes_per_launch']}")
+        print("source_hash", kernel_source_hash())
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     line = run_reference(args) if args.impl == "reference" else run_ours(args)
