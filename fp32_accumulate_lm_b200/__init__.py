@@ -406,13 +406,14 @@ def logits_f32(hidden, W, alpha: float = 1.0, bias=None, out=None, stream=None,
     _check(hidden.is_contiguous() and W.is_contiguous(), "contiguous tensors required")
     rows, H = hidden.shape
     V = W.shape[0]
+    _check(W.device == hidden.device, "hidden and W must be on one device")
     if bias is not None:
         _check(bias.dtype == hidden.dtype and bias.is_cuda and bias.is_contiguous()
                and tuple(bias.shape) == (V,), "bias must be a contiguous [V] tensor of the dtype")
+        _check(bias.device == hidden.device, "bias must be on the inputs' device")
     if out is None:
         out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
     _check_out(out, torch.float32, (rows, V), hidden.device, "out")
-    _check(W.device == hidden.device, "hidden and W must be on one device")
     st = lmhead_logits_f32(hidden.data_ptr(), dt, rows, H, W.data_ptr(), V, float(alpha),
                            0 if bias is None else bias.data_ptr(), out.data_ptr(),
                            _stream_handle(stream))
@@ -434,11 +435,14 @@ def logprobs_f32(hidden, W, targets, alpha: float = 1.0, bias=None, workspace=No
            "contiguous CUDA tensors required")
     rows, H = hidden.shape
     V = W.shape[0]
+    _check(W.device == hidden.device, "hidden and W must be on one device")
     _check(targets.dtype == torch.int32 and targets.is_cuda and targets.is_contiguous()
            and tuple(targets.shape) == (rows,), "targets must be a contiguous int32 [rows] tensor")
+    _check(targets.device == hidden.device, "targets must be on the inputs' device")
     if bias is not None:
         _check(bias.dtype == hidden.dtype and bias.is_cuda and bias.is_contiguous()
                and tuple(bias.shape) == (V,), "bias must be a contiguous [V] tensor of the dtype")
+        _check(bias.device == hidden.device, "bias must be on the inputs' device")
     if out is None:
         lp = torch.empty((rows,), dtype=torch.float32, device=hidden.device)
         lse = torch.empty((rows,), dtype=torch.float32, device=hidden.device)
@@ -484,12 +488,15 @@ def logprobs_shard_stats_f32(hidden, W_shard, v_begin: int, targets, alpha: floa
            and W_shard.is_contiguous(), "contiguous CUDA tensors required")
     rows, H = hidden.shape
     V_shard = W_shard.shape[0]
+    _check(W_shard.device == hidden.device, "hidden and W_shard must be on one device")
     _check(targets.dtype == torch.int32 and targets.is_cuda and targets.is_contiguous()
            and tuple(targets.shape) == (rows,), "targets must be a contiguous int32 [rows] tensor")
+    _check(targets.device == hidden.device, "targets must be on the inputs' device")
     if bias_shard is not None:
         _check(bias_shard.dtype == hidden.dtype and bias_shard.is_cuda
                and bias_shard.is_contiguous() and tuple(bias_shard.shape) == (V_shard,),
                "bias_shard must be a contiguous [V_shard] tensor of the dtype")
+        _check(bias_shard.device == hidden.device, "bias_shard must be on the inputs' device")
     if out is None:
         out = torch.empty((rows, 3), dtype=torch.float32, device=hidden.device)
     _check_out(out, torch.float32, (rows, 3), hidden.device, "out (stats)")
@@ -579,10 +586,12 @@ def logits_vocab_slice_f32(hidden, W_slice, v_begin: int, outs, alpha: float = 1
            and W_slice.is_contiguous(), "contiguous CUDA tensors required")
     rows, H = hidden.shape
     V_slice = W_slice.shape[0]
+    _check(W_slice.device == hidden.device, "hidden and W_slice must be on one device")
     if bias_slice is not None:
         _check(bias_slice.dtype == hidden.dtype and bias_slice.is_cuda
                and bias_slice.is_contiguous() and tuple(bias_slice.shape) == (V_slice,),
                "bias_slice must be a contiguous [V_slice] tensor of the dtype")
+        _check(bias_slice.device == hidden.device, "bias_slice must be on the inputs' device")
     outs = list(outs)
     _check(1 <= len(outs) <= 8, "between 1 and 8 output buffers")
     ld = outs[0].shape[1] if outs[0].dim() == 2 else -1
